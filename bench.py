@@ -1,0 +1,456 @@
+"""Benchmark of one paged decode step on B200.
+
+A step is the whole hot path over one batch: [copy_blocks of the step's
+copy-on-write pairs, if the workload has any] -> reshape_and_cache of one new
+token per sequence -> paged_attn_decode over every cached token.  The default
+workload is the OPT-13B-shaped decode layer (64 sequences, 40 heads x 128,
+fp16, block size 16, context lengths U[1, 2048], 16k-block pool).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  ``value`` is algorithmic bytes per step
+(KV of valid tokens + q + out + table entries + lengths, plus the scatter's
+and the copies' bytes) divided by the device time per step, summed over
+ranks; inputs are resident in HBM and larger than L2.  ``e2e`` is the same
+metric with the step's inputs copied from pinned host memory and the output
+copied back inside the timed region.  ``--impl reference`` times the CPU
+oracle (float64) on the host's cores on a bounded sample of the same workload.
+Under torchrun each rank runs its own batch (weak scaling, no collective on
+the data path); the time is the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from paged_kv_cache_324_b200 import workload as wl  # noqa: E402
+
+METRIC = "paged decode attention KV GB/s and % of B200 HBM peak; sequences/sec"
+UNIT = "GB/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+# DRAM traffic of one paged_decode_kernel + reduce launch measured by ncu
+# (dram__bytes_read.sum + dram__bytes_write.sum), keyed by workload, valid only
+# for the decode kernel source it was measured on (sha256 prefix of decode.cu).
+NCU_TRAFFIC = {}
+
+
+def decode_source_sha() -> str:
+    p = os.path.join(ROOT, "paged_kv_cache_324_b200", "csrc", "decode.cu")
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+
+
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        v = float(json.load(open(p))["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only; no setting is changed)
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], 0
+        self._stop = threading.Event()
+        self.max_mhz = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.ok:
+            self.t.join()
+
+    def report(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# device-resident workload
+# ---------------------------------------------------------------------------
+
+class DeviceStep:
+    """A workload's pools and inputs on one GPU, and the calls of one step."""
+
+    def __init__(self, w: wl.DecodeWorkload, dev):
+        import torch
+        from paged_kv_cache_324_b200 import binding as B
+        self.w, self.dev, self.B, self.torch = w, dev, B, torch
+        self.stream = torch.cuda.current_stream(dev)
+        t16 = {"f16": torch.float16, "bf16": torch.bfloat16}
+
+        def up(bits, dtype):
+            if dtype == "e4m3":
+                return torch.from_numpy(np.ascontiguousarray(bits)).to(dev)
+            return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(t16[dtype])
+
+        self.up = up
+        self.k_pool = up(w.initial_pool("k"), w.kv_dtype)
+        self.v_pool = up(w.initial_pool("v"), w.kv_dtype)
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+        for op in w.setup:   # build the cache with the library's own kernels
+            if isinstance(op, wl.Scatter):
+                B.reshape_and_cache(up(op.k, w.src_dtype), up(op.v, w.src_dtype), self.k_pool, self.v_pool,
+                                    torch.from_numpy(op.slots).to(dev), float(w.k_scale), float(w.v_scale),
+                                    device_error=self.err)
+            else:
+                B.copy_blocks(self.k_pool, self.v_pool, torch.from_numpy(op.pairs).to(dev), device_error=self.err)
+        sc = w.step_scatter
+        self.host = {  # the step's inputs, as raw bits
+            "q": w.q, "k_new": sc.k, "v_new": sc.v, "slots": sc.slots, "tables": w.block_tables,
+            "lens": w.context_lens,
+        }
+        if w.step_copy is not None:
+            self.host["pairs"] = w.step_copy.pairs
+        self.d = {
+            "q": up(w.q, w.q_dtype), "k_new": up(sc.k, w.src_dtype), "v_new": up(sc.v, w.src_dtype),
+            "slots": torch.from_numpy(sc.slots).to(dev), "tables": torch.from_numpy(w.block_tables).to(dev),
+            "lens": torch.from_numpy(w.context_lens).to(dev),
+        }
+        if "pairs" in self.host:
+            self.d["pairs"] = torch.from_numpy(self.host["pairs"]).to(dev)
+        self.out = torch.empty_like(self.d["q"])
+        ws = B.decode_workspace_bytes(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.block_size,
+                                      w.max_context_len, 0)
+        self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
+        self.partition = B.decode_partition_size(w.num_seqs, w.num_kv_heads, w.block_size, w.max_context_len, 0)
+        self.split = w.max_context_len > self.partition
+        torch.cuda.synchronize(dev)
+        assert int(self.err.item()) == 0, "setup raised a device error"
+
+    def launches_per_step(self) -> int:
+        return ("pairs" in self.d) + 1 + 1 + int(self.split)
+
+    def copy_op(self):
+        if "pairs" in self.d:
+            self.B.copy_blocks(self.k_pool, self.v_pool, self.d["pairs"], device_error=self.err,
+                               stream=self.stream)
+
+    def scatter_op(self):
+        w = self.w
+        self.B.reshape_and_cache(self.d["k_new"], self.d["v_new"], self.k_pool, self.v_pool, self.d["slots"],
+                                 float(w.k_scale), float(w.v_scale), device_error=self.err, stream=self.stream)
+
+    def decode_op(self):
+        w = self.w
+        self.B.paged_attn_decode(self.out, self.d["q"], self.k_pool, self.v_pool, self.d["tables"],
+                                 self.d["lens"], float(w.scale), max_context_len=w.max_context_len,
+                                 k_scale=float(w.k_scale), v_scale=float(w.v_scale), workspace=self.ws,
+                                 device_error=self.err, stream=self.stream)
+
+    def step(self):
+        self.copy_op()
+        self.scatter_op()
+        self.decode_op()
+
+
+def barrier_sync(torch, dist_on):
+    if dist_on:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(torch, x: float, dist_on: bool) -> float:
+    if not dist_on:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(torch, x: float, dist_on: bool) -> float:
+    if not dist_on:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    dist_on = world > 1
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = wl.make(args.config)        # weak scaling: every rank runs a batch of the same shape
+    ds = DeviceStep(w, dev)
+    step_bytes = wl.step_algorithmic_bytes(w)
+    dec_bytes = wl.decode_algorithmic_bytes(w)
+
+    for _ in range(args.warmup):
+        ds.step()
+    barrier_sync(torch, dist_on)
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        barrier_sync(torch, dist_on)
+        start.record()
+        for i in range(K):
+            e = ev[i]
+            e[0].record()
+            ds.copy_op()
+            e[1].record()
+            ds.scatter_op()
+            e[2].record()
+            ds.decode_op()
+            e[3].record()
+        end.record()
+        barrier_sync(torch, dist_on)
+    ms_total = start.elapsed_time(end)
+    dec_ms = [ev[i][2].elapsed_time(ev[i][3]) for i in range(K)]
+    sc_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    cp_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
+    assert int(ds.err.item()) == 0, "device error during the timed region"
+    ms_total = max_over_ranks(torch, ms_total, dist_on)
+    ms_step = ms_total / K
+    total_bytes = sum_over_ranks(torch, float(step_bytes), dist_on)
+    value = total_bytes / (ms_step * 1e-3) / 1e9
+    seqs = sum_over_ranks(torch, float(w.num_seqs), dist_on)
+
+    # end to end: the step's inputs from pinned host memory, the output back to the host
+    def pin(a):
+        a = np.ascontiguousarray(a)
+        return torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).pin_memory()
+
+    pinned = {k: pin(v) for k, v in ds.host.items()}
+    dq = {k: (ds.d[k].view(torch.int16) if ds.d[k].dtype in (torch.float16, torch.bfloat16) else ds.d[k])
+          for k in pinned}
+    out_host = torch.empty(ds.out.shape, dtype=ds.out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step():
+        for k, v in pinned.items():
+            dq[k].copy_(v, non_blocking=True)
+        ds.step()
+        out_host.copy_(ds.out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    barrier_sync(torch, dist_on)
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record()
+    for _ in range(K):
+        e2e_step()
+    e2.record()
+    barrier_sync(torch, dist_on)
+    e2e_ms = max_over_ranks(torch, s2.elapsed_time(e2), dist_on) / K
+    e2e_value = total_bytes / (e2e_ms * 1e-3) / 1e9
+
+    peak, peak_kind = hbm_peak()
+    dec_avg = sum(dec_ms) / K
+    achieved = dec_bytes / (dec_avg * 1e-3) / 1e9
+    traffic = None
+    tr = NCU_TRAFFIC.get(args.config)
+    if tr and tr.get("kernel_sha") == decode_source_sha():
+        traffic = tr["bytes_per_launch"]
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": w.kv_dtype if w.kv_dtype != "e4m3" else "e4m3 (KV), f16 (q/out), f32 accumulate",
+        "data": "synthetic (seeded N(0,1) K/V/q; random-byte pool content in unwritten slots)",
+        "config": {
+            "workload": w.description, "name": w.name, "num_seqs": w.num_seqs, "num_heads": w.num_heads,
+            "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "block_size": w.block_size,
+            "num_blocks": w.num_blocks, "max_context_len": w.max_context_len,
+            "total_context_tokens": int(w.context_lens.sum()), "partition_size": ds.partition,
+            "step": ("copy_blocks + " if "pairs" in ds.d else "") + "reshape_and_cache + paged_attn_decode",
+            "step_bytes": step_bytes, "decode_bytes": dec_bytes,
+            "l2": "no flush: each step reads %.2f GB of KV, more than the 126 MB L2" % (dec_bytes / 1e9),
+            "parallelism": f"dp{world}" if world > 1 else "single GPU",
+        },
+        "sequences_per_s": round(seqs / (ms_step * 1e-3), 1),
+        "pct_of_hbm_peak": round(100 * value / world / peak, 2),
+        "pct_of_nominal_8tbs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
+        "kernel_ms": {"paged_attn_decode": round(dec_avg, 5), "reshape_and_cache": round(sum(sc_ms) / K, 5),
+                      "copy_blocks": round(sum(cp_ms) / K, 5) if "pairs" in ds.d else None},
+        "roofline": {"bound": "hbm", "kernel": "paged_decode_kernel + decode_reduce_kernel",
+                     "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "peak_kind": f"{peak_kind} (copy, burst)"},
+        "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "ms_per_step": round(e2e_ms, 5),
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": ds.launches_per_step() * K,
+        "clocks": clk.report(),
+    }
+    return line, w
+
+
+class OracleRunner:
+    """The float64 oracle on the host's cores, holding the workload's pools."""
+
+    def __init__(self, w: wl.DecodeWorkload):
+        import oracle
+        self.o, self.w = oracle, w
+        self.kp, self.vp = w.initial_pool("k"), w.initial_pool("v")
+        for op in w.setup:
+            if isinstance(op, wl.Scatter):
+                oracle.reshape_and_cache(op.k, op.v, w.src_dtype, self.kp, self.vp, w.kv_dtype, op.slots,
+                                         w.k_scale, w.v_scale)
+            else:
+                oracle.copy_blocks(self.kp, self.vp, op.pairs)
+        self.cores = os.cpu_count() or 1
+
+    def step(self, n=None) -> int:
+        """One step on the first n sequences (all by default); returns its algorithmic bytes."""
+        o, w = self.o, self.w
+        n = w.num_seqs if n is None else n
+        b = 0
+        if w.step_copy is not None:
+            o.copy_blocks(self.kp, self.vp, w.step_copy.pairs)
+            b += wl.copy_algorithmic_bytes(w, w.step_copy)
+        sc = w.step_scatter
+        o.reshape_and_cache(sc.k[:n], sc.v[:n], w.src_dtype, self.kp, self.vp, w.kv_dtype, sc.slots[:n],
+                            w.k_scale, w.v_scale)
+        o.paged_attn_decode(w.q[:n], w.q_dtype, self.kp, self.vp, w.kv_dtype, w.block_tables[:n],
+                            w.context_lens[:n], w.scale, w.k_scale, w.v_scale, threads=self.cores)
+        sub = wl.Scatter(sc.k[:n], sc.v[:n], sc.slots[:n])
+        lens = w.context_lens[:n].astype(np.int64)
+        b += wl.scatter_algorithmic_bytes(w, sub)
+        b += int(lens.sum()) * wl.kv_bytes_per_token(1, w.num_kv_heads, w.head_dim, wl.ELEM_BYTES[w.kv_dtype])
+        b += 2 * n * w.num_heads * w.head_dim * wl.ELEM_BYTES[w.q_dtype]
+        b += 4 * int(((lens + w.block_size - 1) // w.block_size).sum()) + 4 * n
+        return b
+
+
+def cpu_oracle_sample(w: wl.DecodeWorkload, budget_s: float):
+    """Whole steps of the workload on the oracle until the budget is spent (at least one)."""
+    r = OracleRunner(w)
+    n, nbytes, t0 = 0, 0, time.perf_counter()
+    while True:
+        nbytes += r.step()
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            return n, nbytes, el, r.cores
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", default="opt13b", choices=list(wl.NAMES))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        w = wl.make(args.config)
+        r = OracleRunner(w)
+        t0 = time.perf_counter()
+        r.step()                                          # calibration: one whole step, untimed
+        t_full = time.perf_counter() - t0
+        per_step_budget = min(30.0, 150.0 / (args.steps + args.warmup))
+        n = max(1, min(w.num_seqs, int(w.num_seqs * per_step_budget / max(t_full, 1e-9))))
+        rates, times = [], []
+        for i in range(args.warmup + args.steps):
+            t0 = time.perf_counter()
+            nbytes = r.step(n)
+            el = time.perf_counter() - t0
+            if i >= args.warmup:
+                rates.append(nbytes / el)
+                times.append(el)
+        value = sum(rates) / len(rates) / 1e9
+        ms = 1e3 * sum(times) / len(times)
+        sample = (f"first {n} of {w.num_seqs} sequences per step (scatter + float64 decode), "
+                  f"{len(times)} timed steps")
+        line = {"metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "impl": "reference",
+                "dtype": "f64", "data": "synthetic", "config": {"workload": w.description, "name": w.name},
+                "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": r.cores, "kind": "oracle",
+                                 "sample": sample},
+                "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    dist_on = world > 1
+    if dist_on:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        line, w = run_ours(args, rank, world, local_rank)
+        if rank == 0 and world == 1:
+            n, nbytes, el, cores = cpu_oracle_sample(w, args.cpu_budget)
+            v = nbytes / el / 1e9
+            line["cpu_baseline"] = {"value": round(v, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
+                                    "sample": f"{n} whole step(s) of the same workload (scatter + float64 decode "
+                                              f"of all {w.num_seqs} sequences), {el:.1f} s"}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if dist_on:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

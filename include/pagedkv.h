@@ -1,0 +1,172 @@
+/*
+ * pagedkv.h -- C ABI of the B200 (sm_100a) paged KV-cache decode library.
+ *
+ * The KV cache of every sequence is split into fixed-size blocks that sit
+ * anywhere in one shared physical pool and are reached through a
+ * per-sequence block table (Ultralytics glossary "PagedAttention", section
+ * "How paging works"; Wikipedia "PagedAttention", section "Description").
+ * The library provides the three GPU operations of a decode step:
+ *
+ *   pkv_reshape_and_cache  write the new tokens' K/V into the pool through a
+ *                          slot mapping (the glossary's worked example:
+ *                          pool[table[pos / B], pos % B] = key);
+ *   pkv_copy_blocks        block-granular copy-on-write of shared blocks
+ *                          (glossary, section "Sharing blocks across
+ *                          sequences"; "vLLM and PagedAttention" transcript:
+ *                          the partially filled shared block is copied);
+ *   pkv_paged_attn_decode  single-query causal attention over the paged pool
+ *                          (Wikipedia "PagedAttention", section "Mathematical
+ *                          formulation": o_i = sum_j V_j A_ij^T over the
+ *                          ceil(i/B) blocks of the sequence).
+ *
+ * Conventions shared by every entry point
+ *   - All pointers except scalars are DEVICE pointers, owned by the caller.
+ *     The library allocates nothing and keeps no per-call state; calls are
+ *     asynchronous on `stream` (a cudaStream_t passed as void*, NULL = the
+ *     legacy default stream) and nothing synchronises.
+ *   - Pools have layout [num_blocks][num_kv_heads][block_size][head_dim],
+ *     row-major, element type kv_dtype.  One (block, kv head) tile is one
+ *     contiguous run of block_size * head_dim elements.  K and V pools have
+ *     the same layout.  Pool base pointers must be 16-byte aligned.
+ *   - A "slot" is block_id * block_size + offset_in_block.
+ *   - Problems the host can see (null pointers, unsupported sizes or dtype
+ *     pairs, misaligned pointers, an undersized workspace) return a non-zero
+ *     status synchronously and launch nothing.  Launch failures return
+ *     PKV_ERR_CUDA.  Data-dependent problems are found on the device: the
+ *     offending item is skipped (attention writes NaN for the affected
+ *     sequence and head group) and a bit is OR-ed into *device_error (if
+ *     device_error is not NULL).  Kernels never trap; every wait inside a
+ *     kernel is bounded, and a wait that gives up sets PKV_DEVERR_TIMEOUT.
+ *     The caller reads *device_error after synchronising and clears it.
+ */
+#ifndef PAGEDKV_H
+#define PAGEDKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PKV_OK = 0,
+    PKV_ERR_INVALID_ARG = 1,   /* null pointer, negative size, inconsistent sizes */
+    PKV_ERR_UNSUPPORTED = 2,   /* valid but not implemented: head_dim, block_size, dtype pair, group size */
+    PKV_ERR_WORKSPACE = 3,     /* workspace missing or smaller than pkv_decode_workspace_bytes() */
+    PKV_ERR_CUDA = 4,          /* a CUDA runtime or driver call failed */
+    PKV_ERR_ALIGNMENT = 5      /* a pointer is not 16-byte aligned */
+} pkv_status;
+
+typedef enum {
+    PKV_F16 = 0,               /* IEEE binary16 */
+    PKV_BF16 = 1,              /* bfloat16 */
+    PKV_FP8_E4M3 = 2           /* OCP E4M3 (no infinities, max finite 448), with a per-tensor scale */
+} pkv_dtype;
+
+/* Bits OR-ed into *device_error. */
+#define PKV_DEVERR_BLOCK_ID    0x1u   /* a block-table entry read by attention is outside [0, num_blocks) */
+#define PKV_DEVERR_SLOT        0x2u   /* a slot >= num_blocks * block_size */
+#define PKV_DEVERR_PAIR        0x4u   /* a copy pair names a block outside [0, num_blocks) */
+#define PKV_DEVERR_CONTEXT_LEN 0x8u   /* context_len < 0, > max_blocks_per_seq * block_size, or > max_context_len */
+#define PKV_DEVERR_TIMEOUT     0x10u  /* a bounded wait inside a kernel gave up */
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int pkv_version(void);
+
+/* Human-readable text for a status code (static storage). */
+const char* pkv_status_string(pkv_status status);
+
+/*
+ * Workspace that pkv_paged_attn_decode needs for the split-context pass
+ * (per sequence, query head and partition: running max, sum and a head_dim
+ * output vector in float32).  Zero when every sequence fits one partition.
+ * partition_size as for pkv_paged_attn_decode (0 = automatic).  Returns 0
+ * for invalid arguments as well.
+ */
+size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                  int block_size, int max_context_len, int partition_size);
+
+/* The partition size (tokens) that pkv_paged_attn_decode uses for these
+ * arguments; equals max_context_len rounded up to block_size when no split
+ * happens.  Returns 0 for invalid arguments. */
+int pkv_decode_partition_size(int num_seqs, int num_kv_heads, int block_size,
+                              int max_context_len, int partition_size);
+
+/*
+ * Paged decode attention (Wikipedia "PagedAttention", section "Mathematical
+ * formulation"; FlashAttention-style tiling and GQA as in the glossary's
+ * section "Related methods").
+ *
+ * For each sequence s with L = context_lens[s] (the new token included, so
+ * its K/V must already be in the pool) and each query head h:
+ *   out[s][h][:] = sum_{t < L} softmax_t(scale * q[s][h] . k_t) * v_t,
+ *   k_t = K_pool[block_tables[s][t / block_size]][h / G][t % block_size][:],
+ *   G = num_heads / num_kv_heads (contiguous query-head groups share a KV head).
+ * For FP8 pools the stored values are multiplied by k_scale / v_scale.
+ * L = 0 gives a zero output.  Table entries at j >= ceil(L / block_size) are
+ * never read.  Physical blocks may be shared between and within sequences.
+ *
+ *   out            [num_seqs][num_heads][head_dim], q_dtype
+ *   q              [num_seqs][num_heads][head_dim], q_dtype in {F16, BF16}
+ *   k_pool/v_pool  see conventions; kv_dtype == q_dtype, or FP8_E4M3
+ *   block_tables   int32 [num_seqs][max_blocks_per_seq]
+ *   context_lens   int32 [num_seqs]
+ *   max_context_len  an upper bound of context_lens (sizes the grid)
+ *   head_dim in {64, 128} (128 only for FP8); block_size in {16, 32};
+ *   num_heads % num_kv_heads == 0 and G <= 16
+ *   partition_size 0 = automatic, else a multiple of block_size: sequences
+ *                  longer than it are split into partitions that run in
+ *                  parallel and are merged exactly by log-sum-exp
+ *   workspace      device buffer of at least pkv_decode_workspace_bytes()
+ *                  bytes (may be NULL when that is 0), 256-byte aligned
+ */
+pkv_status pkv_paged_attn_decode(void* out, const void* q, pkv_dtype q_dtype,
+                                 const void* k_pool, const void* v_pool, pkv_dtype kv_dtype,
+                                 float k_scale, float v_scale,
+                                 const int32_t* block_tables, int max_blocks_per_seq,
+                                 const int32_t* context_lens, int max_context_len,
+                                 int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                 int block_size, int num_blocks, float scale, int partition_size,
+                                 void* workspace, size_t workspace_bytes,
+                                 uint32_t* device_error, void* stream);
+
+/*
+ * Scatter new tokens into the pool (glossary "PagedAttention", section "How
+ * paging works").  For every token t with slot = slot_mapping[t] >= 0 and
+ * every KV head h:
+ *   k_pool[slot / block_size][h][slot % block_size][:] = k[t][h][:]  (same for v)
+ * copied bit for bit when kv_dtype == in_dtype; for an FP8_E4M3 pool each
+ * element is stored as e4m3(x / scale), the division in IEEE float32 and the
+ * conversion round-to-nearest-even saturating at +-448.  Negative slots are
+ * skipped.  Slots must be distinct (two tokens writing one slot race).
+ *
+ *   k, v           [num_tokens][num_kv_heads][head_dim], in_dtype in {F16, BF16}, 16-byte aligned
+ *   slot_mapping   int64 [num_tokens]
+ *   head_dim       a multiple of 8
+ */
+pkv_status pkv_reshape_and_cache(const void* k, const void* v, pkv_dtype in_dtype,
+                                 void* k_pool, void* v_pool, pkv_dtype kv_dtype,
+                                 float k_scale, float v_scale,
+                                 const int64_t* slot_mapping, int num_tokens,
+                                 int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                 uint32_t* device_error, void* stream);
+
+/*
+ * Block-granular copy-on-write (glossary "PagedAttention", section "Sharing
+ * blocks across sequences"): for every pair i,
+ *   k_pool[pairs[i][1]] := k_pool[pairs[i][0]] and the same for v_pool,
+ * block_bytes = num_kv_heads * block_size * head_dim * element size, a
+ * multiple of 16.  pairs is int64 [num_pairs][2] (src, dst) in device memory.
+ * Precondition (not checked): destinations are distinct and no destination
+ * is also a source, so the copies are independent.
+ */
+pkv_status pkv_copy_blocks(void* k_pool, void* v_pool, size_t block_bytes,
+                           const int64_t* pairs, int num_pairs, int num_blocks,
+                           uint32_t* device_error, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H */

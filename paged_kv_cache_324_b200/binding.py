@@ -1,0 +1,164 @@
+"""Thin Python binding over ``libpagedkv.so`` (C ABI in ``include/pagedkv.h``).
+
+Argument marshalling only: shapes, dtypes and pointers of torch tensors are
+read here and passed to the C entry points of the same names (without the
+``pkv_`` prefix); every step of the computation runs in the library's CUDA
+kernels.  There is no fallback: if the library is missing or a call fails,
+an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpagedkv.so")
+
+F16, BF16, FP8_E4M3 = 0, 1, 2
+DEVERR_BLOCK_ID, DEVERR_SLOT, DEVERR_PAIR, DEVERR_CONTEXT_LEN, DEVERR_TIMEOUT = 1, 2, 4, 8, 16
+
+_TORCH_CODES = {torch.float16: F16, torch.bfloat16: BF16, torch.uint8: FP8_E4M3,
+                torch.float8_e4m3fn: FP8_E4M3}
+
+
+class PagedKVError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded CUDA library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                               "`python -m paged_kv_cache_324_b200.build` (no CPU fallback exists)")
+        L = ctypes.CDLL(_LIB_PATH)
+        P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        L.pkv_version.restype = I
+        L.pkv_status_string.argtypes = [I]
+        L.pkv_status_string.restype = ctypes.c_char_p
+        L.pkv_decode_workspace_bytes.argtypes = [I, I, I, I, I, I, I]
+        L.pkv_decode_workspace_bytes.restype = Z
+        L.pkv_decode_partition_size.argtypes = [I, I, I, I, I]
+        L.pkv_decode_partition_size.restype = I
+        L.pkv_paged_attn_decode.argtypes = [P, P, I, P, P, I, F, F, P, I, P, I, I, I, I, I, I, I, F, I,
+                                            P, Z, P, P]
+        L.pkv_paged_attn_decode.restype = I
+        L.pkv_reshape_and_cache.argtypes = [P, P, I, P, P, I, F, F, P, I, I, I, I, I, P, P]
+        L.pkv_reshape_and_cache.restype = I
+        L.pkv_copy_blocks.argtypes = [P, P, Z, P, I, I, P, P]
+        L.pkv_copy_blocks.restype = I
+        _lib = L
+    return _lib
+
+
+def version() -> int:
+    return lib().pkv_version()
+
+
+def status_string(status: int) -> str:
+    return lib().pkv_status_string(status).decode()
+
+
+def _code(t: torch.Tensor) -> int:
+    try:
+        return _TORCH_CODES[t.dtype]
+    except KeyError:
+        raise TypeError(f"unsupported dtype {t.dtype}") from None
+
+
+def _dev(t: Optional[torch.Tensor], name: str):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise PagedKVError(status, what)
+
+
+def decode_partition_size(num_seqs, num_kv_heads, block_size, max_context_len, partition_size=0) -> int:
+    return lib().pkv_decode_partition_size(num_seqs, num_kv_heads, block_size, max_context_len, partition_size)
+
+
+def decode_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len,
+                           partition_size=0) -> int:
+    return lib().pkv_decode_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                            max_context_len, partition_size)
+
+
+def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
+                      block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float, *,
+                      max_context_len: int, k_scale: float = 1.0, v_scale: float = 1.0,
+                      partition_size: int = 0, workspace: Optional[torch.Tensor] = None,
+                      device_error: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """out[S, H, D] = decode attention of q[S, H, D] over pools [NB, Hkv, B, D].
+
+    block_tables int32 [S, max_blocks], context_lens int32 [S].  ``workspace``
+    (uint8, >= decode_workspace_bytes) is allocated with torch if not given.
+    """
+    S, H, D = q.shape
+    NB, Hkv, B, D2 = k_pool.shape
+    if out.shape != q.shape or out.dtype != q.dtype or D2 != D or v_pool.shape != k_pool.shape:
+        raise ValueError("inconsistent shapes or dtypes")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    need = decode_workspace_bytes(S, H, Hkv, D, B, max_context_len, partition_size)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    status = lib().pkv_paged_attn_decode(
+        _dev(out, "out"), _dev(q, "q"), _code(q), _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"),
+        _code(k_pool), float(k_scale), float(v_scale), _dev(block_tables, "block_tables"),
+        block_tables.shape[1], _dev(context_lens, "context_lens"), int(max_context_len), S, H, Hkv, D, B,
+        NB, float(scale), int(partition_size), _dev(workspace, "workspace"), ws_bytes,
+        _dev(device_error, "device_error"), _stream(stream))
+    _check(status, "paged_attn_decode")
+    return out
+
+
+def reshape_and_cache(k: torch.Tensor, v: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
+                      slot_mapping: torch.Tensor, k_scale: float = 1.0, v_scale: float = 1.0, *,
+                      device_error: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Write k, v [T, Hkv, D] into the pools [NB, Hkv, B, D] at slot_mapping (int64 [T])."""
+    T, Hkv, D = k.shape
+    NB, Hkv2, B, D2 = k_pool.shape
+    if (Hkv2, D2) != (Hkv, D) or v.shape != k.shape or v_pool.shape != k_pool.shape:
+        raise ValueError("inconsistent shapes")
+    if slot_mapping.dtype != torch.int64 or slot_mapping.numel() != T:
+        raise TypeError("slot_mapping must be int64 [T]")
+    status = lib().pkv_reshape_and_cache(
+        _dev(k, "k"), _dev(v, "v"), _code(k), _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"),
+        _code(k_pool), float(k_scale), float(v_scale), _dev(slot_mapping, "slot_mapping"), T, Hkv, D, B, NB,
+        _dev(device_error, "device_error"), _stream(stream))
+    _check(status, "reshape_and_cache")
+
+
+def copy_blocks(k_pool: torch.Tensor, v_pool: torch.Tensor, pairs: torch.Tensor, *,
+                device_error: Optional[torch.Tensor] = None, stream=None) -> None:
+    """k_pool[dst] := k_pool[src] (and v) for each row (src, dst) of pairs (int64 [n, 2])."""
+    if pairs.dtype != torch.int64 or (pairs.numel() and pairs.shape[-1] != 2):
+        raise TypeError("pairs must be int64 [n, 2]")
+    block_bytes = k_pool[0].numel() * k_pool.element_size()
+    status = lib().pkv_copy_blocks(
+        _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"), block_bytes, _dev(pairs, "pairs"),
+        pairs.numel() // 2, k_pool.shape[0], _dev(device_error, "device_error"), _stream(stream))
+    _check(status, "copy_blocks")

@@ -177,9 +177,12 @@ class DecodeWorkload:
         return int(np.prod(self.pool_shape)) * ELEM_BYTES[self.kv_dtype]
 
     def initial_pool(self, which: str) -> np.ndarray:
-        """Pool content before any write: uniform random bytes (seeded per pool)."""
+        """Pool content before any write: random bytes (seeded per pool; a 32 MiB random
+        chunk repeated, so that large pools are cheap to make).  Unwritten slots therefore
+        hold arbitrary bit patterns, NaN and Inf included."""
         rng = np.random.default_rng([self.seed, 1 if which == "k" else 2])
-        raw = garbage_bytes(rng, self.pool_bytes)
+        chunk = garbage_bytes(rng, min(self.pool_bytes, 32 << 20))
+        raw = np.resize(chunk, self.pool_bytes)
         dt = np.uint8 if self.kv_dtype == "e4m3" else np.uint16
         return raw.view(dt).reshape(self.pool_shape)
 

@@ -1,0 +1,90 @@
+"""Runs one workload's decode step on the GPU (through the binding) and on the
+oracle (on the host), from the same seeded inputs."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from paged_kv_cache_324_b200 import workload as wl
+
+TORCH16 = {"f16": torch.float16, "bf16": torch.bfloat16}
+
+
+def to_dev_bits(bits: np.ndarray, dtype: str, dev) -> torch.Tensor:
+    """Raw host bits -> device tensor of the named dtype (bit-identical)."""
+    if dtype == "e4m3":
+        return torch.from_numpy(np.ascontiguousarray(bits)).to(dev)
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev)
+    return t.view(TORCH16[dtype])
+
+
+def to_host_bits(t: torch.Tensor) -> np.ndarray:
+    if t.dtype == torch.uint8:
+        return t.cpu().numpy()
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def out_f64(t: torch.Tensor) -> np.ndarray:
+    return t.double().cpu().numpy()
+
+
+def gpu_step(w: wl.DecodeWorkload, partition_size: int = 0, dev="cuda:0", keep_pools=True,
+             block_tables=None, context_lens=None, max_context_len=None):
+    from paged_kv_cache_324_b200 import binding as B
+    dev = torch.device(dev)
+    kp = to_dev_bits(w.initial_pool("k"), w.kv_dtype, dev)
+    vp = to_dev_bits(w.initial_pool("v"), w.kv_dtype, dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def scatter(op):
+        B.reshape_and_cache(to_dev_bits(op.k, w.src_dtype, dev), to_dev_bits(op.v, w.src_dtype, dev),
+                            kp, vp, torch.from_numpy(op.slots).to(dev), float(w.k_scale), float(w.v_scale),
+                            device_error=err)
+
+    def copy(op):
+        B.copy_blocks(kp, vp, torch.from_numpy(op.pairs).to(dev), device_error=err)
+
+    for op in w.setup:
+        scatter(op) if isinstance(op, wl.Scatter) else copy(op)
+    if w.step_copy is not None:
+        copy(w.step_copy)
+    scatter(w.step_scatter)
+    q = to_dev_bits(w.q, w.q_dtype, dev)
+    out = torch.empty_like(q)
+    bt = w.block_tables if block_tables is None else block_tables
+    cl = w.context_lens if context_lens is None else context_lens
+    B.paged_attn_decode(out, q, kp, vp, torch.from_numpy(bt).to(dev), torch.from_numpy(cl).to(dev),
+                        float(w.scale), max_context_len=w.max_context_len if max_context_len is None else max_context_len,
+                        k_scale=float(w.k_scale), v_scale=float(w.v_scale),
+                        partition_size=partition_size, device_error=err)
+    torch.cuda.synchronize()
+    res = {"out": out_f64(out), "err": int(err.item())}
+    if keep_pools:
+        res["k_pool"], res["v_pool"] = to_host_bits(kp), to_host_bits(vp)
+    del kp, vp
+    return res
+
+
+def oracle_pools(w: wl.DecodeWorkload):
+    import oracle
+    kp, vp = w.initial_pool("k"), w.initial_pool("v")
+    for op in w.setup:
+        if isinstance(op, wl.Scatter):
+            oracle.reshape_and_cache(op.k, op.v, w.src_dtype, kp, vp, w.kv_dtype, op.slots, w.k_scale, w.v_scale)
+        else:
+            oracle.copy_blocks(kp, vp, op.pairs)
+    if w.step_copy is not None:
+        oracle.copy_blocks(kp, vp, w.step_copy.pairs)
+    sc = w.step_scatter
+    oracle.reshape_and_cache(sc.k, sc.v, w.src_dtype, kp, vp, w.kv_dtype, sc.slots, w.k_scale, w.v_scale)
+    return kp, vp
+
+
+def oracle_step(w: wl.DecodeWorkload, block_tables=None, context_lens=None):
+    import oracle
+    kp, vp = oracle_pools(w)
+    out = oracle.paged_attn_decode(w.q, w.q_dtype, kp, vp, w.kv_dtype,
+                                   w.block_tables if block_tables is None else block_tables,
+                                   w.context_lens if context_lens is None else context_lens,
+                                   w.scale, w.k_scale, w.v_scale)
+    return {"out": out, "k_pool": kp, "v_pool": vp}

@@ -1,0 +1,106 @@
+"""The C-ABI library: it builds for sm_100a, loads, exports every entry point
+declared in include/pagedkv.h, and rejects bad host-side arguments with the
+documented status codes before touching the GPU (no GPU needed here)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pagedkv.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from paged_kv_cache_324_b200 import binding, build
+    build.build()
+    return binding.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pkv_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for want in ("pkv_paged_attn_decode", "pkv_reshape_and_cache", "pkv_copy_blocks",
+                 "pkv_decode_workspace_bytes", "pkv_status_string", "pkv_version"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from paged_kv_cache_324_b200 import binding
+    out = subprocess.run(["nm", "-D", "--defined-only", binding._LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\bT (pkv_\w+)", out))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    for n in declared_functions():
+        assert hasattr(lib, n)
+
+
+def test_library_is_built_for_sm100a(lib):
+    from paged_kv_cache_324_b200 import binding
+    out = subprocess.run(["cuobjdump", "--list-elf", binding._LIB_PATH], capture_output=True, text=True).stdout
+    assert "sm_100a" in out
+
+
+def test_version_and_status_strings(lib):
+    from paged_kv_cache_324_b200 import binding
+    assert binding.version() >= 100
+    assert binding.status_string(0) == "ok"
+    assert "workspace" in binding.status_string(3)
+
+
+def _decode(lib, **over):
+    P = ctypes.c_void_p
+    args = dict(out=P(16), q=P(16), q_dtype=0, k_pool=P(16), v_pool=P(16), kv_dtype=0, k_scale=1.0,
+                v_scale=1.0, block_tables=P(16), max_blocks=4, context_lens=P(16), max_len=64, S=2, H=8,
+                Hkv=2, D=128, B=16, NB=10, scale=0.1, ps=0, ws=None, ws_bytes=0, err=None, stream=None)
+    args.update(over)
+    return lib.pkv_paged_attn_decode(*args.values())
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(H=0), 1), (dict(H=6, Hkv=4), 1), (dict(S=-1), 1), (dict(ps=24), 1),
+    (dict(B=8), 2), (dict(D=96), 2), (dict(H=34, Hkv=2), 2), (dict(q_dtype=0, kv_dtype=1), 2),
+    (dict(kv_dtype=2, D=64), 2), (dict(kv_dtype=2, k_scale=0.0), 1), (dict(q_dtype=2), 2),
+])
+def test_decode_rejects_bad_arguments(lib, over, status):
+    assert _decode(lib, **over) == status
+
+
+def test_decode_rejects_null_and_misaligned(lib):
+    assert _decode(lib, q=None) == 1
+    assert _decode(lib, out=ctypes.c_void_p(18)) == 5
+
+
+def test_reshape_and_copy_reject_bad_arguments(lib):
+    P = ctypes.c_void_p
+    assert lib.pkv_reshape_and_cache(P(16), P(16), 0, P(16), P(16), 1, 1.0, 1.0, P(16), 4, 2, 128, 16, 10,
+                                     None, None) == 2   # f16 in, bf16 pool
+    assert lib.pkv_reshape_and_cache(P(16), P(16), 0, P(16), P(16), 0, 1.0, 1.0, P(16), 4, 2, 100, 16, 10,
+                                     None, None) == 2   # head_dim not a multiple of 8
+    assert lib.pkv_reshape_and_cache(P(16), P(16), 0, P(16), P(16), 0, 1.0, 1.0, P(16), 0, 2, 128, 16, 10,
+                                     None, None) == 0   # nothing to do
+    assert lib.pkv_copy_blocks(P(16), P(16), 24, P(16), 3, 10, None, None) == 2
+    assert lib.pkv_copy_blocks(P(16), P(16), 32, P(16), -1, 10, None, None) == 1
+    assert lib.pkv_copy_blocks(P(16), P(16), 32, P(16), 0, 10, None, None) == 0
+
+
+def test_workspace_size_rules(lib):
+    from paged_kv_cache_324_b200 import binding as B
+    # fits one partition: no workspace
+    assert B.decode_workspace_bytes(64, 40, 40, 128, 16, 512, 1024) == 0
+    # 32768 tokens in 512-token partitions: 64 partitions of (128 floats + max + sum)
+    n = B.decode_workspace_bytes(16, 64, 8, 128, 16, 32768, 512)
+    rows = 16 * 64 * 64
+    assert n >= rows * (128 * 4 + 8)
+    assert B.decode_partition_size(16, 8, 16, 32768, 512) == 512
+    assert B.decode_partition_size(16, 8, 16, 300, 512) == 304    # one partition, rounded to the block
+    # automatic choice shrinks partitions when there are few work units, never below 4 blocks
+    assert B.decode_partition_size(4, 8, 16, 256, 0) == 64
