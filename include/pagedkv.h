@@ -132,6 +132,40 @@ pkv_status pkv_paged_attn_decode(void* out, const void* q, pkv_dtype q_dtype,
                                  uint32_t* device_error, void* stream);
 
 /*
+ * Size of the library-owned workspace used by pkv_paged_attn_decode_static_ws
+ * (64 MiB of device memory, held by every GPU that loads the library).
+ */
+#define PKV_STATIC_WORKSPACE_BYTES (64ull << 20)
+
+/*
+ * pkv_paged_attn_decode for callers that cannot allocate device memory.  The
+ * pages describe no such call; it exists for this library's users: code that
+ * runs inside a host framework owning every device allocation, or a serving
+ * loop that must not allocate once running (cudaMalloc may synchronise the
+ * device).  The caller still passes inputs and outputs; the split-context
+ * workspace is a file-scope device array of PKV_STATIC_WORKSPACE_BYTES inside
+ * the library, so this call allocates nothing.
+ *
+ * Arguments and results are those of pkv_paged_attn_decode, minus workspace.
+ * Returns PKV_ERR_WORKSPACE, launching nothing, when the call would need more
+ * than PKV_STATIC_WORKSPACE_BYTES (pkv_decode_workspace_bytes tells).  The
+ * first call on each device looks up the array's device address (with that
+ * device current); make that first call before any stream capture.  Every
+ * call shares the one array and leaves its contents behind (nothing in it
+ * needs to start at zero: each call writes every entry it reads), so calls
+ * that overlap on the GPU -- concurrent streams, or several host threads --
+ * race on it; serialise them.
+ */
+pkv_status pkv_paged_attn_decode_static_ws(void* out, const void* q, pkv_dtype q_dtype,
+                                           const void* k_pool, const void* v_pool, pkv_dtype kv_dtype,
+                                           float k_scale, float v_scale,
+                                           const int32_t* block_tables, int max_blocks_per_seq,
+                                           const int32_t* context_lens, int max_context_len,
+                                           int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                           int block_size, int num_blocks, float scale, int partition_size,
+                                           uint32_t* device_error, void* stream);
+
+/*
  * Scatter new tokens into the pool (glossary "PagedAttention", section "How
  * paging works").  For every token t with slot = slot_mapping[t] >= 0 and
  * every KV head h:

@@ -44,6 +44,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <mutex>
 
 #include "pkv_device.cuh"
 #include "pkv_host.h"
@@ -718,4 +719,66 @@ extern "C" pkv_status pkv_paged_attn_decode(void* out, const void* q, pkv_dtype 
                    : dispatch_bs<KV_E4M3, false, 128>(a, km, vm, st, hi);
     }
     return PKV_ERR_UNSUPPORTED;
+}
+
+// ---- decode with a library-owned workspace (no allocation by the caller) ------------
+//
+// For callers that cannot call cudaMalloc: code that runs where every device
+// allocation must go through someone else's allocator (a host framework that
+// owns the device memory budget), or a serving loop that must not allocate
+// after start-up because cudaMalloc can synchronise the device and stall.
+// The split-context workspace then lives in this file-scope device array,
+// which every GPU that loads the library holds until the process exits.
+// Host code cannot use the array's name as a device address (it names a
+// host-side stand-in), so each device's address is looked up once with
+// cudaGetSymbolAddress, with that device current, on the first call made on
+// that device; make that first call before any stream capture.
+
+namespace pkv {
+namespace {
+
+constexpr size_t kStaticWsBytes = 64ull << 20;   // PKV_STATIC_WORKSPACE_BYTES
+static __device__ __align__(256) uint8_t g_static_ws[kStaticWsBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_ws_mu;
+void* g_static_ws_ptr[kMaxDevices] = {};
+
+// Device address of g_static_ws on the current device (set up once per device).
+cudaError_t static_ws_address(void** ptr) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_static_ws_mu);
+    if (!g_static_ws_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_static_ws);
+        if (e != cudaSuccess) return e;
+        g_static_ws_ptr[dev] = p;
+    }
+    *ptr = g_static_ws_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace pkv
+
+static_assert(pkv::kStaticWsBytes == PKV_STATIC_WORKSPACE_BYTES, "header and library disagree");
+
+extern "C" pkv_status pkv_paged_attn_decode_static_ws(
+    void* out, const void* q, pkv_dtype q_dtype, const void* k_pool, const void* v_pool, pkv_dtype kv_dtype,
+    float k_scale, float v_scale, const int32_t* block_tables, int max_blocks_per_seq,
+    const int32_t* context_lens, int max_context_len, int num_seqs, int num_heads, int num_kv_heads,
+    int head_dim, int block_size, int num_blocks, float scale, int partition_size, uint32_t* device_error,
+    void* stream) {
+    const size_t need = pkv_decode_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                                   max_context_len, partition_size);
+    if (need > pkv::kStaticWsBytes) return PKV_ERR_WORKSPACE;
+    void* ws = nullptr;
+    if (need > 0 && pkv::static_ws_address(&ws) != cudaSuccess) return PKV_ERR_CUDA;
+    return pkv_paged_attn_decode(out, q, q_dtype, k_pool, v_pool, kv_dtype, k_scale, v_scale, block_tables,
+                                 max_blocks_per_seq, context_lens, max_context_len, num_seqs, num_heads,
+                                 num_kv_heads, head_dim, block_size, num_blocks, scale, partition_size, ws,
+                                 need > 0 ? pkv::kStaticWsBytes : 0, device_error, stream);
 }
