@@ -386,7 +386,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--config", default="opt13b", choices=list(wl.NAMES))
+    ap.add_argument("--config", default="opt13b", choices=list(wl.NAMES) + list(wl.COMPACT_NAMES))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     args = ap.parse_args()

@@ -308,7 +308,18 @@ def lognormal_lens(rng, n, median, sigma, cap):
 
 def make(name: str, small: bool = False) -> DecodeWorkload:
     """One of the named workloads; ``small`` shrinks batch and lengths for fast parity runs
-    while keeping head shapes, dtypes and the length distribution's shape."""
+    while keeping head shapes, dtypes and the length distribution's shape.  A name with the
+    suffix ``_compact`` is the same workload (same sequences, lengths and values) with the
+    pool cut down to the blocks in use plus 64, which keeps profiler captures small."""
+    if name.endswith("_compact"):
+        w = make(name[: -len("_compact")], small)
+        if w.name == "prefix":
+            raise KeyError(name)
+        nblk = int(((w.context_lens.astype(np.int64) + w.block_size - 1) // w.block_size).sum())
+        rng = np.random.default_rng(w.seed)
+        return independent_sequences(
+            name, w.seed, w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.block_size, nblk + 64,
+            w.q_dtype, w.kv_dtype, w.context_lens, w.description + f" (pool cut to {nblk + 64} blocks)")
     if name == "tiny":
         rng = np.random.default_rng(0)
         lens = rng.integers(1, 257, size=4)
@@ -351,6 +362,7 @@ def make(name: str, small: bool = False) -> DecodeWorkload:
 
 
 NAMES = ("tiny", "opt13b", "gqa", "prefix", "fp8", "fp8_b32")
+COMPACT_NAMES = tuple(n + "_compact" for n in NAMES if n != "prefix")
 
 
 # ---------------------------------------------------------------------------
