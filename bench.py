@@ -43,7 +43,10 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic of one paged_decode_kernel + reduce launch measured by ncu
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by workload, valid only
 # for the decode kernel source it was measured on (sha256 prefix of decode.cu).
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    "opt13b": {"bytes_per_launch": 1_319_549_000, "kernel_sha": "640cda3584e49b53",
+               "capture": "profiles/paged_decode_kernel_opt13b.md (opt13b_compact: same sequences)"},
+}
 
 
 def decode_source_sha() -> str:

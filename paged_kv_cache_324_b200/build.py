@@ -50,15 +50,18 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(f) <= t for f in _inputs())
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    if not force and up_to_date():
+def build(force: bool = False, verbose_ptxas: bool = False, out: str = None, defines=()) -> str:
+    """Compile and link; ``out`` and ``defines`` (NAME=VALUE macros) build a variant elsewhere."""
+    lib_path = out or LIB
+    if not force and out is None and not defines and up_to_date():
         return LIB
-    os.makedirs(BUILD_DIR, exist_ok=True)
+    obj_dir = BUILD_DIR if out is None else os.path.join(BUILD_DIR, "variant-" + str(abs(hash((out, tuple(defines))))))
+    os.makedirs(obj_dir, exist_ok=True)
     cc = nvcc()
-    extra = ["-Xptxas", "-v"] if verbose_ptxas else []
+    extra = (["-Xptxas", "-v"] if verbose_ptxas else []) + [f"-D{d}" for d in defines]
 
     def compile_one(src):
-        obj = os.path.join(BUILD_DIR, os.path.basename(src) + ".o")
+        obj = os.path.join(obj_dir, os.path.basename(src) + ".o")
         cmd = [cc, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
         res = subprocess.run(cmd, capture_output=True, text=True)
         if res.returncode != 0:
@@ -70,14 +73,14 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     if verbose_ptxas:
         for _, log in results:
             sys.stderr.write(log)
-    tmp = LIB + f".{os.getpid()}.tmp"
+    tmp = lib_path + f".{os.getpid()}.tmp"
     cmd = [cc, *ARCH, "-shared", "--cudart", "shared", "-o", tmp, *[o for o, _ in results],
            "-Xlinker", "-rpath,/usr/local/cuda/lib64"]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError(f"link failed:\n{res.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib_path)
+    return lib_path
 
 
 if __name__ == "__main__":

@@ -18,18 +18,21 @@
 //     land in shared memory with 128-byte swizzling, in a ring of stages
 //     guarded by transaction barriers (full: TMA bytes arrived; empty:
 //     consumer done), with evict-first L2 hints since the KV is streamed once.
-//   * Four consumer warps take blocks round-robin.  Each computes
-//     S = Q K^T for its block with mma.sync m16n8k16 (query heads as M,
-//     padded to 16; tokens as N; head_dim as K), an online softmax in
-//     registers (running max and sum, base-2 exponent), and O += P V with the
-//     P fragments taken straight from the S accumulators.  FP8 E4M3 tiles are
-//     widened to f16 (or bf16) in registers, two values per instruction, so
-//     the MMA sees exact values and no dequantised copy is written anywhere.
-//   * Operand fragments are read with 16-byte shared loads.  The head_dim
-//     axis of the QK contraction and the output-column axis of PV are
-//     permuted (the same permutation on both operands, undone on output) so
-//     that each thread's fragment comes from contiguous bytes, and with the
-//     swizzle every 8-lane phase touches 8 distinct bank groups.
+//   * Four consumer warps take ring stages round-robin (a stage is one block,
+//     or two when a block's K+V tiles are under 8 KB).  Each computes
+//     S^T = K Q^T with mma.sync m16n8k16 (16 tokens as M, the query heads of
+//     the group as N in tiles of 8, head_dim as K), an online softmax in
+//     registers per head (running max and sum, base-2 exponent, output
+//     rescaled only when a running max moved), and O^T += V^T P^T with the P^T
+//     fragments made from the S^T accumulators by movmatrix transposes.
+//   * 16-bit tiles are read with ldmatrix (K) and ldmatrix.trans (V^T) from
+//     the swizzled tile; every 8-lane phase touches 8 distinct bank groups.
+//     FP8 E4M3 tiles are read with 16-byte shared loads and widened to f16
+//     (or bf16) in registers, two values per instruction, so the MMA sees
+//     exact values and no dequantised copy is written anywhere; for them the
+//     head_dim axis of QK and of the output is permuted (the same permutation
+//     on both operands, undone on output) so that each lane's fragment comes
+//     from contiguous bytes.
 //   * The four warps' partial states are merged in shared memory; a CTA that
 //     covers its whole sequence writes the output, otherwise it writes
 //     (max, sum, normalised output) to the workspace and a second small
@@ -51,6 +54,13 @@
 
 namespace pkv {
 namespace {
+
+// Occupancy plan: the kernel streams HBM through TMA, so what keeps the memory
+// system busy is the number of consumer warps ready to drain the ring.  With
+// query groups of up to 8 heads a CTA fits in 96 registers per thread and a
+// 32 KB ring, so four CTAs share an SM; larger groups hold twice the
+// accumulators and run two CTAs with 64 KB rings.  PKV_RING_BYTES and
+// PKV_MIN_CTAS override the plan for every instance (used for tuning sweeps).
 
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
@@ -133,50 +143,96 @@ __device__ __forceinline__ uint32_t word(const uint4& v, int i) {
 
 // ---- tile geometry ---------------------------------------------------------------
 
-template <int KV, int D, int BS>
+template <int KV, int D, int BS, bool kHi>
 struct Geo {
     static constexpr int E = KV == KV_E4M3 ? 1 : 2;   // element bytes
     static constexpr int kNsub = D * E / 128;          // 128-byte sub-rows per token row
-    static constexpr int kSubBytes = BS * 128;         // one swizzled sub-tile
-    static constexpr int kTileBytes = kNsub * kSubBytes;
-    static constexpr int kStageBytes = 2 * kTileBytes; // K tile + V tile
-    static constexpr int kDpc = 16 / E;                // elements per 16-byte chunk
+    static constexpr int kSubBytes = BS * 128;         // one swizzled sub-tile (BS rows x 128 B)
+    static constexpr int kTileBytes = kNsub * kSubBytes;   // one (block, KV head) K or V tile
+    // blocks per ring stage: small tiles are paired so a stage moves at least 8 KB
+    static constexpr int kBps = 2 * kTileBytes >= 8192 ? 1 : 8192 / (2 * kTileBytes);
+    static constexpr int kStageTok = kBps * BS;        // tokens per stage
+    static constexpr int kStageBytes = 2 * kBps * kTileBytes;  // K tiles, then V tiles
     static constexpr int kKsteps = D / 16;             // k-steps of the QK contraction
-    static constexpr int kKpc = 4 / E;                 // QK k-steps served by one chunk
-    static constexpr int kNtS = BS / 8;                // score n-tiles per block
-    static constexpr int kKkPV = BS / 16;              // PV k-steps per block
-    static constexpr int kNtO = D / 8;                 // output n-tiles
-    static constexpr int kStages = (65536 / kStageBytes) < 4 ? 4 : ((65536 / kStageBytes) > 16 ? 16 : (65536 / kStageBytes));
+    static constexpr int kMtTok = kStageTok / 16;      // 16-token m-tiles per stage (QK M, PV K)
+    static constexpr int kMtDim = D / 16;              // 16-dim m-tiles of the output (PV M)
+#ifdef PKV_RING_BYTES
+    static constexpr int kRingTarget = PKV_RING_BYTES;
+#else
+    static constexpr int kRingTarget = kHi ? 65536 : 32768;
+#endif
+    static constexpr int kStagesRaw = kRingTarget / kStageBytes / kConsumerWarps * kConsumerWarps;
+    static constexpr int kStages = kStagesRaw < 4 ? 4 : (kStagesRaw > 32 ? 32 : kStagesRaw);
     static constexpr int kRingBytes = kStages * kStageBytes;
     static constexpr int kMergeBytes = kConsumerWarps * 16 * (D + 2) * 4;
     static constexpr int kDataBytes = kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes;
     static constexpr int kSmemBytes = 1024 /* alignment slack */ + kDataBytes + kStages * 16 + 16;
+    // CTAs per SM that the register budget must allow (shared memory permitting)
+    static constexpr int kSmemCtas = (227 * 1024) / (kSmemBytes + 1024);
+#ifdef PKV_MIN_CTAS
+    static constexpr int kMinCtas = PKV_MIN_CTAS;
+#else
+    static constexpr int kMinCtas = (kHi ? 2 : 4) < kSmemCtas ? (kHi ? 2 : 4) : kSmemCtas;
+#endif
     static_assert(D * E == 128 || D * E == 256, "row must be 128 or 256 bytes");
     static_assert(kStages % kConsumerWarps == 0, "stage -> warp mapping must be fixed");
+    static_assert(kStageTok % 16 == 0, "a stage holds whole 16-token m-tiles");
 
-    // First head_dim index of the 4 consecutive elements a thread with quad
-    // index c feeds into QK k-step ks (b0 covers base, base+1; b1 base+2, base+3).
-    __device__ static __forceinline__ int k_base(int c, int ks) {
-        const int qc = ks / kKpc, sub = qc >> 1, i = qc & 1;
-        const int w0 = (ks % kKpc) * E;                  // first 32-bit word of the k-step
-        return sub * (128 / E) + (2 * c + i) * kDpc + w0 * (4 / E);
+    // Byte offset, inside a stage, of 16-byte chunk q of token t's K row (V: add kVOff).
+    static constexpr int kVOff = kBps * kTileBytes;
+    __device__ static __forceinline__ uint32_t at(int t, int q) {
+        return static_cast<uint32_t>((t / BS) * kTileBytes + (q >> 3) * kSubBytes) + swz128(t % BS, q & 7);
     }
-    // head_dim index of output column `col` (0..7) of PV n-tile nt.
-    __device__ static __forceinline__ int o_dim(int nt, int col) {
-        const int sub = nt / kDpc, dd = nt % kDpc;
-        return sub * (128 / E) + col * kDpc + dd;
+    // QK contraction: head_dim index of b0's first element for quad lane c at k-step ks
+    // (b1 starts kQkB1 elements later).  16-bit tiles use the natural order (fragments
+    // come from ldmatrix); FP8 tiles use a permuted order in which each lane's four
+    // k-values of a k-step are four consecutive bytes of the row.
+    __device__ static __forceinline__ int qk_dim(int c, int ks) { return E == 2 ? ks * 16 + 2 * c : 32 * c + 4 * ks; }
+    static constexpr int kQkB1 = E == 2 ? 8 : 2;
+    // PV output: head_dim index held in row rr (0..15) of output m-tile md.
+    __device__ static __forceinline__ int o_dim(int md, int rr) {
+        return E == 2 ? md * 16 + rr : 16 * (rr & 7) + 2 * md + (rr >> 3);
     }
 };
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&a)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+                 : "r"(addr)
+                 : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&a)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+                 : "r"(addr)
+                 : "memory");
+}
+
+// Transpose of an 8x8 16-bit matrix held one row pair per lane (lane/4 = row).
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
+// Zero the 16-bit halves whose token is masked: lo half = token t, hi half = token t + 1.
+__device__ __forceinline__ uint32_t mask_pair(uint32_t x, int t, int valid) {
+    const uint32_t lo = t < valid ? 0x0000ffffu : 0u;
+    const uint32_t hi = t + 1 < valid ? 0xffff0000u : 0u;
+    return x & (lo | hi);
+}
 
 // ---- pass 1: one CTA per (partition, KV head, sequence) ------------------------------
 
 template <int KV, bool kQBf16, int D, int BS, bool kHi>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, (Geo<KV, D, BS, kHi>::kMinCtas))
 paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
                     const __grid_constant__ CUtensorMap vmap) {
-    using Gm = Geo<KV, D, BS>;
+    using Gm = Geo<KV, D, BS, kHi>;
     constexpr bool kBf16 = (KV == KV_BF16) || (KV == KV_E4M3 && kQBf16);
     constexpr int NST = Gm::kStages;
+    constexpr int NTH = kHi ? 2 : 1;   // 8-head n-tiles of the query group
 
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
@@ -210,6 +266,7 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
     const int tok_begin = part * PS;
     const int tok_end = min(L, tok_begin + PS);
     const int nblk = (tok_end - tok_begin + BS - 1) / BS;
+    const int nstage = (nblk + Gm::kBps - 1) / Gm::kBps;
     const int blk0 = tok_begin / BS;
 
     if (threadIdx.x == 0) {
@@ -223,11 +280,20 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
     }
     __syncthreads();
 
-    // per-warp softmax state (consumers); declared here so the merge can see it
-    float o[Gm::kNtO][4];
-    float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.f, l_hi = 0.f;
+    // Per-warp softmax state.  Lane (r = lane/4, c = lane%4) owns query heads
+    // nh*8 + 2c and nh*8 + 2c + 1 and, in the output, head_dim rows o_dim(md, r) and
+    // o_dim(md, r + 8) of every 16-dim m-tile md.
+    float o[Gm::kMtDim][NTH][4];
+    float m_run[NTH][2], l_run[NTH][2];
 #pragma unroll
-    for (int i = 0; i < Gm::kNtO; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    for (int md = 0; md < Gm::kMtDim; ++md)
+#pragma unroll
+        for (int nh = 0; nh < NTH; ++nh) o[md][nh][0] = o[md][nh][1] = o[md][nh][2] = o[md][nh][3] = 0.f;
+#pragma unroll
+    for (int nh = 0; nh < NTH; ++nh) {
+        m_run[nh][0] = m_run[nh][1] = -INFINITY;
+        l_run[nh][0] = l_run[nh][1] = 0.f;
+    }
 
     if (warp == kConsumerWarps) {
         // ================= producer warp =================
@@ -238,12 +304,13 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
         const uint64_t pol = l2_policy_evict_first();
         const int32_t* table = a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq + blk0;
         bool ok = true;
-        int issued = 0;
-        for (int j0 = 0; j0 < nblk && ok; j0 += 32) {
+        int issued = 0;   // stages issued
+        constexpr int kChunk = 32 / Gm::kBps * Gm::kBps;   // table entries per warp-wide load
+        for (int j0 = 0; j0 < nblk && ok; j0 += kChunk) {
             const int jj = j0 + lane;
             int pid = 0;
             bool bad = false;
-            if (jj < nblk) {
+            if (lane < kChunk && jj < nblk) {
                 pid = __ldg(table + jj);
                 bad = pid < 0 || pid >= a.num_blocks;
             }
@@ -252,24 +319,33 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
                 *s_abort = 1;
             }
             if (bad) pid = 0;   // load an in-range block; the output becomes NaN
-            const int cnt = min(32, nblk - j0);
-            for (int i = 0; i < cnt; ++i) {
-                const int j = j0 + i;
-                const int pj = __shfl_sync(0xffffffffu, pid, i);
-                const int stage = j % NST;
+            const int cnt = min(kChunk, nblk - j0);
+            for (int i = 0; i < cnt; i += Gm::kBps) {
+                const int js = (j0 + i) / Gm::kBps;   // stage index within the partition
+                int pj[Gm::kBps];
+#pragma unroll
+                for (int b = 0; b < Gm::kBps; ++b) pj[b] = __shfl_sync(0xffffffffu, pid, (i + b) & 31);
+                const int nb = min(Gm::kBps, cnt - i);
+                const int stage = js % NST;
                 if (lane == 0) {
-                    if (j >= NST && !mbar_wait(bar_empty + 8 * stage, ((j / NST) - 1) & 1)) ok = false;
+                    if (js >= NST && !mbar_wait(bar_empty + 8 * stage, ((js / NST) - 1) & 1)) ok = false;
                     if (ok) {
                         const uint32_t fb = bar_full + 8 * stage;
-                        const uint32_t kdst = base + stage * Gm::kStageBytes;
-                        const uint32_t vdst = kdst + Gm::kTileBytes;
-                        mbar_arrive_expect_tx(fb, Gm::kStageBytes);
+                        const uint32_t sbase = base + stage * Gm::kStageBytes;
+                        mbar_arrive_expect_tx(fb, 2 * nb * Gm::kTileBytes);
 #pragma unroll
-                        for (int sub = 0; sub < Gm::kNsub; ++sub) {
-                            tma_load_4d(kdst + sub * Gm::kSubBytes, &kmap, fb, sub * (128 / Gm::E), 0, kvh, pj, pol);
-                            tma_load_4d(vdst + sub * Gm::kSubBytes, &vmap, fb, sub * (128 / Gm::E), 0, kvh, pj, pol);
+                        for (int b = 0; b < Gm::kBps; ++b) {
+                            if (b < nb) {
+#pragma unroll
+                                for (int sub = 0; sub < Gm::kNsub; ++sub) {
+                                    const uint32_t off = b * Gm::kTileBytes + sub * Gm::kSubBytes;
+                                    tma_load_4d(sbase + off, &kmap, fb, sub * (128 / Gm::E), 0, kvh, pj[b], pol);
+                                    tma_load_4d(sbase + Gm::kVOff + off, &vmap, fb, sub * (128 / Gm::E), 0, kvh, pj[b],
+                                                pol);
+                                }
+                            }
                         }
-                        issued = j + 1;
+                        issued = js + 1;
                     }
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -292,26 +368,33 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
     } else {
         // ================= consumer warps =================
         const int r = lane >> 2, c = lane & 3;
-        const bool lo_ok = r < G, hi_ok = kHi && (r + 8) < G;
-        // Q fragments (A operand, rows = query heads of the group)
-        uint32_t qa[Gm::kKsteps][4];
-        {
-            const uint16_t* qbase = static_cast<const uint16_t*>(a.q) + out_row0 * D;
-            const uint32_t* qlo = reinterpret_cast<const uint32_t*>(qbase + static_cast<size_t>(lo_ok ? r : 0) * D);
-            const uint32_t* qhi = reinterpret_cast<const uint32_t*>(qbase + static_cast<size_t>(hi_ok ? r + 8 : 0) * D);
+        // Q^T fragments: B operand of S^T = K Q^T (k = head_dim, n = query head)
+        uint32_t qb[Gm::kKsteps][NTH][2];
+#pragma unroll
+        for (int nh = 0; nh < NTH; ++nh) {
+            const int hq = nh * 8 + r;
+            const bool ok = hq < G;
+            const uint32_t* qrow = reinterpret_cast<const uint32_t*>(static_cast<const uint16_t*>(a.q) +
+                                                                     (out_row0 + (ok ? hq : 0)) * D);
 #pragma unroll
             for (int ks = 0; ks < Gm::kKsteps; ++ks) {
-                const int b2 = Gm::k_base(c, ks) >> 1;
-                qa[ks][0] = lo_ok ? __ldg(qlo + b2) : 0u;
-                qa[ks][1] = hi_ok ? __ldg(qhi + b2) : 0u;
-                qa[ks][2] = lo_ok ? __ldg(qlo + b2 + 1) : 0u;
-                qa[ks][3] = hi_ok ? __ldg(qhi + b2 + 1) : 0u;
+                const int d0 = Gm::qk_dim(c, ks);
+                qb[ks][nh][0] = ok ? __ldg(qrow + (d0 >> 1)) : 0u;
+                qb[ks][nh][1] = ok ? __ldg(qrow + ((d0 + Gm::kQkB1) >> 1)) : 0u;
             }
         }
+        // per-lane ldmatrix row addresses (16-bit tiles): lane supplies row (lane & 7) of
+        // matrix lane >> 3; the swizzle XOR only depends on (lane & 7)
+        const int li = lane >> 3, l7 = lane & 7;
+        const int k_tok = (li & 1) * 8 + l7;           // K: matrices (t0-7,k0-7) (t8-15,k0-7) (t0-7,k8-15) (t8-15,k8-15)
+        const int k_hi = li >> 1;
+        const int v_tok = (li >> 1) * 8 + l7;          // V^T: (d0-7,t0-7) (d8-15,t0-7) (d0-7,t8-15) (d8-15,t8-15)
+        const int v_hi = li & 1;
         const float qk = a.qk_scale_log2;
-        for (int j = warp; j < nblk; j += kConsumerWarps) {
-            const int stage = j % NST;
-            const bool got = mbar_wait(bar_full + 8 * stage, (j / NST) & 1);
+
+        for (int js = warp; js < nstage; js += kConsumerWarps) {
+            const int stage = js % NST;
+            const bool got = mbar_wait(bar_full + 8 * stage, (js / NST) & 1);
             if (!__all_sync(0xffffffffu, got)) {
                 if (lane == 0) {
                     raise_error(a.err, PKV_DEVERR_TIMEOUT);
@@ -319,111 +402,138 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
                 }
                 break;
             }
-            const uint32_t kt = base + stage * Gm::kStageBytes;
-            const uint32_t vt = kt + Gm::kTileBytes;
-            const int valid = min(BS, tok_end - (tok_begin + j * BS));
+            const uint32_t sb = base + stage * Gm::kStageBytes;
+            const int valid = min(Gm::kStageTok, tok_end - (tok_begin + js * Gm::kStageTok));
 
-            // ---- S = Q K^T ----
-            float sc[Gm::kNtS][4];
+            // ---- S^T = K Q^T  (M = 16 tokens, N = 8 heads, K = head_dim) ----
+            float sc[Gm::kMtTok][NTH][4];
 #pragma unroll
-            for (int nt = 0; nt < Gm::kNtS; ++nt) {
-                sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
-                const int row = nt * 8 + r;
-                uint4 kw[2 * Gm::kNsub];
+            for (int mt = 0; mt < Gm::kMtTok; ++mt)
 #pragma unroll
-                for (int qc = 0; qc < 2 * Gm::kNsub; ++qc)
-                    kw[qc] = lds128(kt + (qc >> 1) * Gm::kSubBytes + swz128(row, 2 * c + (qc & 1)));
+                for (int nh = 0; nh < NTH; ++nh) sc[mt][nh][0] = sc[mt][nh][1] = sc[mt][nh][2] = sc[mt][nh][3] = 0.f;
+            if constexpr (Gm::E == 2) {
 #pragma unroll
                 for (int ks = 0; ks < Gm::kKsteps; ++ks) {
-                    const uint4& v = kw[ks / Gm::kKpc];
-                    uint32_t b0, b1;
-                    if constexpr (Gm::E == 2) {
-                        const int w0 = (ks % Gm::kKpc) * 2;
-                        b0 = word(v, w0);
-                        b1 = word(v, w0 + 1);
-                    } else {
-                        const uint32_t x = word(v, ks % Gm::kKpc);
-                        b0 = widen_e4m3x2<kBf16>(x);
-                        b1 = widen_e4m3x2<kBf16>(x >> 16);
+#pragma unroll
+                    for (int mt = 0; mt < Gm::kMtTok; ++mt) {
+                        uint32_t ka[4];
+                        ldsm_x4(ka, sb + Gm::at(mt * 16 + k_tok, 2 * ks + k_hi));
+#pragma unroll
+                        for (int nh = 0; nh < NTH; ++nh) mma16816<kBf16>(sc[mt][nh], ka, qb[ks][nh][0], qb[ks][nh][1]);
                     }
-                    mma16816<kBf16>(sc[nt], qa[ks], b0, b1);
+                }
+            } else {
+#pragma unroll
+                for (int mt = 0; mt < Gm::kMtTok; ++mt) {
+                    const int t0 = mt * 16 + r;
+                    const uint4 x0 = lds128(sb + Gm::at(t0, 2 * c)), x1 = lds128(sb + Gm::at(t0, 2 * c + 1));
+                    const uint4 y0 = lds128(sb + Gm::at(t0 + 8, 2 * c)), y1 = lds128(sb + Gm::at(t0 + 8, 2 * c + 1));
+#pragma unroll
+                    for (int ks = 0; ks < Gm::kKsteps; ++ks) {
+                        const uint32_t wr = word(ks < 4 ? x0 : x1, ks & 3);   // token r, 4 bytes
+                        const uint32_t wr8 = word(ks < 4 ? y0 : y1, ks & 3);  // token r + 8
+                        uint32_t ka[4];
+                        ka[0] = widen_e4m3x2<kBf16>(wr);
+                        ka[1] = widen_e4m3x2<kBf16>(wr8);
+                        ka[2] = widen_e4m3x2<kBf16>(wr >> 16);
+                        ka[3] = widen_e4m3x2<kBf16>(wr8 >> 16);
+#pragma unroll
+                        for (int nh = 0; nh < NTH; ++nh) mma16816<kBf16>(sc[mt][nh], ka, qb[ks][nh][0], qb[ks][nh][1]);
+                    }
                 }
             }
-            // ---- scale, mask, online softmax ----
-            float mx_lo = -INFINITY, mx_hi = -INFINITY;
+            // ---- scale, mask, online softmax over the stage's tokens, per head ----
 #pragma unroll
-            for (int nt = 0; nt < Gm::kNtS; ++nt) {
+            for (int mt = 0; mt < Gm::kMtTok; ++mt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int col = nt * 8 + 2 * c + (e & 1);
-                    const float x = sc[nt][e] * qk;
-                    sc[nt][e] = col < valid ? x : -INFINITY;
+                for (int nh = 0; nh < NTH; ++nh)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int t = mt * 16 + r + (e >> 1) * 8;
+                        const float x = sc[mt][nh][e] * qk;
+                        sc[mt][nh][e] = t < valid ? x : -INFINITY;
+                    }
+            float alpha[NTH][2];
+            bool rescale = false;
+#pragma unroll
+            for (int nh = 0; nh < NTH; ++nh)
+#pragma unroll
+                for (int hc = 0; hc < 2; ++hc) {
+                    float mx = -INFINITY;
+#pragma unroll
+                    for (int mt = 0; mt < Gm::kMtTok; ++mt) mx = fmaxf(mx, fmaxf(sc[mt][nh][hc], sc[mt][nh][hc + 2]));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                    const float mnew = fmaxf(m_run[nh][hc], mx);
+                    alpha[nh][hc] = exp2f(m_run[nh][hc] - mnew);
+                    rescale |= alpha[nh][hc] != 1.f;
+                    m_run[nh][hc] = mnew;
+                    float sum = 0.f;
+#pragma unroll
+                    for (int mt = 0; mt < Gm::kMtTok; ++mt) {
+                        sc[mt][nh][hc] = exp2f(sc[mt][nh][hc] - mnew);
+                        sc[mt][nh][hc + 2] = exp2f(sc[mt][nh][hc + 2] - mnew);
+                        sum += sc[mt][nh][hc] + sc[mt][nh][hc + 2];
+                    }
+                    l_run[nh][hc] = l_run[nh][hc] * alpha[nh][hc] + sum;
                 }
-                mx_lo = fmaxf(mx_lo, fmaxf(sc[nt][0], sc[nt][1]));
-                if constexpr (kHi) mx_hi = fmaxf(mx_hi, fmaxf(sc[nt][2], sc[nt][3]));
-            }
-            mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 1));
-            mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 2));
-            const float mnew_lo = fmaxf(m_lo, mx_lo);
-            const float alpha_lo = exp2f(m_lo - mnew_lo);
-            m_lo = mnew_lo;
-            float alpha_hi = 1.f;
-            if constexpr (kHi) {
-                mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 1));
-                mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 2));
-                const float mnew_hi = fmaxf(m_hi, mx_hi);
-                alpha_hi = exp2f(m_hi - mnew_hi);
-                m_hi = mnew_hi;
-            }
-            float sum_lo = 0.f, sum_hi = 0.f;
+            if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
-            for (int nt = 0; nt < Gm::kNtS; ++nt) {
-                sc[nt][0] = exp2f(sc[nt][0] - m_lo);
-                sc[nt][1] = exp2f(sc[nt][1] - m_lo);
-                sum_lo += sc[nt][0] + sc[nt][1];
-                if constexpr (kHi) {
-                    sc[nt][2] = exp2f(sc[nt][2] - m_hi);
-                    sc[nt][3] = exp2f(sc[nt][3] - m_hi);
-                    sum_hi += sc[nt][2] + sc[nt][3];
-                } else {
-                    sc[nt][2] = sc[nt][3] = 0.f;
+                for (int md = 0; md < Gm::kMtDim; ++md)
+#pragma unroll
+                    for (int nh = 0; nh < NTH; ++nh) {
+                        o[md][nh][0] *= alpha[nh][0];
+                        o[md][nh][1] *= alpha[nh][1];
+                        o[md][nh][2] *= alpha[nh][0];
+                        o[md][nh][3] *= alpha[nh][1];
+                    }
+            }
+            // ---- P^T fragments (B operand of O^T = V^T P^T): transpose S^T's 8x8 blocks ----
+            uint32_t pb[Gm::kMtTok][NTH][2], pl[Gm::kMtTok][NTH][2];
+#pragma unroll
+            for (int mt = 0; mt < Gm::kMtTok; ++mt)
+#pragma unroll
+                for (int nh = 0; nh < NTH; ++nh) {
+                    pb[mt][nh][0] = movmatrix_t(pack2<kBf16>(sc[mt][nh][0], sc[mt][nh][1]));
+                    pb[mt][nh][1] = movmatrix_t(pack2<kBf16>(sc[mt][nh][2], sc[mt][nh][3]));
+                    if constexpr (kBf16) {
+                        pl[mt][nh][0] = movmatrix_t(pack2<true>(bf16_residual(sc[mt][nh][0]), bf16_residual(sc[mt][nh][1])));
+                        pl[mt][nh][1] = movmatrix_t(pack2<true>(bf16_residual(sc[mt][nh][2]), bf16_residual(sc[mt][nh][3])));
+                    }
                 }
-            }
-            l_lo = l_lo * alpha_lo + sum_lo;
-            if constexpr (kHi) l_hi = l_hi * alpha_hi + sum_hi;
+            // ---- O^T += V^T P^T  (M = 16 head_dim rows, N = 8 heads, K = 16 tokens) ----
+            const bool partial = valid < Gm::kStageTok;
+            if constexpr (Gm::E == 2) {
 #pragma unroll
-            for (int nt = 0; nt < Gm::kNtO; ++nt) {
-                o[nt][0] *= alpha_lo;
-                o[nt][1] *= alpha_lo;
-                if constexpr (kHi) {
-                    o[nt][2] *= alpha_hi;
-                    o[nt][3] *= alpha_hi;
+                for (int mt = 0; mt < Gm::kMtTok; ++mt) {
+                    const int t0 = mt * 16 + 2 * c;   // tokens of this lane's A halves: t0, t0+1 / t0+8, t0+9
+#pragma unroll
+                    for (int md = 0; md < Gm::kMtDim; ++md) {
+                        uint32_t va[4];
+                        ldsm_x4_trans(va, sb + Gm::kVOff + Gm::at(mt * 16 + v_tok, 2 * md + v_hi));
+                        if (partial) {
+                            va[0] = mask_pair(va[0], t0, valid);
+                            va[1] = mask_pair(va[1], t0, valid);
+                            va[2] = mask_pair(va[2], t0 + 8, valid);
+                            va[3] = mask_pair(va[3], t0 + 8, valid);
+                        }
+#pragma unroll
+                        for (int nh = 0; nh < NTH; ++nh) {
+                            mma16816<kBf16>(o[md][nh], va, pb[mt][nh][0], pb[mt][nh][1]);
+                            if constexpr (kBf16) mma16816<kBf16>(o[md][nh], va, pl[mt][nh][0], pl[mt][nh][1]);
+                        }
+                    }
                 }
-            }
-            // ---- O += P V ----
+            } else {
 #pragma unroll
-            for (int kk = 0; kk < Gm::kKkPV; ++kk) {
-                uint32_t pa[4], pl[4];
-                pa[0] = pack2<kBf16>(sc[2 * kk][0], sc[2 * kk][1]);
-                pa[1] = pack2<kBf16>(sc[2 * kk][2], sc[2 * kk][3]);
-                pa[2] = pack2<kBf16>(sc[2 * kk + 1][0], sc[2 * kk + 1][1]);
-                pa[3] = pack2<kBf16>(sc[2 * kk + 1][2], sc[2 * kk + 1][3]);
-                if constexpr (kBf16) {
-                    pl[0] = pack2<true>(bf16_residual(sc[2 * kk][0]), bf16_residual(sc[2 * kk][1]));
-                    pl[1] = pack2<true>(bf16_residual(sc[2 * kk][2]), bf16_residual(sc[2 * kk][3]));
-                    pl[2] = pack2<true>(bf16_residual(sc[2 * kk + 1][0]), bf16_residual(sc[2 * kk + 1][1]));
-                    pl[3] = pack2<true>(bf16_residual(sc[2 * kk + 1][2]), bf16_residual(sc[2 * kk + 1][3]));
-                }
-                const int t0 = kk * 16 + 2 * c;     // this thread's four V rows: t0, t0+1, t0+8, t0+9
-                constexpr int kVsub = Gm::E == 2 ? Gm::kNsub : 1;
-#pragma unroll
-                for (int sub = 0; sub < kVsub; ++sub) {
-                    const uint32_t vs = vt + sub * Gm::kSubBytes;
-                    uint4 v0 = lds128(vs + swz128(t0, r));
-                    uint4 v1 = lds128(vs + swz128(t0 + 1, r));
-                    uint4 v2 = lds128(vs + swz128(t0 + 8, r));
-                    uint4 v3 = lds128(vs + swz128(t0 + 9, r));
-                    if (valid < BS) {
+                for (int mt = 0; mt < Gm::kMtTok; ++mt) {
+                    const int t0 = mt * 16 + 2 * c;
+                    uint4 v0 = lds128(sb + Gm::kVOff + Gm::at(t0, r));
+                    uint4 v1 = lds128(sb + Gm::kVOff + Gm::at(t0 + 1, r));
+                    uint4 v2 = lds128(sb + Gm::kVOff + Gm::at(t0 + 8, r));
+                    uint4 v3 = lds128(sb + Gm::kVOff + Gm::at(t0 + 9, r));
+                    if (partial) {
                         const uint4 z = make_uint4(0u, 0u, 0u, 0u);
                         if (t0 >= valid) v0 = z;
                         if (t0 + 1 >= valid) v1 = z;
@@ -433,27 +543,25 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
 #pragma unroll
                     for (int w = 0; w < 4; ++w) {
                         const uint32_t x0 = word(v0, w), x1 = word(v1, w), x2 = word(v2, w), x3 = word(v3, w);
-                        if constexpr (Gm::E == 2) {
+                        // (dim d, token pair) bytes: d = 16r + 4w + {0,1} in e, {2,3} in f
+                        const uint32_t e01 = __byte_perm(x0, x1, 0x5140u), e23 = __byte_perm(x2, x3, 0x5140u);
+                        const uint32_t f01 = __byte_perm(x0, x1, 0x7362u), f23 = __byte_perm(x2, x3, 0x7362u);
+                        uint32_t va[4], vb[4];
+                        va[0] = widen_e4m3x2<kBf16>(e01);
+                        va[1] = widen_e4m3x2<kBf16>(e01 >> 16);
+                        va[2] = widen_e4m3x2<kBf16>(e23);
+                        va[3] = widen_e4m3x2<kBf16>(e23 >> 16);
+                        vb[0] = widen_e4m3x2<kBf16>(f01);
+                        vb[1] = widen_e4m3x2<kBf16>(f01 >> 16);
+                        vb[2] = widen_e4m3x2<kBf16>(f23);
+                        vb[3] = widen_e4m3x2<kBf16>(f23 >> 16);
 #pragma unroll
-                            for (int h = 0; h < 2; ++h) {
-                                const uint32_t sel = h ? 0x7632u : 0x5410u;
-                                const uint32_t b0 = __byte_perm(x0, x1, sel);
-                                const uint32_t b1 = __byte_perm(x2, x3, sel);
-                                const int nt = sub * 8 + 2 * w + h;
-                                mma16816<kBf16>(o[nt], pa, b0, b1);
-                                if constexpr (kBf16) mma16816<kBf16>(o[nt], pl, b0, b1);
-                            }
-                        } else {
-                            const uint32_t e01 = __byte_perm(x0, x1, 0x5140u), e23 = __byte_perm(x2, x3, 0x5140u);
-                            const uint32_t f01 = __byte_perm(x0, x1, 0x7362u), f23 = __byte_perm(x2, x3, 0x7362u);
-                            const uint32_t bb[4][2] = {{e01, e23}, {e01 >> 16, e23 >> 16}, {f01, f23}, {f01 >> 16, f23 >> 16}};
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                const uint32_t b0 = widen_e4m3x2<kBf16>(bb[q][0]);
-                                const uint32_t b1 = widen_e4m3x2<kBf16>(bb[q][1]);
-                                const int nt = 4 * w + q;
-                                mma16816<kBf16>(o[nt], pa, b0, b1);
-                                if constexpr (kBf16) mma16816<kBf16>(o[nt], pl, b0, b1);
+                        for (int nh = 0; nh < NTH; ++nh) {
+                            mma16816<kBf16>(o[2 * w][nh], va, pb[mt][nh][0], pb[mt][nh][1]);
+                            mma16816<kBf16>(o[2 * w + 1][nh], vb, pb[mt][nh][0], pb[mt][nh][1]);
+                            if constexpr (kBf16) {
+                                mma16816<kBf16>(o[2 * w][nh], va, pl[mt][nh][0], pl[mt][nh][1]);
+                                mma16816<kBf16>(o[2 * w + 1][nh], vb, pl[mt][nh][0], pl[mt][nh][1]);
                             }
                         }
                     }
@@ -462,39 +570,45 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_empty + 8 * stage);
         }
-        // complete the row sums across the quad
-        l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 1);
-        l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 2);
-        if constexpr (kHi) {
-            l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 1);
-            l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 2);
-        }
+        // complete the per-head sums across the 8 lanes that share c
+#pragma unroll
+        for (int nh = 0; nh < NTH; ++nh)
+#pragma unroll
+            for (int hc = 0; hc < 2; ++hc) {
+                float v = l_run[nh][hc];
+                v += __shfl_xor_sync(0xffffffffu, v, 4);
+                v += __shfl_xor_sync(0xffffffffu, v, 8);
+                v += __shfl_xor_sync(0xffffffffu, v, 16);
+                l_run[nh][hc] = v;
+            }
     }
     __syncthreads();   // ring fully consumed: reuse it for the merge
 
-    float* sm_o = reinterpret_cast<float*>(gbase);                    // [warps][16][D]
+    float* sm_o = reinterpret_cast<float*>(gbase);                    // [warps][16 heads][D]
     float* sm_m = sm_o + kConsumerWarps * 16 * D;                      // [warps][16]
     float* sm_l = sm_m + kConsumerWarps * 16;                          // [warps][16]
     if (warp < kConsumerWarps) {
         const int r = lane >> 2, c = lane & 3;
         float* ow = sm_o + warp * 16 * D;
 #pragma unroll
-        for (int nt = 0; nt < Gm::kNtO; ++nt) {
-            const int d0 = Gm::o_dim(nt, 2 * c), d1 = Gm::o_dim(nt, 2 * c + 1);
-            ow[r * D + d0] = o[nt][0];
-            ow[r * D + d1] = o[nt][1];
-            if constexpr (kHi) {
-                ow[(r + 8) * D + d0] = o[nt][2];
-                ow[(r + 8) * D + d1] = o[nt][3];
+        for (int md = 0; md < Gm::kMtDim; ++md)
+#pragma unroll
+            for (int nh = 0; nh < NTH; ++nh) {
+                const int h0 = nh * 8 + 2 * c;
+                const int d0 = Gm::o_dim(md, r), d1 = Gm::o_dim(md, r + 8);
+                ow[h0 * D + d0] = o[md][nh][0];
+                ow[(h0 + 1) * D + d0] = o[md][nh][1];
+                ow[h0 * D + d1] = o[md][nh][2];
+                ow[(h0 + 1) * D + d1] = o[md][nh][3];
             }
-        }
-        if (c == 0) {
-            sm_m[warp * 16 + r] = m_lo;
-            sm_l[warp * 16 + r] = l_lo;
-            if constexpr (kHi) {
-                sm_m[warp * 16 + r + 8] = m_hi;
-                sm_l[warp * 16 + r + 8] = l_hi;
-            }
+        if (r == 0) {
+#pragma unroll
+            for (int nh = 0; nh < NTH; ++nh)
+#pragma unroll
+                for (int hc = 0; hc < 2; ++hc) {
+                    sm_m[warp * 16 + nh * 8 + 2 * c + hc] = m_run[nh][hc];
+                    sm_l[warp * 16 + nh * 8 + 2 * c + hc] = l_run[nh][hc];
+                }
         }
     }
     __syncthreads();
@@ -589,7 +703,7 @@ bool encode_pool_map(CUtensorMap* map, const void* pool, int kv_dtype, int head_
 template <int KV, bool kQBf16, int D, int BS, bool kHi>
 pkv_status launch_decode(const DecodeArgs& a, const CUtensorMap& km, const CUtensorMap& vm,
                          cudaStream_t st) {
-    using Gm = Geo<KV, D, BS>;
+    using Gm = Geo<KV, D, BS, kHi>;
     auto kern = paged_decode_kernel<KV, kQBf16, D, BS, kHi>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Gm::kSmemBytes) != cudaSuccess)
         return PKV_ERR_CUDA;
