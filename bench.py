@@ -125,7 +125,7 @@ class ClockSampler:
 class DeviceStep:
     """A workload's pools and inputs on one GPU, and the calls of one step."""
 
-    def __init__(self, w: wl.DecodeWorkload, dev):
+    def __init__(self, w: wl.DecodeWorkload, dev, partition_size: int = 0):
         import torch
         from paged_kv_cache_324_b200 import binding as B
         self.w, self.dev, self.B, self.torch = w, dev, B, torch
@@ -163,10 +163,12 @@ class DeviceStep:
         if "pairs" in self.host:
             self.d["pairs"] = torch.from_numpy(self.host["pairs"]).to(dev)
         self.out = torch.empty_like(self.d["q"])
-        ws = B.decode_workspace_bytes(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.block_size,
-                                      w.max_context_len, 0)
+        ws = B.decode_workspace_bytes(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.kv_dtype,
+                                      w.block_size, w.max_context_len, partition_size)
         self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
-        self.partition = B.decode_partition_size(w.num_seqs, w.num_kv_heads, w.block_size, w.max_context_len, 0)
+        self.partition_arg = partition_size
+        self.partition = B.decode_partition_size(w.num_seqs, w.num_kv_heads, w.head_dim, w.kv_dtype, w.block_size,
+                                                 w.max_context_len, partition_size)
         self.split = w.max_context_len > self.partition
         torch.cuda.synchronize(dev)
         assert int(self.err.item()) == 0, "setup raised a device error"
@@ -189,7 +191,7 @@ class DeviceStep:
         self.B.paged_attn_decode(self.out, self.d["q"], self.k_pool, self.v_pool, self.d["tables"],
                                  self.d["lens"], float(w.scale), max_context_len=w.max_context_len,
                                  k_scale=float(w.k_scale), v_scale=float(w.v_scale), workspace=self.ws,
-                                 device_error=self.err, stream=self.stream)
+                                 partition_size=self.partition_arg, device_error=self.err, stream=self.stream)
 
     def step(self):
         self.copy_op()
@@ -228,7 +230,8 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = wl.make(args.config)        # weak scaling: every rank runs a batch of the same shape
-    ds = DeviceStep(w, dev)
+    ps = w.partition_size if args.partition == "config" else (0 if args.partition == "auto" else int(args.partition))
+    ds = DeviceStep(w, dev, ps)
     step_bytes = wl.step_algorithmic_bytes(w)
     dec_bytes = wl.decode_algorithmic_bytes(w)
 
@@ -313,6 +316,7 @@ def run_ours(args, rank, world, local_rank):
             "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "block_size": w.block_size,
             "num_blocks": w.num_blocks, "max_context_len": w.max_context_len,
             "total_context_tokens": int(w.context_lens.sum()), "partition_size": ds.partition,
+            "partition_rule": "automatic" if ds.partition_arg == 0 else "set by the workload or --partition",
             "step": ("copy_blocks + " if "pairs" in ds.d else "") + "reshape_and_cache + paged_attn_decode",
             "step_bytes": step_bytes, "decode_bytes": dec_bytes,
             "l2": "no flush: each step reads %.2f GB of KV, more than the 126 MB L2" % (dec_bytes / 1e9),
@@ -391,6 +395,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--config", default="opt13b", choices=list(wl.NAMES) + list(wl.COMPACT_NAMES))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--partition", default="config",
+                    help="'config' (the workload's stated partition size, else automatic), 'auto', or tokens")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     args = ap.parse_args()
     if args.warmup < 3:

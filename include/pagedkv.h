@@ -85,13 +85,17 @@ const char* pkv_status_string(pkv_status status);
  * for invalid arguments as well.
  */
 size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
-                                  int block_size, int max_context_len, int partition_size);
+                                  pkv_dtype kv_dtype, int block_size, int max_context_len,
+                                  int partition_size);
 
 /* The partition size (tokens) that pkv_paged_attn_decode uses for these
  * arguments; equals max_context_len rounded up to block_size when no split
- * happens.  Returns 0 for invalid arguments. */
-int pkv_decode_partition_size(int num_seqs, int num_kv_heads, int block_size,
-                              int max_context_len, int partition_size);
+ * happens.  The automatic choice (partition_size 0) aims at about 512 KB of
+ * K+V per partition and KV head (1,024 tokens of 16-bit head_dim 128, 2,048 of
+ * FP8), shrunk while there are fewer than two work units per SM.  Returns 0
+ * for invalid arguments. */
+int pkv_decode_partition_size(int num_seqs, int num_kv_heads, int head_dim, pkv_dtype kv_dtype,
+                              int block_size, int max_context_len, int partition_size);
 
 /*
  * Paged decode attention (Wikipedia "PagedAttention", section "Mathematical

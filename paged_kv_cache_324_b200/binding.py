@@ -44,9 +44,9 @@ def lib() -> ctypes.CDLL:
         L.pkv_version.restype = I
         L.pkv_status_string.argtypes = [I]
         L.pkv_status_string.restype = ctypes.c_char_p
-        L.pkv_decode_workspace_bytes.argtypes = [I, I, I, I, I, I, I]
+        L.pkv_decode_workspace_bytes.argtypes = [I, I, I, I, I, I, I, I]
         L.pkv_decode_workspace_bytes.restype = Z
-        L.pkv_decode_partition_size.argtypes = [I, I, I, I, I]
+        L.pkv_decode_partition_size.argtypes = [I, I, I, I, I, I, I]
         L.pkv_decode_partition_size.restype = I
         L.pkv_paged_attn_decode.argtypes = [P, P, I, P, P, I, F, F, P, I, P, I, I, I, I, I, I, I, F, I,
                                             P, Z, P, P]
@@ -95,14 +95,26 @@ def _check(status: int, what: str):
         raise PagedKVError(status, what)
 
 
-def decode_partition_size(num_seqs, num_kv_heads, block_size, max_context_len, partition_size=0) -> int:
-    return lib().pkv_decode_partition_size(num_seqs, num_kv_heads, block_size, max_context_len, partition_size)
+_CODES_BY_NAME = {"f16": F16, "bf16": BF16, "e4m3": FP8_E4M3}
 
 
-def decode_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len,
+def _kv_code(kv_dtype) -> int:
+    if isinstance(kv_dtype, torch.dtype):
+        return _TORCH_CODES[kv_dtype]
+    return _CODES_BY_NAME[kv_dtype] if isinstance(kv_dtype, str) else int(kv_dtype)
+
+
+def decode_partition_size(num_seqs, num_kv_heads, head_dim, kv_dtype, block_size, max_context_len,
+                          partition_size=0) -> int:
+    """Partition size the decode call uses; kv_dtype as a torch dtype, 'f16'/'bf16'/'e4m3' or a code."""
+    return lib().pkv_decode_partition_size(num_seqs, num_kv_heads, head_dim, _kv_code(kv_dtype), block_size,
+                                           max_context_len, partition_size)
+
+
+def decode_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, kv_dtype, block_size, max_context_len,
                            partition_size=0) -> int:
-    return lib().pkv_decode_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
-                                            max_context_len, partition_size)
+    return lib().pkv_decode_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, _kv_code(kv_dtype),
+                                            block_size, max_context_len, partition_size)
 
 
 def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
@@ -121,7 +133,7 @@ def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_pool: torch.Tensor, 
         raise ValueError("inconsistent shapes or dtypes")
     if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
         raise TypeError("block_tables and context_lens must be int32")
-    need = decode_workspace_bytes(S, H, Hkv, D, B, max_context_len, partition_size)
+    need = decode_workspace_bytes(S, H, Hkv, D, k_pool.dtype, B, max_context_len, partition_size)
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0

@@ -157,7 +157,7 @@ class DecodeWorkload:
     setup: list                  # Scatter / Copy operations that build the cache
     step_copy: Optional[Copy]    # block copies inside the step (None = none)
     step_scatter: Scatter        # the step's appended tokens (one per sequence)
-    partition_size: int = 512
+    partition_size: int = 0      # split-context partition (tokens) the workload states; 0 = automatic
     description: str = ""
 
     @property
@@ -192,7 +192,7 @@ def _new_values(rng, tokens, hkv, d, dtype):
 
 
 def _finish(name, seed, rng, S, H, Hkv, D, B, NB, q_dtype, kv_dtype, lens, tables,
-            setup, step_copy, new_slots, description, partition_size=512):
+            setup, step_copy, new_slots, description, partition_size=0):
     src_dtype = q_dtype if kv_dtype != "e4m3" else "f16"
     q = normal_bits(rng, (S, H, D), q_dtype)
     nk, nv = _new_values(rng, len(new_slots), Hkv, D, src_dtype)
@@ -214,7 +214,7 @@ def _finish(name, seed, rng, S, H, Hkv, D, B, NB, q_dtype, kv_dtype, lens, table
 
 
 def independent_sequences(name, seed, S, H, Hkv, D, B, NB, q_dtype, kv_dtype, lens,
-                          description="", partition_size=512) -> DecodeWorkload:
+                          description="", partition_size=0) -> DecodeWorkload:
     """Sequences with private blocks; the step appends token L_s - 1 of each sequence.
 
     Blocks come from a seeded shuffle of range(NB) popped from the front.
@@ -240,7 +240,7 @@ def independent_sequences(name, seed, S, H, Hkv, D, B, NB, q_dtype, kv_dtype, le
 
 def shared_prefix_sampling(name, seed, prompts, samples, H, Hkv, D, B, NB, dtype,
                            prefix_blocks, tail_max, description="",
-                           partition_size=512) -> DecodeWorkload:
+                           partition_size=0) -> DecodeWorkload:
     """Parallel sampling: ``samples`` sequences per prompt share the prompt's blocks.
 
     Prompt p has ``prefix_blocks * B + r_p`` tokens, r_p ~ U{1..B-1}, so its
@@ -319,7 +319,8 @@ def make(name: str, small: bool = False) -> DecodeWorkload:
         rng = np.random.default_rng(w.seed)
         return independent_sequences(
             name, w.seed, w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.block_size, nblk + 64,
-            w.q_dtype, w.kv_dtype, w.context_lens, w.description + f" (pool cut to {nblk + 64} blocks)")
+            w.q_dtype, w.kv_dtype, w.context_lens, w.description + f" (pool cut to {nblk + 64} blocks)",
+            partition_size=w.partition_size)
     if name == "tiny":
         rng = np.random.default_rng(0)
         lens = rng.integers(1, 257, size=4)
@@ -357,7 +358,7 @@ def make(name: str, small: bool = False) -> DecodeWorkload:
         return independent_sequences(
             name, 4, S, 64, 8, 128, B, NB, "f16", "e4m3", np.full(S, L),
             f"long-context FP8: batch {S}, L={L}, 64 q / 8 KV heads, head_dim 128, "
-            f"q fp16, K/V e4m3 per-tensor scale, B={B}, 512-token partitions")
+            f"q fp16, K/V e4m3 per-tensor scale, B={B}, 512-token partitions", partition_size=512)
     raise KeyError(name)
 
 

@@ -28,10 +28,12 @@ def out_f64(t: torch.Tensor) -> np.ndarray:
     return t.double().cpu().numpy()
 
 
-def gpu_step(w: wl.DecodeWorkload, partition_size: int = 0, dev="cuda:0", keep_pools=True,
+def gpu_step(w: wl.DecodeWorkload, partition_size=None, dev="cuda:0", keep_pools=True,
              block_tables=None, context_lens=None, max_context_len=None):
     from paged_kv_cache_324_b200 import binding as B
     dev = torch.device(dev)
+    if partition_size is None:
+        partition_size = w.partition_size
     kp = to_dev_bits(w.initial_pool("k"), w.kv_dtype, dev)
     vp = to_dev_bits(w.initial_pool("v"), w.kv_dtype, dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)

@@ -95,12 +95,15 @@ def test_reshape_and_copy_reject_bad_arguments(lib):
 def test_workspace_size_rules(lib):
     from paged_kv_cache_324_b200 import binding as B
     # fits one partition: no workspace
-    assert B.decode_workspace_bytes(64, 40, 40, 128, 16, 512, 1024) == 0
+    assert B.decode_workspace_bytes(64, 40, 40, 128, "f16", 16, 512, 1024) == 0
     # 32768 tokens in 512-token partitions: 64 partitions of (128 floats + max + sum)
-    n = B.decode_workspace_bytes(16, 64, 8, 128, 16, 32768, 512)
+    n = B.decode_workspace_bytes(16, 64, 8, 128, "e4m3", 16, 32768, 512)
     rows = 16 * 64 * 64
     assert n >= rows * (128 * 4 + 8)
-    assert B.decode_partition_size(16, 8, 16, 32768, 512) == 512
-    assert B.decode_partition_size(16, 8, 16, 300, 512) == 304    # one partition, rounded to the block
-    # automatic choice shrinks partitions when there are few work units, never below 4 blocks
-    assert B.decode_partition_size(4, 8, 16, 256, 0) == 64
+    assert B.decode_partition_size(16, 8, 128, "e4m3", 16, 32768, 512) == 512
+    assert B.decode_partition_size(16, 8, 128, "f16", 16, 300, 512) == 304    # one partition, rounded to the block
+    # automatic choice: ~512 KB of K+V per partition and KV head
+    assert B.decode_partition_size(256, 8, 128, "bf16", 16, 4096, 0) == 1024
+    assert B.decode_partition_size(16, 8, 128, "e4m3", 16, 32768, 0) == 2048
+    # ... shrunk when there are few work units, never below 4 blocks
+    assert B.decode_partition_size(4, 8, 64, "f16", 16, 256, 0) == 64

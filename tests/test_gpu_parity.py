@@ -14,7 +14,7 @@ from tests.parity import attention_close
 pytestmark = pytest.mark.gpu
 
 
-def check_step(w, partition_size=0, pools=True):
+def check_step(w, partition_size=None, pools=True):
     g = H.gpu_step(w, partition_size=partition_size, keep_pools=pools)
     o = H.oracle_step(w)
     assert g["err"] == 0, f"device error word {g['err']:#x}"
@@ -171,7 +171,15 @@ def test_gpu_output_fails_against_mutated_oracle():
 
 @pytest.mark.parametrize("name", ["tiny", "opt13b", "gqa", "prefix", "fp8", "fp8_b32"])
 def test_full_size_workload(name):
-    """The five workloads at full size, in the launch configuration the benchmark times."""
+    """The five workloads at full size, in the launch configuration the benchmark times
+    (the workload's stated partition size, else the automatic one)."""
     w = wl.make(name)
     g, o, rep = check_step(w)
     print(name, rep)
+
+
+def test_full_size_fp8_automatic_partitions():
+    """The long-context FP8 workload with the automatic (2,048-token) partitions as well."""
+    w = wl.make("fp8")
+    g, o, rep = check_step(w, partition_size=0, pools=False)
+    print("fp8 auto", rep)

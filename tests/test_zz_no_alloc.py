@@ -63,7 +63,7 @@ def test_static_workspace_matches_caller_workspace_on_two_calls():
     f = static_entry()
     cases = [(wl.make("gqa", small=True), 64), (wl.make("fp8", small=True), 512)]
     for w, ps in cases:
-        need = B.decode_workspace_bytes(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.block_size,
+        need = B.decode_workspace_bytes(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.kv_dtype, w.block_size,
                                         w.max_context_len, ps)
         assert 0 < need <= STATIC_WS_BYTES      # the workspace is really used
     for w, ps in cases:                          # two calls in a row, each checked
@@ -90,7 +90,7 @@ def test_static_workspace_rejects_oversized_requests():
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     # claim a context long enough that the workspace would exceed the library's array
     big_len, ps = 1 << 22, w.block_size
-    assert B.decode_workspace_bytes(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.block_size,
+    assert B.decode_workspace_bytes(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.kv_dtype, w.block_size,
                                     big_len, ps) > STATIC_WS_BYTES
     stream = torch.cuda.current_stream().cuda_stream
     status = f(out.data_ptr(), t["q"].data_ptr(), CODES[w.q_dtype], t["kp"].data_ptr(), t["vp"].data_ptr(),
