@@ -99,17 +99,25 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
             : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Two E4M3 values (low byte first) -> two MMA operands packed in 32 bits (exact).
+// Four E4M3 values (bytes of x, low byte first) -> two MMA operand words: lo holds
+// bytes 0-1, hi bytes 2-3, each as a pair of 16-bit values (exact widening).
 template <bool kBf16>
-__device__ __forceinline__ uint32_t widen_e4m3x2(uint32_t two_bytes) {
-    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_bytes & 0xffffu),
-                                                     __NV_E4M3);
+__device__ __forceinline__ void widen_e4m3x4(uint32_t x, uint32_t& lo, uint32_t& hi) {
+    uint32_t h0, h1;
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+        : "=r"(h0), "=r"(h1)
+        : "r"(x));
     if constexpr (!kBf16) {
-        return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+        lo = h0;
+        hi = h1;
     } else {
-        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
-        const __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);
-        return *reinterpret_cast<const uint32_t*>(&b);
+        const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
+        const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
+        const __nv_bfloat162 b0 = __floats2bfloat162_rn(f0.x, f0.y);
+        const __nv_bfloat162 b1 = __floats2bfloat162_rn(f1.x, f1.y);
+        lo = *reinterpret_cast<const uint32_t*>(&b0);
+        hi = *reinterpret_cast<const uint32_t*>(&b1);
     }
 }
 
@@ -433,10 +441,8 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
                         const uint32_t wr = word(ks < 4 ? x0 : x1, ks & 3);   // token r, 4 bytes
                         const uint32_t wr8 = word(ks < 4 ? y0 : y1, ks & 3);  // token r + 8
                         uint32_t ka[4];
-                        ka[0] = widen_e4m3x2<kBf16>(wr);
-                        ka[1] = widen_e4m3x2<kBf16>(wr8);
-                        ka[2] = widen_e4m3x2<kBf16>(wr >> 16);
-                        ka[3] = widen_e4m3x2<kBf16>(wr8 >> 16);
+                        widen_e4m3x4<kBf16>(wr, ka[0], ka[2]);
+                        widen_e4m3x4<kBf16>(wr8, ka[1], ka[3]);
 #pragma unroll
                         for (int nh = 0; nh < NTH; ++nh) mma16816<kBf16>(sc[mt][nh], ka, qb[ks][nh][0], qb[ks][nh][1]);
                     }
@@ -547,14 +553,10 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
                         const uint32_t e01 = __byte_perm(x0, x1, 0x5140u), e23 = __byte_perm(x2, x3, 0x5140u);
                         const uint32_t f01 = __byte_perm(x0, x1, 0x7362u), f23 = __byte_perm(x2, x3, 0x7362u);
                         uint32_t va[4], vb[4];
-                        va[0] = widen_e4m3x2<kBf16>(e01);
-                        va[1] = widen_e4m3x2<kBf16>(e01 >> 16);
-                        va[2] = widen_e4m3x2<kBf16>(e23);
-                        va[3] = widen_e4m3x2<kBf16>(e23 >> 16);
-                        vb[0] = widen_e4m3x2<kBf16>(f01);
-                        vb[1] = widen_e4m3x2<kBf16>(f01 >> 16);
-                        vb[2] = widen_e4m3x2<kBf16>(f23);
-                        vb[3] = widen_e4m3x2<kBf16>(f23 >> 16);
+                        widen_e4m3x4<kBf16>(e01, va[0], va[1]);
+                        widen_e4m3x4<kBf16>(e23, va[2], va[3]);
+                        widen_e4m3x4<kBf16>(f01, vb[0], vb[1]);
+                        widen_e4m3x4<kBf16>(f23, vb[2], vb[3]);
 #pragma unroll
                         for (int nh = 0; nh < NTH; ++nh) {
                             mma16816<kBf16>(o[2 * w][nh], va, pb[mt][nh][0], pb[mt][nh][1]);
@@ -640,26 +642,60 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
 
 // ---- pass 2: merge partitions by log-sum-exp -------------------------------------
 
+// One CTA of D threads per (sequence, query head): the partitions' (max, sum) pairs
+// are staged in shared memory, the weights 2^(m_p - M) l_p computed once, and each
+// thread (one head_dim element) sums its column with eight loads in flight.
 template <bool kQBf16, int D>
 __global__ void __launch_bounds__(D) decode_reduce_kernel(const DecodeArgs a) {
+    extern __shared__ float sw[];   // [max_partitions] weights, then [D / 32] partial values
     const int qh = blockIdx.x, s = blockIdx.y, d = threadIdx.x;
     const int L = __ldg(a.context_lens + s);
     if (L <= 0 || L > a.max_blocks_per_seq * a.block_size || L > a.max_context_len) return;
-    const int nparts = (L + a.partition_size - 1) / a.partition_size;
-    if (nparts <= 1) return;
+    const int np = (L + a.partition_size - 1) / a.partition_size;
+    if (np <= 1) return;
     const size_t row = static_cast<size_t>(s) * a.num_heads + qh;
     const float2* ml = a.ws_ml + row * a.max_partitions;
     const float* wo = a.ws_o + row * a.max_partitions * D;
-    float M = -INFINITY;
-    for (int p = 0; p < nparts; ++p) M = fmaxf(M, ml[p].x);
-    float num = 0.f, den = 0.f;
-    for (int p = 0; p < nparts; ++p) {
+    float* red = sw + a.max_partitions;
+    // M = max_p m_p
+    float mx = -INFINITY;
+    for (int p = d; p < np; p += D) mx = fmaxf(mx, ml[p].x);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((d & 31) == 0) red[d >> 5] = mx;
+    __syncthreads();
+    float M = red[0];
+#pragma unroll
+    for (int w = 1; w < D / 32; ++w) M = fmaxf(M, red[w]);
+    // weights and their sum
+    float den = 0.f;
+    for (int p = d; p < np; p += D) {
         const float2 v = ml[p];
         const float w = exp2f(v.x - M) * v.y;
-        num += w * wo[static_cast<size_t>(p) * D + d];
+        sw[p] = w;
         den += w;
     }
-    store_out<kQBf16>(a.out, row * D + d, num / den);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    __syncthreads();   // every thread has read red[] for M and written its weights
+    if ((d & 31) == 0) red[d >> 5] = den;
+    __syncthreads();
+    float total = 0.f;
+#pragma unroll
+    for (int w = 0; w < D / 32; ++w) total += red[w];
+    // weighted column sums, eight independent loads at a time
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    int p = 0;
+    for (; p + 8 <= np; p += 8) {
+        float o[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) o[i] = wo[static_cast<size_t>(p + i) * D + d];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] += sw[p + i] * o[i];
+    }
+    for (; p < np; ++p) acc[0] += sw[p] * wo[static_cast<size_t>(p) * D + d];
+    const float num = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+    store_out<kQBf16>(a.out, row * D + d, num / total);
 }
 
 // ---- host side -----------------------------------------------------------------------
@@ -719,7 +755,13 @@ pkv_status launch_decode(const DecodeArgs& a, const CUtensorMap& km, const CUten
     kern<<<grid, kThreads, Gm::kSmemBytes, st>>>(a, km, vm);
     if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
     if (a.max_partitions > 1) {
-        decode_reduce_kernel<kQBf16, D><<<dim3(a.num_heads, a.num_seqs), D, 0, st>>>(a);
+        const size_t rsmem = (static_cast<size_t>(a.max_partitions) + D / 32) * sizeof(float);
+        auto rk = decode_reduce_kernel<kQBf16, D>;
+        if (rsmem > 48 * 1024 &&
+            cudaFuncSetAttribute(rk, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(rsmem)) !=
+                cudaSuccess)
+            return PKV_ERR_CUDA;
+        rk<<<dim3(a.num_heads, a.num_seqs), D, rsmem, st>>>(a);
         if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
     }
     return PKV_OK;
