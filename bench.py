@@ -206,22 +206,32 @@ def barrier_sync(torch, dist_on):
     torch.cuda.synchronize()
 
 
-def max_over_ranks(torch, x: float, dist_on: bool) -> float:
+def max_over_ranks(torch, x: float, dist_on: bool, device: str = "cuda") -> float:
+    """Slowest rank's time: the job's time under weak scaling."""
     if not dist_on:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
-def sum_over_ranks(torch, x: float, dist_on: bool) -> float:
+def sum_over_ranks(torch, x: float, dist_on: bool, device: str = "cuda") -> float:
+    """Whole-job quantity (bytes, sequences) summed over ranks."""
     if not dist_on:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def job_throughput(step_bytes_this_rank: float, ms_total_this_rank: float, steps: int, dist_on: bool,
+                   torch, device: str = "cuda"):
+    """(GB/s of the whole job, ms per step): bytes of all ranks / the slowest rank's time."""
+    ms_step = max_over_ranks(torch, ms_total_this_rank, dist_on, device) / steps
+    total = sum_over_ranks(torch, float(step_bytes_this_rank), dist_on, device)
+    return total / (ms_step * 1e-3) / 1e9, ms_step
 
 
 def run_ours(args, rank, world, local_rank):
@@ -262,10 +272,8 @@ def run_ours(args, rank, world, local_rank):
     sc_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
     cp_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
     assert int(ds.err.item()) == 0, "device error during the timed region"
-    ms_total = max_over_ranks(torch, ms_total, dist_on)
-    ms_step = ms_total / K
+    value, ms_step = job_throughput(step_bytes, ms_total, K, dist_on, torch)
     total_bytes = sum_over_ranks(torch, float(step_bytes), dist_on)
-    value = total_bytes / (ms_step * 1e-3) / 1e9
     seqs = sum_over_ranks(torch, float(w.num_seqs), dist_on)
 
     # end to end: the step's inputs from pinned host memory, the output back to the host

@@ -203,6 +203,17 @@ pkv_status pkv_copy_blocks(void* k_pool, void* v_pool, size_t block_bytes,
                            const int64_t* pairs, int num_pairs, int num_blocks,
                            uint32_t* device_error, void* stream);
 
+/*
+ * Diagnostic for the failure handling above (no counterpart on the pages): runs one
+ * kernel whose single wait can never be satisfied; the wait gives up after
+ * timeout_us microseconds (1 .. 10,000,000) and OR-s PKV_DEVERR_TIMEOUT into
+ * *device_error (device pointer, required).  Nothing faults or hangs; the
+ * context stays usable.  A decode call given a device_error word that already
+ * holds PKV_DEVERR_TIMEOUT finishes at once and writes NaN (a grid that saw a
+ * wait give up stops early), so clear the word after reading it.
+ */
+pkv_status pkv_selftest_bounded_wait(uint32_t* device_error, unsigned timeout_us, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

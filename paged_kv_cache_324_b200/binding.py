@@ -55,6 +55,8 @@ def lib() -> ctypes.CDLL:
         L.pkv_reshape_and_cache.restype = I
         L.pkv_copy_blocks.argtypes = [P, P, Z, P, I, I, P, P]
         L.pkv_copy_blocks.restype = I
+        L.pkv_selftest_bounded_wait.argtypes = [P, ctypes.c_uint, P]
+        L.pkv_selftest_bounded_wait.restype = I
         _lib = L
     return _lib
 
@@ -174,3 +176,9 @@ def copy_blocks(k_pool: torch.Tensor, v_pool: torch.Tensor, pairs: torch.Tensor,
         _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"), block_bytes, _dev(pairs, "pairs"),
         pairs.numel() // 2, k_pool.shape[0], _dev(device_error, "device_error"), _stream(stream))
     _check(status, "copy_blocks")
+
+
+def selftest_bounded_wait(device_error: torch.Tensor, timeout_us: int, stream=None) -> None:
+    """Run one bounded wait that nothing completes; it sets DEVERR_TIMEOUT in device_error."""
+    _check(lib().pkv_selftest_bounded_wait(_dev(device_error, "device_error"), int(timeout_us), _stream(stream)),
+           "selftest_bounded_wait")

@@ -4,6 +4,7 @@
 
 #include <mutex>
 
+#include "pkv_device.cuh"
 #include "pkv_host.h"
 
 namespace pkv {
@@ -43,4 +44,33 @@ extern "C" const char* pkv_status_string(pkv_status s) {
     case PKV_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
     }
     return "unknown status";
+}
+
+// ---- diagnostic: one bounded wait that nothing completes ---------------------------
+
+namespace pkv {
+namespace {
+
+// Waits on phase 0 of a fresh barrier that no thread arrives on; the wait gives up
+// after timeout_ns and reports PKV_DEVERR_TIMEOUT, exercising the same bounded
+// wait the decode kernel uses for its TMA and ring barriers.
+__global__ void selftest_wait_kernel(uint32_t* err, unsigned long long timeout_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t b = smem_addr(&bar);
+    if (threadIdx.x == 0) {
+        mbar_init(b, 1);
+        mbar_fence_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !mbar_wait(b, 0, global_timer_ns() + timeout_ns)) raise_error(err, PKV_DEVERR_TIMEOUT);
+}
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" pkv_status pkv_selftest_bounded_wait(uint32_t* device_error, unsigned timeout_us, void* stream) {
+    if (!device_error || timeout_us == 0 || timeout_us > 10u * 1000u * 1000u) return PKV_ERR_INVALID_ARG;
+    pkv::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        device_error, static_cast<unsigned long long>(timeout_us) * 1000ull);
+    return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }

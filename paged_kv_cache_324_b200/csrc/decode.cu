@@ -654,6 +654,10 @@ __global__ void __launch_bounds__(D) decode_reduce_kernel(const DecodeArgs a) {
     const int np = (L + a.partition_size - 1) / a.partition_size;
     if (np <= 1) return;
     const size_t row = static_cast<size_t>(s) * a.num_heads + qh;
+    if (grid_timed_out(a.err)) {   // pass 1 gave up somewhere: its partials are not to be trusted
+        store_out<kQBf16>(a.out, row * D + d, __int_as_float(0x7fc00000));
+        return;
+    }
     const float2* ml = a.ws_ml + row * a.max_partitions;
     const float* wo = a.ws_o + row * a.max_partitions * D;
     float* red = sw + a.max_partitions;
