@@ -30,6 +30,8 @@ reshape_and_cache_kernel(const uint4* __restrict__ k, const uint4* __restrict__ 
                          const int64_t* __restrict__ slot_mapping, int num_tokens,
                          int num_kv_heads, int head_dim, int block_size, int num_blocks,
                          float k_scale, float v_scale, uint32_t* err) {
+    pdl_trigger();
+    pdl_wait();   // the previous kernel may still read the pool
     const int vec_per_row = head_dim / 8;                 // 8 elements per 16-byte input vector
     const int vec_per_tok = num_kv_heads * vec_per_row;
     const long long total = static_cast<long long>(num_tokens) * vec_per_tok;
@@ -92,6 +94,8 @@ __global__ void __launch_bounds__(256)
 copy_blocks_kernel(uint8_t* __restrict__ k_pool, uint8_t* __restrict__ v_pool,
                    size_t block_bytes, const int64_t* __restrict__ pairs, int num_pairs,
                    int num_blocks, uint32_t* err) {
+    pdl_trigger();
+    pdl_wait();   // the previous kernel may still read the pool
     uint8_t* pool = blockIdx.z == 0 ? k_pool : v_pool;
     const size_t nvec = block_bytes / 16;
     for (int p = blockIdx.y; p < num_pairs; p += gridDim.y) {
@@ -138,18 +142,19 @@ extern "C" pkv_status pkv_reshape_and_cache(const void* k, const void* v, pkv_dt
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const bool fp8 = kv_dtype == PKV_FP8_E4M3, bf16 = in_dtype == PKV_BF16;
     auto launch = [&](auto kern) {
-        kern<<<static_cast<unsigned>(blocks), threads, 0, st>>>(
-            static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint8_t*>(k_pool),
-            static_cast<uint8_t*>(v_pool), slot_mapping, num_tokens, num_kv_heads, head_dim, block_size,
-            num_blocks, k_scale, v_scale, device_error);
+        return launch_pdl(kern, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, st,
+                          static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint8_t*>(k_pool),
+                          static_cast<uint8_t*>(v_pool), slot_mapping, num_tokens, num_kv_heads, head_dim,
+                          block_size, num_blocks, k_scale, v_scale, device_error);
     };
+    cudaError_t e;
     if (!fp8)
-        launch(reshape_and_cache_kernel<false, false>);
+        e = launch(reshape_and_cache_kernel<false, false>);
     else if (bf16)
-        launch(reshape_and_cache_kernel<true, true>);
+        e = launch(reshape_and_cache_kernel<true, true>);
     else
-        launch(reshape_and_cache_kernel<true, false>);
-    return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+        e = launch(reshape_and_cache_kernel<true, false>);
+    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
 extern "C" pkv_status pkv_copy_blocks(void* k_pool, void* v_pool, size_t block_bytes,
@@ -168,8 +173,8 @@ extern "C" pkv_status pkv_copy_blocks(void* k_pool, void* v_pool, size_t block_b
     if (gx == 0) gx = 1;
     unsigned gy = static_cast<unsigned>(num_pairs < 65535 ? num_pairs : 65535);
     dim3 grid(gx, gy, 2);
-    copy_blocks_kernel<<<grid, threads, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<uint8_t*>(k_pool), static_cast<uint8_t*>(v_pool), block_bytes, pairs, num_pairs,
-        num_blocks, device_error);
-    return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+    const cudaError_t e = launch_pdl(copy_blocks_kernel, grid, dim3(threads), 0, static_cast<cudaStream_t>(stream),
+                                     static_cast<uint8_t*>(k_pool), static_cast<uint8_t*>(v_pool), block_bytes,
+                                     pairs, num_pairs, num_blocks, device_error);
+    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }

@@ -261,6 +261,7 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
     const bool give_up = grid_timed_out(a.err);
     if (bad_len || L == 0 || give_up) {
         if (part == 0) {
+            pdl_wait();
             if (bad_len && threadIdx.x == 0) raise_error(a.err, PKV_DEVERR_CONTEXT_LEN);
             const float v = (bad_len || give_up) ? __int_as_float(0x7fc00000) : 0.f;
             for (int e = threadIdx.x; e < G * D; e += kThreads)
@@ -327,6 +328,7 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
                 *s_abort = 1;
             }
             if (bad) pid = 0;   // load an in-range block; the output becomes NaN
+            if (j0 == 0) pdl_wait();   // the pool may still be written by the previous kernel
             const int cnt = min(kChunk, nblk - j0);
             for (int i = 0; i < cnt; i += Gm::kBps) {
                 const int js = (j0 + i) / Gm::kBps;   // stage index within the partition
@@ -391,6 +393,7 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
                 qb[ks][nh][1] = ok ? __ldg(qrow + ((d0 + Gm::kQkB1) >> 1)) : 0u;
             }
         }
+        pdl_wait();   // outputs and partials are written only after the previous kernel
         // per-lane ldmatrix row addresses (16-bit tiles): lane supplies row (lane & 7) of
         // matrix lane >> 3; the swizzle XOR only depends on (lane & 7)
         const int li = lane >> 3, l7 = lane & 7;
@@ -584,6 +587,7 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
                 l_run[nh][hc] = v;
             }
     }
+    pdl_trigger();     // the merge kernel (or the next step) may start its prologue
     __syncthreads();   // ring fully consumed: reuse it for the merge
 
     float* sm_o = reinterpret_cast<float*>(gbase);                    // [warps][16 heads][D]
@@ -648,6 +652,8 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
 template <bool kQBf16, int D>
 __global__ void __launch_bounds__(D) decode_reduce_kernel(const DecodeArgs a) {
     extern __shared__ float sw[];   // [max_partitions] weights, then [D / 32] partial values
+    pdl_trigger();
+    pdl_wait();
     const int qh = blockIdx.x, s = blockIdx.y, d = threadIdx.x;
     const int L = __ldg(a.context_lens + s);
     if (L <= 0 || L > a.max_blocks_per_seq * a.block_size || L > a.max_context_len) return;
@@ -660,6 +666,30 @@ __global__ void __launch_bounds__(D) decode_reduce_kernel(const DecodeArgs a) {
     }
     const float2* ml = a.ws_ml + row * a.max_partitions;
     const float* wo = a.ws_o + row * a.max_partitions * D;
+    if (np <= 8) {   // few partitions: every thread reads the pairs itself, all loads at once
+        float2 v[8];
+        float o[8];
+#pragma unroll
+        for (int p = 0; p < 8; ++p)
+            if (p < np) {
+                v[p] = ml[p];
+                o[p] = wo[static_cast<size_t>(p) * D + d];
+            }
+        float M = -INFINITY;
+#pragma unroll
+        for (int p = 0; p < 8; ++p)
+            if (p < np) M = fmaxf(M, v[p].x);
+        float num = 0.f, den = 0.f;
+#pragma unroll
+        for (int p = 0; p < 8; ++p)
+            if (p < np) {
+                const float w = exp2f(v[p].x - M) * v[p].y;
+                num += w * o[p];
+                den += w;
+            }
+        store_out<kQBf16>(a.out, row * D + d, num / den);
+        return;
+    }
     float* red = sw + a.max_partitions;
     // M = max_p m_p
     float mx = -INFINITY;
@@ -756,8 +786,7 @@ pkv_status launch_decode(const DecodeArgs& a, const CUtensorMap& km, const CUten
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Gm::kSmemBytes) != cudaSuccess)
         return PKV_ERR_CUDA;
     dim3 grid(a.max_partitions, a.num_kv_heads, a.num_seqs);
-    kern<<<grid, kThreads, Gm::kSmemBytes, st>>>(a, km, vm);
-    if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
+    if (launch_pdl(kern, grid, dim3(kThreads), Gm::kSmemBytes, st, a, km, vm) != cudaSuccess) return PKV_ERR_CUDA;
     if (a.max_partitions > 1) {
         const size_t rsmem = (static_cast<size_t>(a.max_partitions) + D / 32) * sizeof(float);
         auto rk = decode_reduce_kernel<kQBf16, D>;
@@ -765,7 +794,8 @@ pkv_status launch_decode(const DecodeArgs& a, const CUtensorMap& km, const CUten
             cudaFuncSetAttribute(rk, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(rsmem)) !=
                 cudaSuccess)
             return PKV_ERR_CUDA;
-        rk<<<dim3(a.num_heads, a.num_seqs), D, rsmem, st>>>(a);
+        if (launch_pdl(rk, dim3(a.num_heads, a.num_seqs), dim3(D), rsmem, st, a) != cudaSuccess)
+            return PKV_ERR_CUDA;
         if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
     }
     return PKV_OK;

@@ -81,6 +81,15 @@ __device__ __forceinline__ bool grid_timed_out(const uint32_t* err) {
     return err && (*reinterpret_cast<const volatile uint32_t*>(err) & PKV_DEVERR_TIMEOUT);
 }
 
+// ---- programmatic dependent launch ------------------------------------------
+// Kernels are launched so that they may start while the previous kernel on the
+// stream finishes; pdl_wait() blocks until that kernel has completed and its
+// memory is visible, and must precede any access to data it may write or read.
+// pdl_trigger() lets the next kernel on the stream start its own prologue.
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---- TMA ------------------------------------------------------------------
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
