@@ -55,7 +55,8 @@ typedef enum {
     PKV_ERR_UNSUPPORTED = 2,   /* valid but not implemented: head_dim, block_size, dtype pair, group size */
     PKV_ERR_WORKSPACE = 3,     /* workspace missing or smaller than pkv_decode_workspace_bytes() */
     PKV_ERR_CUDA = 4,          /* a CUDA runtime or driver call failed */
-    PKV_ERR_ALIGNMENT = 5      /* a pointer is not 16-byte aligned */
+    PKV_ERR_ALIGNMENT = 5,     /* a pointer is not 16-byte aligned */
+    PKV_ERR_OUT_OF_BLOCKS = 6  /* the block manager's free list cannot serve the request */
 } pkv_status;
 
 typedef enum {
@@ -202,6 +203,47 @@ pkv_status pkv_reshape_and_cache(const void* k, const void* v, pkv_dtype in_dtyp
 pkv_status pkv_copy_blocks(void* k_pool, void* v_pool, size_t block_bytes,
                            const int64_t* pairs, int num_pairs, int num_blocks,
                            uint32_t* device_error, void* stream);
+
+/*
+ * Host-side block manager (no GPU involved): the bookkeeping that produces block
+ * tables, slot mappings and copy-on-write pairs for the kernels above
+ * (glossary "PagedAttention", sections "How paging works" and "Sharing blocks
+ * across sequences").  Blocks are handed out from a FIFO free list; a sequence
+ * takes a new block only when its last one is full; a fork shares every block of
+ * its parent (reference counts); appending to a partially filled block that other
+ * sequences still reference first moves the writer to a fresh block and reports
+ * the (src, dst) copy for pkv_copy_blocks -- the last holder writes in place;
+ * freeing a sequence returns blocks whose count drops to zero to the back of the
+ * free list.  All arrays are HOST memory.  Calls on one manager are serialised
+ * internally (thread-safe).  A call that fails returns a status and changes
+ * nothing.
+ */
+typedef struct pkv_block_manager pkv_block_manager;
+
+/* free_order: a permutation of 0..num_blocks-1 giving the initial free-list order
+ * (NULL = ascending).  Returns NULL for invalid arguments or memory exhaustion. */
+pkv_block_manager* pkv_bm_create(int num_blocks, int block_size, const int32_t* free_order);
+void pkv_bm_destroy(pkv_block_manager* m);
+int pkv_bm_num_free(pkv_block_manager* m);
+/* A new empty sequence; PKV_ERR_INVALID_ARG if seq_id exists. */
+pkv_status pkv_bm_add_sequence(pkv_block_manager* m, int64_t seq_id);
+/* child starts as a copy of parent's table and length, sharing every block. */
+pkv_status pkv_bm_fork(pkv_block_manager* m, int64_t parent, int64_t child);
+/* Append one token to each of the n distinct sequences, in order: slots[i] is the
+ * slot (block_id * block_size + offset) where sequence i's new token goes; copy
+ * pairs (int64 [max_pairs][2], src then dst) are written for shared partial
+ * blocks and their count stored in *num_pairs.  PKV_ERR_OUT_OF_BLOCKS if the free
+ * list is too short (nothing changes: the caller may free or preempt and retry). */
+pkv_status pkv_bm_append_slots(pkv_block_manager* m, const int64_t* seq_ids, int n, int64_t* slots,
+                               int64_t* pairs, int max_pairs, int* num_pairs);
+/* Drop a sequence; its blocks' reference counts fall, unreferenced blocks return. */
+pkv_status pkv_bm_free_sequence(pkv_block_manager* m, int64_t seq_id);
+/* Rows of int32 [n][max_blocks] block tables (entries past a sequence's last block
+ * set to pad) and, if context_lens is not NULL, the sequences' lengths. */
+pkv_status pkv_bm_block_tables(pkv_block_manager* m, const int64_t* seq_ids, int n, int32_t* tables,
+                               int max_blocks, int32_t pad, int32_t* context_lens);
+int pkv_bm_ref_count(pkv_block_manager* m, int32_t block);          /* -1 if out of range */
+int64_t pkv_bm_sequence_length(pkv_block_manager* m, int64_t seq_id);  /* -1 if unknown */
 
 /*
  * Diagnostic for the failure handling above (no counterpart on the pages): runs one

@@ -182,3 +182,85 @@ def selftest_bounded_wait(device_error: torch.Tensor, timeout_us: int, stream=No
     """Run one bounded wait that nothing completes; it sets DEVERR_TIMEOUT in device_error."""
     _check(lib().pkv_selftest_bounded_wait(_dev(device_error, "device_error"), int(timeout_us), _stream(stream)),
            "selftest_bounded_wait")
+
+
+class BlockManager:
+    """Host-side block manager of the library (pkv_bm_* in include/pagedkv.h)."""
+
+    def __init__(self, num_blocks: int, block_size: int, free_order=None):
+        import numpy as np
+        L = lib()
+        P, I, I64, I32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_int32
+        L.pkv_bm_create.argtypes = [I, I, P]
+        L.pkv_bm_create.restype = P
+        L.pkv_bm_destroy.argtypes = [P]
+        L.pkv_bm_num_free.argtypes = [P]
+        L.pkv_bm_add_sequence.argtypes = [P, I64]
+        L.pkv_bm_fork.argtypes = [P, I64, I64]
+        L.pkv_bm_append_slots.argtypes = [P, P, I, P, P, I, P]
+        L.pkv_bm_free_sequence.argtypes = [P, I64]
+        L.pkv_bm_block_tables.argtypes = [P, P, I, P, I, I32, P]
+        L.pkv_bm_ref_count.argtypes = [P, I32]
+        L.pkv_bm_sequence_length.argtypes = [P, I64]
+        L.pkv_bm_sequence_length.restype = I64
+        self._L, self._np = L, np
+        order = None
+        if free_order is not None:
+            order = np.ascontiguousarray(free_order, dtype=np.int32)
+        self.block_size = block_size
+        self._h = L.pkv_bm_create(num_blocks, block_size,
+                                  order.ctypes.data_as(P) if order is not None else None)
+        if not self._h:
+            raise ValueError("invalid block manager arguments (free_order must be a permutation)")
+
+    def __del__(self):
+        if getattr(self, "_h", None):
+            self._L.pkv_bm_destroy(self._h)
+            self._h = None
+
+    def _ok(self, status, what):
+        _check(status, what)
+
+    @property
+    def num_free(self) -> int:
+        return self._L.pkv_bm_num_free(self._h)
+
+    def add_sequence(self, seq_id: int):
+        self._ok(self._L.pkv_bm_add_sequence(self._h, seq_id), "add_sequence")
+
+    def fork(self, parent: int, child: int):
+        self._ok(self._L.pkv_bm_fork(self._h, parent, child), "fork")
+
+    def append_slots(self, seq_ids):
+        """One new token per sequence: (slots int64 [n], copy pairs int64 [k, 2])."""
+        np = self._np
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        n = ids.size
+        slots = np.empty(n, np.int64)
+        pairs = np.empty((max(n, 1), 2), np.int64)
+        k = ctypes.c_int(0)
+        P = ctypes.c_void_p
+        self._ok(self._L.pkv_bm_append_slots(self._h, ids.ctypes.data_as(P), n, slots.ctypes.data_as(P),
+                                             pairs.ctypes.data_as(P), pairs.shape[0], ctypes.byref(k)),
+                 "append_slots")
+        return slots, pairs[:k.value].copy()
+
+    def free_sequence(self, seq_id: int):
+        self._ok(self._L.pkv_bm_free_sequence(self._h, seq_id), "free_sequence")
+
+    def block_tables(self, seq_ids, max_blocks: int, pad: int = -1):
+        """(int32 [n, max_blocks] tables, int32 [n] lengths)."""
+        np = self._np
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        t = np.empty((ids.size, max_blocks), np.int32)
+        lens = np.empty(ids.size, np.int32)
+        P = ctypes.c_void_p
+        self._ok(self._L.pkv_bm_block_tables(self._h, ids.ctypes.data_as(P), ids.size, t.ctypes.data_as(P),
+                                             max_blocks, pad, lens.ctypes.data_as(P)), "block_tables")
+        return t, lens
+
+    def ref_count(self, block: int) -> int:
+        return self._L.pkv_bm_ref_count(self._h, block)
+
+    def sequence_length(self, seq_id: int) -> int:
+        return self._L.pkv_bm_sequence_length(self._h, seq_id)

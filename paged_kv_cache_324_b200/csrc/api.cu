@@ -42,6 +42,7 @@ extern "C" const char* pkv_status_string(pkv_status s) {
     case PKV_ERR_WORKSPACE: return "workspace missing or too small";
     case PKV_ERR_CUDA: return "CUDA error";
     case PKV_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case PKV_ERR_OUT_OF_BLOCKS: return "out of free blocks";
     }
     return "unknown status";
 }
