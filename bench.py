@@ -39,6 +39,7 @@ from paged_kv_cache_324_b200 import workload as wl  # noqa: E402
 METRIC = "paged decode attention KV GB/s and % of B200 HBM peak; sequences/sec"
 UNIT = "GB/s"
 NOMINAL_HBM_GBS = 8000.0
+L2_BYTES = 126 * 1000 * 1000
 FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic of one paged_decode_kernel + reduce launch measured by ncu
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by workload, valid only
@@ -125,7 +126,7 @@ class ClockSampler:
 class DeviceStep:
     """A workload's pools and inputs on one GPU, and the calls of one step."""
 
-    def __init__(self, w: wl.DecodeWorkload, dev, partition_size: int = 0):
+    def __init__(self, w: wl.DecodeWorkload, dev, partition_size: int = 0, prefix_aware: bool = False):
         import torch
         from paged_kv_cache_324_b200 import binding as B
         self.w, self.dev, self.B, self.torch = w, dev, B, torch
@@ -169,12 +170,23 @@ class DeviceStep:
         self.partition_arg = partition_size
         self.partition = B.decode_partition_size(w.num_seqs, w.num_kv_heads, w.head_dim, w.kv_dtype, w.block_size,
                                                  w.max_context_len, partition_size)
+        self.prefix_aware = prefix_aware
+        if prefix_aware:   # read each shared prompt once per unit of samples
+            G = w.num_heads // w.num_kv_heads
+            spl, us, ul, mp = B.find_shared_prefixes(w.block_tables, w.context_lens, w.block_size, 16 // G)
+            self.sp = {"seq_prefix_len": torch.from_numpy(spl).to(dev), "unit_seqs": torch.from_numpy(us).to(dev),
+                       "unit_len": torch.from_numpy(ul).to(dev), "max_prefix_len": mp, "units": len(ul)}
+            n = B.shared_prefix_workspace_bytes(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.kv_dtype,
+                                                w.block_size, w.max_context_len, len(ul), mp, partition_size)
+            self.ws = torch.empty(max(n, 256), dtype=torch.uint8, device=dev)
         self.split = w.max_context_len > self.partition
         torch.cuda.synchronize(dev)
         assert int(self.err.item()) == 0, "setup raised a device error"
 
     def launches_per_step(self) -> int:
-        return ("pairs" in self.d) + 1 + 1 + int(self.split)
+        if self.prefix_aware:   # prefix pass (if any unit), own-token pass, merge
+            return ("pairs" in self.d) + 1 + (self.sp["units"] > 0) + 2
+        return ("pairs" in self.d) + 1 + 1 + int(self.w.max_context_len > self.partition) + int(self.split)
 
     def copy_op(self):
         if "pairs" in self.d:
@@ -188,6 +200,15 @@ class DeviceStep:
 
     def decode_op(self):
         w = self.w
+        if self.prefix_aware:
+            sp = self.sp
+            self.B.paged_attn_decode_shared_prefix(
+                self.out, self.d["q"], self.k_pool, self.v_pool, self.d["tables"], self.d["lens"], float(w.scale),
+                max_context_len=w.max_context_len, seq_prefix_len=sp["seq_prefix_len"], unit_seqs=sp["unit_seqs"],
+                unit_len=sp["unit_len"], max_prefix_len=sp["max_prefix_len"], k_scale=float(w.k_scale),
+                v_scale=float(w.v_scale), partition_size=self.partition_arg, workspace=self.ws,
+                device_error=self.err, stream=self.stream)
+            return
         self.B.paged_attn_decode(self.out, self.d["q"], self.k_pool, self.v_pool, self.d["tables"],
                                  self.d["lens"], float(w.scale), max_context_len=w.max_context_len,
                                  k_scale=float(w.k_scale), v_scale=float(w.v_scale), workspace=self.ws,
@@ -241,9 +262,11 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     w = wl.make(args.config)        # weak scaling: every rank runs a batch of the same shape
     ps = w.partition_size if args.partition == "config" else (0 if args.partition == "auto" else int(args.partition))
-    ds = DeviceStep(w, dev, ps)
+    ds = DeviceStep(w, dev, ps, prefix_aware=args.prefix_aware)
     step_bytes = wl.step_algorithmic_bytes(w)
     dec_bytes = wl.decode_algorithmic_bytes(w)
+    # the roofline counts each physical KV slot once: on shared prompts that is what must cross HBM
+    roof_bytes = wl.decode_distinct_bytes(w)
 
     for _ in range(args.warmup):
         ds.step()
@@ -314,7 +337,7 @@ def run_ours(args, rank, world, local_rank):
 
     peak, peak_kind = hbm_peak()
     dec_avg = sum(dec_ms) / K
-    achieved = dec_bytes / (dec_avg * 1e-3) / 1e9
+    achieved = roof_bytes / (dec_avg * 1e-3) / 1e9
     traffic = None
     tr = NCU_TRAFFIC.get(args.config)
     if tr and tr.get("kernel_sha") == decode_source_sha():
@@ -331,9 +354,13 @@ def run_ours(args, rank, world, local_rank):
             "num_blocks": w.num_blocks, "max_context_len": w.max_context_len,
             "total_context_tokens": int(w.context_lens.sum()), "partition_size": ds.partition,
             "partition_rule": "automatic" if ds.partition_arg == 0 else "set by the workload or --partition",
-            "step": ("copy_blocks + " if "pairs" in ds.d else "") + "reshape_and_cache + paged_attn_decode",
-            "step_bytes": step_bytes, "decode_bytes": dec_bytes,
-            "l2": "no flush: each step reads %.2f GB of KV, more than the 126 MB L2" % (dec_bytes / 1e9),
+            "step": ("copy_blocks + " if "pairs" in ds.d else "") + "reshape_and_cache + " +
+                    ("paged_attn_decode_shared_prefix" if ds.prefix_aware else "paged_attn_decode"),
+            "step_bytes": step_bytes, "decode_bytes": dec_bytes, "decode_distinct_bytes": roof_bytes,
+            "l2": (("no flush: each step reads %.2f GB of distinct KV, more than the 126 MB L2" % (roof_bytes / 1e9))
+                   if roof_bytes > L2_BYTES else
+                   ("no flush: the %.0f MB of distinct KV fit in the 126 MB L2, so repeated reads of shared "
+                    "blocks may hit L2" % (roof_bytes / 1e6))),
             "parallelism": f"dp{world}" if world > 1 else "single GPU",
         },
         "sequences_per_s": round(seqs / (ms_step * 1e-3), 1),
@@ -344,6 +371,8 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "hbm", "kernel": "paged_decode_kernel + decode_reduce_kernel",
                      "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "bytes_per_launch": roof_bytes,
+                     "bytes_counted": "distinct KV slots attended (each once) + q + out + table entries + lengths",
                      "peak_kind": f"{peak_kind} (copy, burst)"},
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "ms_per_step": round(e2e_ms, 5),
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -409,8 +438,10 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--config", default="opt13b", choices=list(wl.NAMES) + list(wl.COMPACT_NAMES))
+    ap.add_argument("--config", default="opt13b", choices=list(wl.NAMES) + list(wl.EXTRA_NAMES) + list(wl.COMPACT_NAMES))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--prefix-aware", action="store_true",
+                    help="decode with pkv_paged_attn_decode_shared_prefix (shared prompts read once per unit)")
     ap.add_argument("--partition", default="config",
                     help="'config' (the workload's stated partition size, else automatic), 'auto', or tokens")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")

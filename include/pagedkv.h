@@ -137,6 +137,58 @@ pkv_status pkv_paged_attn_decode(void* out, const void* q, pkv_dtype q_dtype,
                                  uint32_t* device_error, void* stream);
 
 /*
+ * Shared-prefix decode: pkv_paged_attn_decode's result, computed with each shared
+ * prefix read once per unit instead of once per sequence (several sequences whose
+ * tables begin with the same full blocks -- parallel samples or beam candidates of
+ * one prompt, glossary "PagedAttention", section "Sharing blocks across
+ * sequences").  Pass 1 runs every unit's query rows (all heads of up to
+ * unit_width members, unit_width * G <= 16) over the unit's shared tokens; pass 2
+ * runs every sequence over its own tokens, from the end of its prefix; a merge
+ * combines both sets of partials exactly by log-sum-exp.  The prefix pass picks its
+ * own partition size (the automatic rule applied to units instead of sequences).
+ *
+ *   seq_prefix_len  device int32 [num_seqs]: shared tokens of each sequence (a
+ *                   multiple of block_size, <= its context length; 0 = none)
+ *   unit_seqs       device int32 [num_units][unit_width]: member sequences of each
+ *                   unit (-1 pads the last slots); members must share their first
+ *                   unit_len[u] / block_size table entries and have that prefix length
+ *   unit_len        device int32 [num_units]
+ *   max_prefix_len  bound of the prefix lengths
+ *   workspace       >= pkv_shared_prefix_workspace_bytes() bytes (always needed)
+ * Other arguments, errors and results as for pkv_paged_attn_decode.
+ * pkv_find_shared_prefixes() builds the three arrays from host copies of the tables.
+ */
+size_t pkv_shared_prefix_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                         pkv_dtype kv_dtype, int block_size, int max_context_len,
+                                         int num_units, int max_prefix_len, int partition_size);
+
+pkv_status pkv_paged_attn_decode_shared_prefix(void* out, const void* q, pkv_dtype q_dtype,
+                                               const void* k_pool, const void* v_pool, pkv_dtype kv_dtype,
+                                               float k_scale, float v_scale,
+                                               const int32_t* block_tables, int max_blocks_per_seq,
+                                               const int32_t* context_lens, int max_context_len,
+                                               int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                               int block_size, int num_blocks, float scale, int partition_size,
+                                               const int32_t* seq_prefix_len, const int32_t* unit_seqs,
+                                               const int32_t* unit_len, int num_units, int unit_width,
+                                               int max_prefix_len, void* workspace, size_t workspace_bytes,
+                                               uint32_t* device_error, void* stream);
+
+/*
+ * Host helper (HOST arrays): groups sequences whose tables start with the same
+ * block ids, takes the longest run of leading blocks common to a group and full in
+ * every member as its shared prefix, and packs each group into units of at most
+ * unit_width members.  Sequences alone in their group get prefix 0 and no unit.
+ * Fills seq_prefix_len [num_seqs], unit_seqs [max_units][unit_width], unit_len
+ * [max_units], *num_units and *max_prefix_len; PKV_ERR_INVALID_ARG if more than
+ * max_units units are needed.
+ */
+pkv_status pkv_find_shared_prefixes(const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                                    int max_blocks_per_seq, int block_size, int unit_width,
+                                    int32_t* seq_prefix_len, int32_t* unit_seqs, int32_t* unit_len,
+                                    int max_units, int* num_units, int* max_prefix_len);
+
+/*
  * Size of the library-owned workspace used by pkv_paged_attn_decode_static_ws
  * (64 MiB of device memory, held by every GPU that loads the library).
  */

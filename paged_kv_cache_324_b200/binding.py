@@ -264,3 +264,63 @@ class BlockManager:
 
     def sequence_length(self, seq_id: int) -> int:
         return self._L.pkv_bm_sequence_length(self._h, seq_id)
+
+
+def find_shared_prefixes(block_tables, context_lens, block_size: int, unit_width: int):
+    """Host arrays in, (seq_prefix_len int32 [S], unit_seqs int32 [U, W], unit_len int32 [U], max_prefix_len)."""
+    import numpy as np
+    L = lib()
+    P, I = ctypes.c_void_p, ctypes.c_int
+    L.pkv_find_shared_prefixes.argtypes = [P, P, I, I, I, I, P, P, P, I, P, P]
+    t = np.ascontiguousarray(block_tables, dtype=np.int32)
+    lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+    S, maxb = t.shape
+    cap = max(S, 1)
+    spl = np.empty(S, np.int32)
+    us = np.empty((cap, unit_width), np.int32)
+    ul = np.empty(cap, np.int32)
+    nu, mp = ctypes.c_int(0), ctypes.c_int(0)
+    _check(L.pkv_find_shared_prefixes(t.ctypes.data_as(P), lens.ctypes.data_as(P), S, maxb, block_size, unit_width,
+                                      spl.ctypes.data_as(P), us.ctypes.data_as(P), ul.ctypes.data_as(P), cap,
+                                      ctypes.byref(nu), ctypes.byref(mp)), "find_shared_prefixes")
+    return spl, us[:nu.value].copy(), ul[:nu.value].copy(), mp.value
+
+
+def shared_prefix_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, kv_dtype, block_size,
+                                  max_context_len, num_units, max_prefix_len, partition_size=0) -> int:
+    L = lib()
+    I = ctypes.c_int
+    L.pkv_shared_prefix_workspace_bytes.argtypes = [I, I, I, I, I, I, I, I, I, I]
+    L.pkv_shared_prefix_workspace_bytes.restype = ctypes.c_size_t
+    return L.pkv_shared_prefix_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, _kv_code(kv_dtype),
+                                               block_size, max_context_len, num_units, max_prefix_len,
+                                               partition_size)
+
+
+def paged_attn_decode_shared_prefix(out, q, k_pool, v_pool, block_tables, context_lens, scale, *,
+                                    max_context_len: int, seq_prefix_len, unit_seqs, unit_len,
+                                    max_prefix_len: int, k_scale: float = 1.0, v_scale: float = 1.0,
+                                    partition_size: int = 0, workspace=None, device_error=None, stream=None):
+    """Shared-prefix decode: device tensors; seq_prefix_len int32 [S], unit_seqs int32 [U, W], unit_len int32 [U]."""
+    L = lib()
+    P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    L.pkv_paged_attn_decode_shared_prefix.argtypes = [P, P, I, P, P, I, F, F, P, I, P, I, I, I, I, I, I, I, F, I,
+                                                      P, P, P, I, I, I, P, Z, P, P]
+    S, H, D = q.shape
+    NB, Hkv, B, _ = k_pool.shape
+    need = shared_prefix_workspace_bytes(S, H, Hkv, D, k_pool.dtype, B, max_context_len, unit_len.numel(),
+                                         max_prefix_len, partition_size)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    U = unit_len.numel()
+    W = unit_seqs.shape[1] if unit_seqs.dim() == 2 and U else 1
+    status = L.pkv_paged_attn_decode_shared_prefix(
+        _dev(out, "out"), _dev(q, "q"), _code(q), _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"), _code(k_pool),
+        float(k_scale), float(v_scale), _dev(block_tables, "block_tables"), block_tables.shape[1],
+        _dev(context_lens, "context_lens"), int(max_context_len), S, H, Hkv, D, B, NB, float(scale),
+        int(partition_size), _dev(seq_prefix_len, "seq_prefix_len"),
+        _dev(unit_seqs, "unit_seqs") if U else None, _dev(unit_len, "unit_len") if U else None, U, W,
+        int(max_prefix_len), _dev(workspace, "workspace"), workspace.numel(), _dev(device_error, "device_error"),
+        _stream(stream))
+    _check(status, "paged_attn_decode_shared_prefix")
+    return out

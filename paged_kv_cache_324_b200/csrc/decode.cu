@@ -79,6 +79,13 @@ struct DecodeArgs {
     int block_size, partition_size, max_partitions;
     float qk_scale_log2;  // scale * k_scale * log2(e)
     float v_scale;        // 1 for 16-bit pools
+    // shared-prefix decode (all null / zero in the plain call)
+    const int32_t* seq_start;   // [S] first token each sequence attends in this pass (its shared prefix length)
+    const int32_t* unit_seqs;   // prefix pass: [units][unit_width] member sequences of each unit, -1 pads
+    const int32_t* unit_len;    // prefix pass: [units] shared tokens of each unit
+    int unit_width;
+    int slot_base;              // first partition slot of the workspace this pass writes
+    int prefix_partition_size;  // merge: partition size of the prefix pass
 };
 
 // ---- MMA and conversions ------------------------------------------------------
@@ -250,25 +257,52 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
     const uint32_t bar_empty = bar_full + NST * 8;
     volatile int* s_abort = reinterpret_cast<volatile int*>(gbase + Gm::kDataBytes + NST * 16);
 
-    const int part = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
+    const int part = blockIdx.x, kvh = blockIdx.y, z = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = a.num_heads / a.num_kv_heads;
     const int H = a.num_heads;
-    const int L = __ldg(a.context_lens + s);
-    const size_t out_row0 = static_cast<size_t>(s) * H + static_cast<size_t>(kvh) * G;
-
-    const bool bad_len = L < 0 || L > a.max_blocks_per_seq * BS || L > a.max_context_len;
-    const bool give_up = grid_timed_out(a.err);
-    if (bad_len || L == 0 || give_up) {
-        if (part == 0) {
-            pdl_wait();
-            if (bad_len && threadIdx.x == 0) raise_error(a.err, PKV_DEVERR_CONTEXT_LEN);
-            const float v = (bad_len || give_up) ? __int_as_float(0x7fc00000) : 0.f;
-            for (int e = threadIdx.x; e < G * D; e += kThreads)
-                store_out<kQBf16>(a.out, out_row0 * D + e, v);
+    // The CTA's query rows: the G heads of sequence z, or (prefix pass) the G heads of
+    // every member of prefix unit z.  Tokens [start, start + L) of table row `tseq`.
+    const bool prefix_pass = a.unit_seqs != nullptr;
+    int rows = G, L, start = 0, tseq = z;
+    bool bad_len;
+    if (prefix_pass) {
+        const int32_t* mem = a.unit_seqs + static_cast<size_t>(z) * a.unit_width;
+        tseq = __ldg(mem);
+        int members = 0;
+        for (int m = 0; m < a.unit_width; ++m) members += __ldg(mem + m) >= 0;
+        rows = members * G;
+        L = __ldg(a.unit_len + z);
+        bad_len = tseq < 0 || tseq >= a.num_seqs || L < 0 || L % BS != 0 || L > a.max_blocks_per_seq * BS;
+        if (bad_len || L == 0 || grid_timed_out(a.err)) {
+            if (bad_len && part == 0 && threadIdx.x == 0) raise_error(a.err, PKV_DEVERR_CONTEXT_LEN);
+            return;   // members' merges see a bad or empty prefix and answer for it
         }
-        return;
+    } else {
+        const int Lt = __ldg(a.context_lens + z);
+        start = a.seq_start ? __ldg(a.seq_start + z) : 0;
+        bad_len = Lt < 0 || Lt > a.max_blocks_per_seq * BS || Lt > a.max_context_len || start < 0 || start > Lt ||
+                  start % BS != 0;
+        L = Lt - start;
+        const bool give_up = grid_timed_out(a.err);
+        if (bad_len || L == 0 || give_up) {
+            if (part == 0 && (start == 0 || bad_len)) {
+                pdl_wait();
+                if (bad_len && threadIdx.x == 0) raise_error(a.err, PKV_DEVERR_CONTEXT_LEN);
+                const float v = (bad_len || give_up) ? __int_as_float(0x7fc00000) : 0.f;
+                const size_t row0 = static_cast<size_t>(z) * H + static_cast<size_t>(kvh) * G;
+                for (int e = threadIdx.x; e < G * D; e += kThreads) store_out<kQBf16>(a.out, row0 * D + e, v);
+            }
+            return;
+        }
     }
+    // global q / out row of CTA row r
+    auto row_of = [&](int r) -> size_t {
+        if (!prefix_pass) return static_cast<size_t>(z) * H + static_cast<size_t>(kvh) * G + r;
+        const int m = r / G;
+        return static_cast<size_t>(__ldg(a.unit_seqs + static_cast<size_t>(z) * a.unit_width + m)) * H +
+               static_cast<size_t>(kvh) * G + (r - m * G);
+    };
     const int PS = a.partition_size;
     const int nparts = (L + PS - 1) / PS;
     if (part >= nparts) return;
@@ -276,7 +310,7 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
     const int tok_end = min(L, tok_begin + PS);
     const int nblk = (tok_end - tok_begin + BS - 1) / BS;
     const int nstage = (nblk + Gm::kBps - 1) / Gm::kBps;
-    const int blk0 = tok_begin / BS;
+    const int blk0 = (start + tok_begin) / BS;
 
     if (threadIdx.x == 0) {
 #pragma unroll
@@ -311,7 +345,7 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
             tma_prefetch_desc(&vmap);
         }
         const uint64_t pol = l2_policy_evict_first();
-        const int32_t* table = a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq + blk0;
+        const int32_t* table = a.block_tables + static_cast<size_t>(tseq) * a.max_blocks_per_seq + blk0;
         bool ok = true;
         int issued = 0;   // stages issued
         constexpr int kChunk = 32 / Gm::kBps * Gm::kBps;   // table entries per warp-wide load
@@ -383,9 +417,9 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
 #pragma unroll
         for (int nh = 0; nh < NTH; ++nh) {
             const int hq = nh * 8 + r;
-            const bool ok = hq < G;
+            const bool ok = hq < rows;
             const uint32_t* qrow = reinterpret_cast<const uint32_t*>(static_cast<const uint16_t*>(a.q) +
-                                                                     (out_row0 + (ok ? hq : 0)) * D);
+                                                                     row_of(ok ? hq : 0) * D);
 #pragma unroll
             for (int ks = 0; ks < Gm::kKsteps; ++ks) {
                 const int d0 = Gm::qk_dim(c, ks);
@@ -619,8 +653,8 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
     }
     __syncthreads();
     const bool aborted = *s_abort != 0;
-    const bool single = nparts == 1;
-    for (int e = threadIdx.x; e < G * D; e += kThreads) {
+    const bool single = nparts == 1 && start == 0 && !prefix_pass;   // otherwise partials for the merge
+    for (int e = threadIdx.x; e < rows * D; e += kThreads) {
         const int hh = e / D, d = e - hh * D;
         float M = -INFINITY;
 #pragma unroll
@@ -635,9 +669,9 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
         float val = num / den * a.v_scale;
         if (aborted) val = __int_as_float(0x7fc00000);
         if (single) {
-            store_out<kQBf16>(a.out, (out_row0 + hh) * D + d, val);
+            store_out<kQBf16>(a.out, row_of(hh) * D + d, val);
         } else {
-            const size_t slot = (out_row0 + hh) * a.max_partitions + part;
+            const size_t slot = row_of(hh) * a.max_partitions + a.slot_base + part;
             a.ws_o[slot * D + d] = val;
             if (d == 0) a.ws_ml[slot] = make_float2(aborted ? __int_as_float(0x7fc00000) : M, den);
         }
@@ -656,14 +690,25 @@ __global__ void __launch_bounds__(D) decode_reduce_kernel(const DecodeArgs a) {
     pdl_wait();
     const int qh = blockIdx.x, s = blockIdx.y, d = threadIdx.x;
     const int L = __ldg(a.context_lens + s);
-    if (L <= 0 || L > a.max_blocks_per_seq * a.block_size || L > a.max_context_len) return;
-    const int np = (L + a.partition_size - 1) / a.partition_size;
-    if (np <= 1) return;
+    const int PS = a.partition_size;
+    // partials of a sequence: its prefix partitions in slots [0, np_pre) (shared-prefix
+    // call only), then its own partitions from slot a.slot_base on
+    const int start = a.seq_start ? __ldg(a.seq_start + s) : 0;
     const size_t row = static_cast<size_t>(s) * a.num_heads + qh;
-    if (grid_timed_out(a.err)) {   // pass 1 gave up somewhere: its partials are not to be trusted
+    if (L < 0 || L > a.max_blocks_per_seq * a.block_size || L > a.max_context_len || start < 0 || start > L ||
+        start % a.block_size != 0) {
+        if (start > 0) store_out<kQBf16>(a.out, row * D + d, __int_as_float(0x7fc00000));
+        return;   // (a sequence without a prefix got its NaN from pass 1)
+    }
+    const int np_pre = start > 0 ? (start + a.prefix_partition_size - 1) / a.prefix_partition_size : 0;
+    const int np_tail = (L - start + PS - 1) / PS;
+    const int np = np_pre + np_tail;
+    if (np_pre == 0 && np_tail <= 1) return;   // written by pass 1
+    if (grid_timed_out(a.err)) {   // a pass gave up somewhere: its partials are not to be trusted
         store_out<kQBf16>(a.out, row * D + d, __int_as_float(0x7fc00000));
         return;
     }
+    auto slot = [&](int p) { return p < np_pre ? p : a.slot_base + (p - np_pre); };
     const float2* ml = a.ws_ml + row * a.max_partitions;
     const float* wo = a.ws_o + row * a.max_partitions * D;
     if (np <= 8) {   // few partitions: every thread reads the pairs itself, all loads at once
@@ -672,8 +717,8 @@ __global__ void __launch_bounds__(D) decode_reduce_kernel(const DecodeArgs a) {
 #pragma unroll
         for (int p = 0; p < 8; ++p)
             if (p < np) {
-                v[p] = ml[p];
-                o[p] = wo[static_cast<size_t>(p) * D + d];
+                v[p] = ml[slot(p)];
+                o[p] = wo[static_cast<size_t>(slot(p)) * D + d];
             }
         float M = -INFINITY;
 #pragma unroll
@@ -693,7 +738,7 @@ __global__ void __launch_bounds__(D) decode_reduce_kernel(const DecodeArgs a) {
     float* red = sw + a.max_partitions;
     // M = max_p m_p
     float mx = -INFINITY;
-    for (int p = d; p < np; p += D) mx = fmaxf(mx, ml[p].x);
+    for (int p = d; p < np; p += D) mx = fmaxf(mx, ml[slot(p)].x);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     if ((d & 31) == 0) red[d >> 5] = mx;
@@ -704,7 +749,7 @@ __global__ void __launch_bounds__(D) decode_reduce_kernel(const DecodeArgs a) {
     // weights and their sum
     float den = 0.f;
     for (int p = d; p < np; p += D) {
-        const float2 v = ml[p];
+        const float2 v = ml[slot(p)];
         const float w = exp2f(v.x - M) * v.y;
         sw[p] = w;
         den += w;
@@ -723,11 +768,11 @@ __global__ void __launch_bounds__(D) decode_reduce_kernel(const DecodeArgs a) {
     for (; p + 8 <= np; p += 8) {
         float o[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) o[i] = wo[static_cast<size_t>(p + i) * D + d];
+        for (int i = 0; i < 8; ++i) o[i] = wo[static_cast<size_t>(slot(p + i)) * D + d];
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] += sw[p + i] * o[i];
     }
-    for (; p < np; ++p) acc[0] += sw[p] * wo[static_cast<size_t>(p) * D + d];
+    for (; p < np; ++p) acc[0] += sw[p] * wo[static_cast<size_t>(slot(p)) * D + d];
     const float num = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
     store_out<kQBf16>(a.out, row * D + d, num / total);
 }
@@ -779,36 +824,128 @@ bool encode_pool_map(CUtensorMap* map, const void* pool, int kv_dtype, int head_
 }
 
 template <int KV, bool kQBf16, int D, int BS, bool kHi>
-pkv_status launch_decode(const DecodeArgs& a, const CUtensorMap& km, const CUtensorMap& vm,
-                         cudaStream_t st) {
+pkv_status launch_pass1(const DecodeArgs& a, const CUtensorMap& km, const CUtensorMap& vm, unsigned gx, unsigned gz,
+                        cudaStream_t st) {
     using Gm = Geo<KV, D, BS, kHi>;
     auto kern = paged_decode_kernel<KV, kQBf16, D, BS, kHi>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Gm::kSmemBytes) != cudaSuccess)
         return PKV_ERR_CUDA;
-    dim3 grid(a.max_partitions, a.num_kv_heads, a.num_seqs);
-    if (launch_pdl(kern, grid, dim3(kThreads), Gm::kSmemBytes, st, a, km, vm) != cudaSuccess) return PKV_ERR_CUDA;
-    if (a.max_partitions > 1) {
-        const size_t rsmem = (static_cast<size_t>(a.max_partitions) + D / 32) * sizeof(float);
-        auto rk = decode_reduce_kernel<kQBf16, D>;
-        if (rsmem > 48 * 1024 &&
-            cudaFuncSetAttribute(rk, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(rsmem)) !=
-                cudaSuccess)
-            return PKV_ERR_CUDA;
-        if (launch_pdl(rk, dim3(a.num_heads, a.num_seqs), dim3(D), rsmem, st, a) != cudaSuccess)
-            return PKV_ERR_CUDA;
-        if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
+    const dim3 grid(gx, static_cast<unsigned>(a.num_kv_heads), gz);
+    return launch_pdl(kern, grid, dim3(kThreads), Gm::kSmemBytes, st, a, km, vm) == cudaSuccess ? PKV_OK
+                                                                                                : PKV_ERR_CUDA;
+}
+
+template <bool kQBf16, int D>
+pkv_status launch_merge(const DecodeArgs& a, cudaStream_t st) {
+    const size_t rsmem = (static_cast<size_t>(a.max_partitions) + D / 32) * sizeof(float);
+    auto rk = decode_reduce_kernel<kQBf16, D>;
+    if (rsmem > 48 * 1024 &&
+        cudaFuncSetAttribute(rk, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(rsmem)) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    return launch_pdl(rk, dim3(a.num_heads, a.num_seqs), dim3(D), rsmem, st, a) == cudaSuccess ? PKV_OK
+                                                                                               : PKV_ERR_CUDA;
+}
+
+struct Pass1 {
+    const DecodeArgs& a;
+    const CUtensorMap& km;
+    const CUtensorMap& vm;
+    unsigned gx, gz;
+    cudaStream_t st;
+    template <int KV, bool QB, int D, int BS, bool HI>
+    pkv_status run() const { return launch_pass1<KV, QB, D, BS, HI>(a, km, vm, gx, gz, st); }
+};
+
+struct Merge {
+    const DecodeArgs& a;
+    cudaStream_t st;
+    template <int KV, bool QB, int D, int BS, bool HI>
+    pkv_status run() const { return launch_merge<QB, D>(a, st); }
+};
+
+template <int KV, bool QB, int D, class F>
+pkv_status with_bs(int bs, bool hi, const F& f) {
+    if (bs == 16) return hi ? f.template run<KV, QB, D, 16, true>() : f.template run<KV, QB, D, 16, false>();
+    return hi ? f.template run<KV, QB, D, 32, true>() : f.template run<KV, QB, D, 32, false>();
+}
+
+// Calls f.run<...>() for the kernel instance of these (validated) arguments.
+template <class F>
+pkv_status with_instance(pkv_dtype kv, pkv_dtype qd, int D, int bs, bool hi, const F& f) {
+    switch (kv) {
+    case PKV_F16:
+        return D == 64 ? with_bs<KV_F16, false, 64>(bs, hi, f) : with_bs<KV_F16, false, 128>(bs, hi, f);
+    case PKV_BF16:
+        return D == 64 ? with_bs<KV_BF16, true, 64>(bs, hi, f) : with_bs<KV_BF16, true, 128>(bs, hi, f);
+    case PKV_FP8_E4M3:
+        return qd == PKV_BF16 ? with_bs<KV_E4M3, true, 128>(bs, hi, f) : with_bs<KV_E4M3, false, 128>(bs, hi, f);
     }
+    return PKV_ERR_UNSUPPORTED;
+}
+
+// Checks shared by the decode entry points (host-visible arguments only).
+pkv_status validate(const void* out, const void* q, pkv_dtype q_dtype, const void* k_pool, const void* v_pool,
+                    pkv_dtype kv_dtype, float k_scale, float v_scale, const int32_t* block_tables,
+                    int max_blocks_per_seq, const int32_t* context_lens, int max_context_len, int num_seqs,
+                    int num_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale,
+                    int partition_size) {
+    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        num_blocks <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0 || partition_size < 0)
+        return PKV_ERR_INVALID_ARG;
+    if (num_heads % num_kv_heads != 0) return PKV_ERR_INVALID_ARG;
+    if (!(scale == scale)) return PKV_ERR_INVALID_ARG;
+    if (num_heads / num_kv_heads > 16) return PKV_ERR_UNSUPPORTED;
+    if (block_size != 16 && block_size != 32) return PKV_ERR_UNSUPPORTED;
+    if (partition_size % block_size != 0) return PKV_ERR_INVALID_ARG;
+    if (q_dtype != PKV_F16 && q_dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
+    if (kv_dtype != q_dtype && kv_dtype != PKV_FP8_E4M3) return PKV_ERR_UNSUPPORTED;
+    if (kv_dtype == PKV_FP8_E4M3) {
+        if (head_dim != 128) return PKV_ERR_UNSUPPORTED;
+        if (!(k_scale > 0.f && v_scale > 0.f)) return PKV_ERR_INVALID_ARG;
+    } else if (head_dim != 64 && head_dim != 128) {
+        return PKV_ERR_UNSUPPORTED;
+    }
+    if (num_seqs > 65535 || num_kv_heads > 65535) return PKV_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return PKV_OK;
+    if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens) return PKV_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) ||
+        (reinterpret_cast<uintptr_t>(block_tables) & 3) || (reinterpret_cast<uintptr_t>(context_lens) & 3))
+        return PKV_ERR_ALIGNMENT;
     return PKV_OK;
 }
 
-template <int KV, bool kQBf16, int D>
-pkv_status dispatch_bs(const DecodeArgs& a, const CUtensorMap& km, const CUtensorMap& vm, cudaStream_t st,
-                       bool hi) {
-    if (a.block_size == 16)
-        return hi ? launch_decode<KV, kQBf16, D, 16, true>(a, km, vm, st)
-                  : launch_decode<KV, kQBf16, D, 16, false>(a, km, vm, st);
-    return hi ? launch_decode<KV, kQBf16, D, 32, true>(a, km, vm, st)
-              : launch_decode<KV, kQBf16, D, 32, false>(a, km, vm, st);
+DecodeArgs base_args(void* out, const void* q, const int32_t* block_tables, int max_blocks_per_seq,
+                     const int32_t* context_lens, int max_context_len, int num_seqs, int num_heads,
+                     int num_kv_heads, int num_blocks, int block_size, pkv_dtype kv_dtype, float k_scale,
+                     float v_scale, float scale, int ps, uint32_t* device_error) {
+    DecodeArgs a{};
+    a.out = out;
+    a.q = q;
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    a.err = device_error;
+    a.max_blocks_per_seq = max_blocks_per_seq;
+    a.max_context_len = max_context_len;
+    a.num_seqs = num_seqs;
+    a.num_heads = num_heads;
+    a.num_kv_heads = num_kv_heads;
+    a.num_blocks = num_blocks;
+    a.block_size = block_size;
+    a.partition_size = ps;
+    const float ks = kv_dtype == PKV_FP8_E4M3 ? k_scale : 1.f;
+    a.qk_scale_log2 = static_cast<float>(static_cast<double>(scale) * ks * 1.4426950408889634);
+    a.v_scale = kv_dtype == PKV_FP8_E4M3 ? v_scale : 1.f;
+    return a;
+}
+
+size_t partials_bytes(size_t rows, int head_dim) {
+    return (rows * head_dim * sizeof(float) + 255) / 256 * 256 + rows * sizeof(float2);
+}
+
+void set_partials(DecodeArgs& a, void* workspace, size_t rows, int head_dim) {
+    a.ws_o = static_cast<float*>(workspace);
+    a.ws_ml = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) +
+                                        (rows * head_dim * sizeof(float) + 255) / 256 * 256);
 }
 
 }  // namespace
@@ -831,9 +968,7 @@ extern "C" size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int nu
     if (ps <= 0 || num_heads <= 0 || head_dim <= 0) return 0;
     const long long parts = (static_cast<long long>(max_context_len) + ps - 1) / ps;
     if (parts <= 1) return 0;
-    const size_t rows = static_cast<size_t>(num_seqs) * num_heads * static_cast<size_t>(parts);
-    const size_t o_bytes = (rows * head_dim * sizeof(float) + 255) / 256 * 256;
-    return o_bytes + rows * sizeof(float2);
+    return pkv::partials_bytes(static_cast<size_t>(num_seqs) * num_heads * static_cast<size_t>(parts), head_dim);
 }
 
 extern "C" pkv_status pkv_paged_attn_decode(void* out, const void* q, pkv_dtype q_dtype, const void* k_pool,
@@ -844,30 +979,10 @@ extern "C" pkv_status pkv_paged_attn_decode(void* out, const void* q, pkv_dtype 
                                             int num_blocks, float scale, int partition_size, void* workspace,
                                             size_t workspace_bytes, uint32_t* device_error, void* stream) {
     using namespace pkv;
-    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
-        num_blocks <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0 || partition_size < 0)
-        return PKV_ERR_INVALID_ARG;
-    if (num_heads % num_kv_heads != 0) return PKV_ERR_INVALID_ARG;
-    if (!(scale == scale)) return PKV_ERR_INVALID_ARG;
-    const int G = num_heads / num_kv_heads;
-    if (G > 16) return PKV_ERR_UNSUPPORTED;
-    if (block_size != 16 && block_size != 32) return PKV_ERR_UNSUPPORTED;
-    if (partition_size % block_size != 0) return PKV_ERR_INVALID_ARG;
-    if (q_dtype != PKV_F16 && q_dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
-    if (kv_dtype != q_dtype && kv_dtype != PKV_FP8_E4M3) return PKV_ERR_UNSUPPORTED;
-    if (kv_dtype == PKV_FP8_E4M3) {
-        if (head_dim != 128) return PKV_ERR_UNSUPPORTED;
-        if (!(k_scale > 0.f && v_scale > 0.f)) return PKV_ERR_INVALID_ARG;
-    } else if (head_dim != 64 && head_dim != 128) {
-        return PKV_ERR_UNSUPPORTED;
-    }
-    if (num_seqs > 65535 || num_kv_heads > 65535) return PKV_ERR_UNSUPPORTED;
-    if (num_seqs == 0) return PKV_OK;
-    if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens) return PKV_ERR_INVALID_ARG;
-    if (!aligned16(out) || !aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) ||
-        (reinterpret_cast<uintptr_t>(block_tables) & 3) || (reinterpret_cast<uintptr_t>(context_lens) & 3))
-        return PKV_ERR_ALIGNMENT;
-
+    const pkv_status v = validate(out, q, q_dtype, k_pool, v_pool, kv_dtype, k_scale, v_scale, block_tables,
+                                  max_blocks_per_seq, context_lens, max_context_len, num_seqs, num_heads,
+                                  num_kv_heads, head_dim, block_size, num_blocks, scale, partition_size);
+    if (v != PKV_OK || num_seqs == 0) return v;
     const int ps = pick_partition(num_seqs, num_kv_heads, head_dim, kv_dtype == PKV_FP8_E4M3 ? 1 : 2, block_size,
                                   max_context_len, partition_size);
     const int parts = max_context_len > 0 ? (max_context_len + ps - 1) / ps : 1;
@@ -876,51 +991,119 @@ extern "C" pkv_status pkv_paged_attn_decode(void* out, const void* q, pkv_dtype 
     if (need > 0 && (!workspace || workspace_bytes < need)) return PKV_ERR_WORKSPACE;
     if (need > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255)) return PKV_ERR_ALIGNMENT;
 
-    DecodeArgs a{};
-    a.out = out;
-    a.q = q;
-    a.block_tables = block_tables;
-    a.context_lens = context_lens;
-    const size_t rows = static_cast<size_t>(num_seqs) * num_heads * static_cast<size_t>(parts);
-    a.ws_o = need ? static_cast<float*>(workspace) : nullptr;
-    a.ws_ml = need ? reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) +
-                                               (rows * head_dim * sizeof(float) + 255) / 256 * 256)
-                   : nullptr;
-    a.err = device_error;
-    a.max_blocks_per_seq = max_blocks_per_seq;
-    a.max_context_len = max_context_len;
-    a.num_seqs = num_seqs;
-    a.num_heads = num_heads;
-    a.num_kv_heads = num_kv_heads;
-    a.num_blocks = num_blocks;
-    a.block_size = block_size;
-    a.partition_size = ps;
+    DecodeArgs a = base_args(out, q, block_tables, max_blocks_per_seq, context_lens, max_context_len, num_seqs,
+                             num_heads, num_kv_heads, num_blocks, block_size, kv_dtype, k_scale, v_scale, scale, ps,
+                             device_error);
     a.max_partitions = parts;
-    const float ks = kv_dtype == PKV_FP8_E4M3 ? k_scale : 1.f;
-    a.qk_scale_log2 = static_cast<float>(static_cast<double>(scale) * ks * 1.4426950408889634);
-    a.v_scale = kv_dtype == PKV_FP8_E4M3 ? v_scale : 1.f;
+    if (need) set_partials(a, workspace, static_cast<size_t>(num_seqs) * num_heads * parts, head_dim);
 
     alignas(64) CUtensorMap km;
     alignas(64) CUtensorMap vm;
     if (!encode_pool_map(&km, k_pool, kv_dtype, head_dim, block_size, num_kv_heads, num_blocks) ||
         !encode_pool_map(&vm, v_pool, kv_dtype, head_dim, block_size, num_kv_heads, num_blocks))
         return PKV_ERR_CUDA;
-
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const bool hi = G > 8;
-    const bool qbf = q_dtype == PKV_BF16;
-    switch (kv_dtype) {
-    case PKV_F16:
-        return head_dim == 64 ? dispatch_bs<KV_F16, false, 64>(a, km, vm, st, hi)
-                              : dispatch_bs<KV_F16, false, 128>(a, km, vm, st, hi);
-    case PKV_BF16:
-        return head_dim == 64 ? dispatch_bs<KV_BF16, true, 64>(a, km, vm, st, hi)
-                              : dispatch_bs<KV_BF16, true, 128>(a, km, vm, st, hi);
-    case PKV_FP8_E4M3:
-        return qbf ? dispatch_bs<KV_E4M3, true, 128>(a, km, vm, st, hi)
-                   : dispatch_bs<KV_E4M3, false, 128>(a, km, vm, st, hi);
+    const bool hi = num_heads / num_kv_heads > 8;
+    pkv_status r = with_instance(kv_dtype, q_dtype, head_dim, block_size, hi,
+                                 Pass1{a, km, vm, static_cast<unsigned>(parts), static_cast<unsigned>(num_seqs), st});
+    if (r == PKV_OK && parts > 1) r = with_instance(kv_dtype, q_dtype, head_dim, block_size, hi, Merge{a, st});
+    return r;
+}
+
+// ---- shared-prefix decode -----------------------------------------------------------------
+
+namespace pkv {
+namespace {
+// The prefix pass is partitioned on its own: it has one work unit per (unit, KV head)
+// and partition, so its partitions shrink until the SMs have enough of them.
+int prefix_partition(int num_units, int num_kv_heads, int head_dim, pkv_dtype kv_dtype, int block_size,
+                     int max_prefix_len, int partition_size) {
+    if (max_prefix_len <= 0) return block_size;
+    return pkv_decode_partition_size(num_units > 0 ? num_units : 1, num_kv_heads, head_dim, kv_dtype, block_size,
+                                     max_prefix_len, partition_size);
+}
+}  // namespace
+}  // namespace pkv
+
+extern "C" size_t pkv_shared_prefix_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                                    pkv_dtype kv_dtype, int block_size, int max_context_len,
+                                                    int num_units, int max_prefix_len, int partition_size) {
+    const int ps = pkv_decode_partition_size(num_seqs, num_kv_heads, head_dim, kv_dtype, block_size,
+                                             max_context_len, partition_size);
+    if (ps <= 0 || num_heads <= 0 || head_dim <= 0 || max_prefix_len < 0 || max_prefix_len > max_context_len)
+        return 0;
+    const int ps_pre = pkv::prefix_partition(num_units, num_kv_heads, head_dim, kv_dtype, block_size, max_prefix_len,
+                                             partition_size);
+    if (ps_pre <= 0) return 0;
+    const int parts = (max_prefix_len + ps_pre - 1) / ps_pre + (max_context_len + ps - 1) / ps;
+    return pkv::partials_bytes(static_cast<size_t>(num_seqs) * num_heads * static_cast<size_t>(parts), head_dim);
+}
+
+extern "C" pkv_status pkv_paged_attn_decode_shared_prefix(
+    void* out, const void* q, pkv_dtype q_dtype, const void* k_pool, const void* v_pool, pkv_dtype kv_dtype,
+    float k_scale, float v_scale, const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+    int max_context_len, int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+    int num_blocks, float scale, int partition_size, const int32_t* seq_prefix_len, const int32_t* unit_seqs,
+    const int32_t* unit_len, int num_units, int unit_width, int max_prefix_len, void* workspace,
+    size_t workspace_bytes, uint32_t* device_error, void* stream) {
+    using namespace pkv;
+    const pkv_status v = validate(out, q, q_dtype, k_pool, v_pool, kv_dtype, k_scale, v_scale, block_tables,
+                                  max_blocks_per_seq, context_lens, max_context_len, num_seqs, num_heads,
+                                  num_kv_heads, head_dim, block_size, num_blocks, scale, partition_size);
+    if (v != PKV_OK || num_seqs == 0) return v;
+    const int G = num_heads / num_kv_heads;
+    if (num_units < 0 || num_units > 65535 || unit_width <= 0 || max_prefix_len < 0 ||
+        max_prefix_len > max_context_len || max_prefix_len % block_size != 0)
+        return PKV_ERR_INVALID_ARG;
+    if (unit_width * G > 16) return PKV_ERR_UNSUPPORTED;
+    if (!seq_prefix_len || (num_units > 0 && (!unit_seqs || !unit_len))) return PKV_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(seq_prefix_len) & 3) || (reinterpret_cast<uintptr_t>(unit_seqs) & 3) ||
+        (reinterpret_cast<uintptr_t>(unit_len) & 3))
+        return PKV_ERR_ALIGNMENT;
+    const int ps = pick_partition(num_seqs, num_kv_heads, head_dim, kv_dtype == PKV_FP8_E4M3 ? 1 : 2, block_size,
+                                  max_context_len, partition_size);
+    const int ps_pre = prefix_partition(num_units, num_kv_heads, head_dim, kv_dtype, block_size, max_prefix_len,
+                                        partition_size);
+    const int p_pre = (max_prefix_len + ps_pre - 1) / ps_pre;
+    const int p_tail = max_context_len > 0 ? (max_context_len + ps - 1) / ps : 1;
+    const size_t need = pkv_shared_prefix_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, kv_dtype,
+                                                          block_size, max_context_len, num_units, max_prefix_len,
+                                                          partition_size);
+    if (!workspace || workspace_bytes < need) return PKV_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255) return PKV_ERR_ALIGNMENT;
+
+    DecodeArgs a = base_args(out, q, block_tables, max_blocks_per_seq, context_lens, max_context_len, num_seqs,
+                             num_heads, num_kv_heads, num_blocks, block_size, kv_dtype, k_scale, v_scale, scale, ps,
+                             device_error);
+    a.max_partitions = p_pre + p_tail;
+    set_partials(a, workspace, static_cast<size_t>(num_seqs) * num_heads * a.max_partitions, head_dim);
+
+    alignas(64) CUtensorMap km;
+    alignas(64) CUtensorMap vm;
+    if (!encode_pool_map(&km, k_pool, kv_dtype, head_dim, block_size, num_kv_heads, num_blocks) ||
+        !encode_pool_map(&vm, v_pool, kv_dtype, head_dim, block_size, num_kv_heads, num_blocks))
+        return PKV_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    pkv_status r = PKV_OK;
+    if (num_units > 0 && p_pre > 0) {   // shared tokens: every unit's rows against its prefix, once
+        DecodeArgs ap = a;
+        ap.partition_size = ps_pre;
+        ap.unit_seqs = unit_seqs;
+        ap.unit_len = unit_len;
+        ap.unit_width = unit_width;
+        ap.slot_base = 0;
+        r = with_instance(kv_dtype, q_dtype, head_dim, block_size, unit_width * G > 8,
+                          Pass1{ap, km, vm, static_cast<unsigned>(p_pre), static_cast<unsigned>(num_units), st});
     }
-    return PKV_ERR_UNSUPPORTED;
+    DecodeArgs at = a;   // each sequence's own tokens, from the end of its prefix
+    at.seq_start = seq_prefix_len;
+    at.slot_base = p_pre;
+    at.prefix_partition_size = ps_pre;
+    if (r == PKV_OK)
+        r = with_instance(kv_dtype, q_dtype, head_dim, block_size, G > 8,
+                          Pass1{at, km, vm, static_cast<unsigned>(p_tail), static_cast<unsigned>(num_seqs), st});
+    if (r == PKV_OK) r = with_instance(kv_dtype, q_dtype, head_dim, block_size, G > 8, Merge{at, st});
+    return r;
 }
 
 // ---- decode with a library-owned workspace (no allocation by the caller) ------------

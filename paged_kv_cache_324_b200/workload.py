@@ -313,7 +313,7 @@ def make(name: str, small: bool = False) -> DecodeWorkload:
     pool cut down to the blocks in use plus 64, which keeps profiler captures small."""
     if name.endswith("_compact"):
         w = make(name[: -len("_compact")], small)
-        if w.name == "prefix":
+        if w.name.startswith("prefix"):
             raise KeyError(name)
         nblk = int(((w.context_lens.astype(np.int64) + w.block_size - 1) // w.block_size).sum())
         rng = np.random.default_rng(w.seed)
@@ -350,6 +350,13 @@ def make(name: str, small: bool = False) -> DecodeWorkload:
             prefix_blocks=32, tail_max=tail_max,
             description=f"shared-prefix sampling: {prompts} prompts x 8 samples, 32 q / 8 KV heads, "
                         f"head_dim 128, fp16, 512+r token prompts, tails U[1,{tail_max}]")
+    if name == "prefix_long":
+        prompts, tail_max, pblocks = (2, 100, 80) if small else (16, 256, 256)
+        return shared_prefix_sampling(
+            "prefix_long", 5, prompts, 8, 32, 8, 128, 16, 8192 if not small else 1024, "f16",
+            prefix_blocks=pblocks, tail_max=tail_max,
+            description=f"long shared prompts: {prompts} prompts x 8 samples, 32 q / 8 KV heads, head_dim 128, "
+                        f"fp16, {pblocks * 16}+r token prompts, tails U[1,{tail_max}]")
     if name in ("fp8", "fp8_b32"):
         B = 32 if name == "fp8_b32" else 16
         S, L = (4, 3000) if small else (16, 32768)
@@ -363,6 +370,7 @@ def make(name: str, small: bool = False) -> DecodeWorkload:
 
 
 NAMES = ("tiny", "opt13b", "gqa", "prefix", "fp8", "fp8_b32")
+EXTRA_NAMES = ("prefix_long",)
 COMPACT_NAMES = tuple(n + "_compact" for n in NAMES if n != "prefix")
 
 
@@ -382,6 +390,21 @@ def decode_algorithmic_bytes(w: DecodeWorkload) -> int:
     qo = 2 * w.num_seqs * w.num_heads * w.head_dim * ELEM_BYTES[w.q_dtype]
     nblk = int(((w.context_lens.astype(np.int64) + w.block_size - 1) // w.block_size).sum())
     return kv + qo + 4 * nblk + 4 * w.num_seqs
+
+
+def decode_distinct_bytes(w: DecodeWorkload) -> int:
+    """decode_algorithmic_bytes with each physical KV slot counted once, however many
+    sequences attend to it: the least a decode call over shared blocks has to read."""
+    B = w.block_size
+    slots = []
+    for s in range(w.num_seqs):
+        L = int(w.context_lens[s])
+        p = np.arange(L, dtype=np.int64)
+        slots.append(w.block_tables[s, p // B].astype(np.int64) * B + p % B)
+    n = int(np.unique(np.concatenate(slots)).size) if slots else 0
+    kv = n * kv_bytes_per_token(1, w.num_kv_heads, w.head_dim, ELEM_BYTES[w.kv_dtype])
+    return decode_algorithmic_bytes(w) - int(w.context_lens.astype(np.int64).sum()) * kv_bytes_per_token(
+        1, w.num_kv_heads, w.head_dim, ELEM_BYTES[w.kv_dtype]) + kv
 
 
 def scatter_algorithmic_bytes(w: DecodeWorkload, sc: Scatter) -> int:
