@@ -45,8 +45,12 @@ FALLBACK_HBM_GBS = 6650.0
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by workload, valid only
 # for the decode kernel source it was measured on (sha256 prefix of decode.cu).
 NCU_TRAFFIC = {
-    "opt13b": {"bytes_per_launch": 1_319_549_000, "kernel_sha": "640cda3584e49b53",
+    "opt13b": {"bytes_per_launch": 1_316_705_536, "kernel_sha": "50dd0cd8f2ba18ba",
                "capture": "profiles/paged_decode_kernel_opt13b.md (opt13b_compact: same sequences)"},
+    "gqa": {"bytes_per_launch": 1_224_799_136, "kernel_sha": "50dd0cd8f2ba18ba",
+            "capture": "profiles/paged_decode_kernel_gqa.md (gqa_compact: same sequences)"},
+    "fp8": {"bytes_per_launch": 1_118_479_160, "kernel_sha": "50dd0cd8f2ba18ba",
+            "capture": "profiles/paged_decode_kernel_fp8.md (fp8_compact: same sequences, 512-token partitions)"},
 }
 
 
@@ -340,7 +344,9 @@ def run_ours(args, rank, world, local_rank):
     achieved = roof_bytes / (dec_avg * 1e-3) / 1e9
     traffic = None
     tr = NCU_TRAFFIC.get(args.config)
-    if tr and tr.get("kernel_sha") == decode_source_sha():
+    # the capture ran the plain decode at the workload's own partition size
+    if (tr and tr.get("kernel_sha") == decode_source_sha() and args.partition == "config"
+            and not args.prefix_aware):
         traffic = tr["bytes_per_launch"]
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
