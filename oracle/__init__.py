@@ -2,7 +2,7 @@
 
 Python access to the float64 CPU oracle in ``pagedkv_oracle.c``: the plain
 definition of paged decode attention (gather through the block table, then
-textbook two-pass softmax), the scatter of new tokens into the pool, the
+textbook two-pass softmax) and of chunked prefill over the same cache, the scatter of new tokens into the pool, the
 block copy used for copy-on-write, and the number-format codecs.
 
 Only the test suite, ``__graft_entry__.smoke()`` and the benchmark's CPU
@@ -58,6 +58,8 @@ def _load():
         P, I, D, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_float, ctypes.c_size_t
         lib.orc_paged_attn_decode.argtypes = [P, P, I, P, P, I, D, D, P, I, P, I, I, I, I, I, I, D, I]
         lib.orc_paged_attn_decode.restype = I
+        lib.orc_paged_attn_prefill.argtypes = [P, P, I, P, P, I, D, D, P, I, P, P, I, I, I, I, I, I, D, I]
+        lib.orc_paged_attn_prefill.restype = I
         lib.orc_reshape_and_cache.argtypes = [P, P, I, P, P, I, F, F, P, I, I, I, I, I]
         lib.orc_reshape_and_cache.restype = I
         lib.orc_copy_blocks.argtypes = [P, P, Z, P, I, I]
@@ -124,6 +126,35 @@ def paged_attn_decode(q_bits, q_dtype, k_pool, v_pool, kv_dtype, block_tables, c
         _ptr(out), _ptr(q_bits), _code(q_dtype), _ptr(k_pool), _ptr(v_pool), _code(kv_dtype),
         float(k_scale), float(v_scale), _ptr(block_tables), block_tables.shape[1],
         _ptr(context_lens), S, H, Hkv, D, B, NB, float(scale), int(threads)))
+    return out
+
+
+def paged_attn_prefill(q_bits, q_dtype, k_pool, v_pool, kv_dtype, block_tables, context_lens,
+                       query_start, scale, k_scale=1.0, v_scale=1.0, threads=0) -> np.ndarray:
+    """float64 out[T, H, D] of chunked prefill over the paged pool.
+
+    q_bits: uint16 [T, H, D], the chunks of all sequences packed in order;
+    query_start: int32 [S + 1], row offsets of each sequence's chunk (starts at
+    0, ends at T); context_lens int32 [S] count the chunk's tokens, which are
+    already in the pool.  Row query_start[s] + j attends to positions
+    0 .. context_lens[s] - C_s + j of sequence s.
+    """
+    q_bits = np.ascontiguousarray(q_bits)
+    k_pool = np.ascontiguousarray(k_pool)
+    v_pool = np.ascontiguousarray(v_pool)
+    block_tables = np.ascontiguousarray(block_tables, dtype=np.int32)
+    context_lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+    query_start = np.ascontiguousarray(query_start, dtype=np.int32)
+    T, H, D = q_bits.shape
+    NB, Hkv, B, D2 = k_pool.shape
+    S = context_lens.shape[0]
+    assert D2 == D and v_pool.shape == k_pool.shape
+    assert query_start.shape == (S + 1,) and int(query_start[-1]) == T
+    out = np.empty((T, H, D), np.float64)
+    _check(_load().orc_paged_attn_prefill(
+        _ptr(out), _ptr(q_bits), _code(q_dtype), _ptr(k_pool), _ptr(v_pool), _code(kv_dtype),
+        float(k_scale), float(v_scale), _ptr(block_tables), block_tables.shape[1],
+        _ptr(context_lens), _ptr(query_start), S, H, Hkv, D, B, NB, float(scale), int(threads)))
     return out
 
 

@@ -20,6 +20,12 @@
  *   [PT]  "vLLM and PagedAttention: virtual memory for LLM inference"
  *         (podcast transcript): copy of the partially filled shared block on
  *         write, full shared blocks stay shared.
+ *   [PT]  (same transcript, opening paragraph): inference splits into the
+ *         prefill of the prompt, whose tokens are all known at once and map
+ *         onto large matrix products, and the token-by-token decode.
+ *   [HJ]  "Paged Attention" study notes (huajishe.fun), section on
+ *         points to watch: the first forward pass of a new request (prefill)
+ *         needs its own handling.
  *   [OCP] OCP 8-bit Floating Point Specification (OFP8), E4M3 encoding:
  *         bias 7, no infinities, S.1111.111 is NaN, max finite 448,
  *         subnormals m * 2^-9.  The pages only say "8-bit"; the choice of
@@ -234,6 +240,106 @@ int orc_paged_attn_decode(double* out, const void* q, int q_dtype,
                 size_t row = (((size_t)pid * num_kv_heads + kvh) * block_size + t % block_size) * head_dim;
                 for (int d = 0; d < head_dim; ++d)
                     o[d] += p * load_elem(v_pool, row + d, kv_dtype, vs);
+            }
+            for (int d = 0; d < head_dim; ++d)
+                o[d] /= l;
+        }
+        free(x);
+        free(qv);
+    }
+    return ORC_OK;
+}
+
+/* ---------------------------------------------------------------------- */
+/* Chunked prefill ([WP] token form for every query position of a chunk;   */
+/* [PT] prefill; [HJ] prefill handling).                                    */
+/* ---------------------------------------------------------------------- */
+
+/*
+ * Sequence s holds L_s = context_lens[s] tokens in the cache; its last
+ * C_s = query_start[s+1] - query_start[s] tokens are the chunk being
+ * prefilled (their K/V already scattered into the pool, as for decode).
+ * Query row r = query_start[s] + j (j < C_s) is token position
+ * p = L_s - C_s + j and attends causally to positions 0..p:
+ *   out[r][h][:] = sum_{t<=p} softmax_t(scale * q[r][h] . k_t) v_t,
+ * with k_t, v_t read through the block table as in decode.  Decode is the
+ * case C_s = 1.  q is [num_tokens][H][D] with num_tokens = query_start[S].
+ */
+int orc_paged_attn_prefill(double* out, const void* q, int q_dtype,
+                           const void* k_pool, const void* v_pool, int kv_dtype,
+                           double k_scale, double v_scale,
+                           const int32_t* block_tables, int max_blocks_per_seq,
+                           const int32_t* context_lens, const int32_t* query_start,
+                           int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                           int block_size, int num_blocks, double scale, int num_threads)
+{
+    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        block_size <= 0 || num_blocks <= 0 || num_heads % num_kv_heads != 0 ||
+        (q_dtype != ORC_F16 && q_dtype != ORC_BF16) ||
+        (kv_dtype != ORC_F16 && kv_dtype != ORC_BF16 && kv_dtype != ORC_E4M3) ||
+        query_start[0] != 0)
+        return ORC_BAD_ARG;
+    const int G = num_heads / num_kv_heads;
+    const double ks = kv_dtype == ORC_E4M3 ? k_scale : 1.0;
+    const double vs = kv_dtype == ORC_E4M3 ? v_scale : 1.0;
+    for (int s = 0; s < num_seqs; ++s) {
+        const int L = context_lens[s], C = query_start[s + 1] - query_start[s];
+        if (C < 0 || C > L)
+            return ORC_BAD_ARG;
+        if (L > (long)max_blocks_per_seq * block_size)
+            return ORC_BAD_LEN;
+        for (int j = 0; j < (L + block_size - 1) / block_size; ++j) {
+            int pid = block_tables[(size_t)s * max_blocks_per_seq + j];
+            if (pid < 0 || pid >= num_blocks)
+                return ORC_BAD_BLOCK;
+        }
+    }
+    const long rows = query_start[num_seqs];
+#ifdef _OPENMP
+    if (num_threads > 0)
+        omp_set_num_threads(num_threads);
+#else
+    (void)num_threads;
+#endif
+#pragma omp parallel
+    {
+        int maxL = 1;
+        for (int s = 0; s < num_seqs; ++s)
+            if (context_lens[s] > maxL) maxL = context_lens[s];
+        double* x = (double*)malloc(sizeof(double) * (size_t)maxL);
+        double* qv = (double*)malloc(sizeof(double) * (size_t)head_dim);
+#pragma omp for schedule(dynamic, 1)
+        for (long u = 0; u < rows * num_heads; ++u) {
+            const long r = u / num_heads;
+            const int h = (int)(u % num_heads), kvh = h / G;
+            int s = 0;
+            while (query_start[s + 1] <= r) ++s;          /* the sequence row r belongs to */
+            const int L = context_lens[s];
+            const int C = query_start[s + 1] - query_start[s];
+            const int p = L - C + (int)(r - query_start[s]);   /* its token position */
+            double* o = out + (size_t)u * head_dim;
+            for (int d = 0; d < head_dim; ++d) {
+                o[d] = 0.0;
+                qv[d] = load_elem(q, (size_t)u * head_dim + d, q_dtype, 1.0);
+            }
+            double m = -INFINITY;
+            for (int t = 0; t <= p; ++t) {
+                int pid = block_tables[(size_t)s * max_blocks_per_seq + t / block_size];
+                size_t krow = (((size_t)pid * num_kv_heads + kvh) * block_size + t % block_size) * head_dim;
+                double dot = 0.0;
+                for (int d = 0; d < head_dim; ++d)
+                    dot += qv[d] * load_elem(k_pool, krow + d, kv_dtype, ks);
+                x[t] = scale * dot;
+                if (x[t] > m) m = x[t];
+            }
+            double l = 0.0;
+            for (int t = 0; t <= p; ++t) {
+                double w = exp(x[t] - m);
+                l += w;
+                int pid = block_tables[(size_t)s * max_blocks_per_seq + t / block_size];
+                size_t vrow = (((size_t)pid * num_kv_heads + kvh) * block_size + t % block_size) * head_dim;
+                for (int d = 0; d < head_dim; ++d)
+                    o[d] += w * load_elem(v_pool, vrow + d, kv_dtype, vs);
             }
             for (int d = 0; d < head_dim; ++d)
                 o[d] /= l;
