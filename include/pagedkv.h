@@ -18,6 +18,10 @@
  *                          (Wikipedia "PagedAttention", section "Mathematical
  *                          formulation": o_i = sum_j V_j A_ij^T over the
  *                          ceil(i/B) blocks of the sequence).
+ * and the prefill of a chunk of new tokens over the same cache
+ * (pkv_paged_attn_prefill: every query of the chunk attends causally, the
+ * dense phase of the "vLLM and PagedAttention" transcript's opening
+ * paragraph), on the 5th-generation tensor cores.
  *
  * Conventions shared by every entry point
  *   - All pointers except scalars are DEVICE pointers, owned by the caller.
@@ -221,6 +225,46 @@ pkv_status pkv_paged_attn_decode_static_ws(void* out, const void* q, pkv_dtype q
                                            int num_seqs, int num_heads, int num_kv_heads, int head_dim,
                                            int block_size, int num_blocks, float scale, int partition_size,
                                            uint32_t* device_error, void* stream);
+
+/*
+ * Chunked prefill over the paged cache (Wikipedia "PagedAttention", section
+ * "Mathematical formulation", token form, for every query position of a
+ * chunk; "vLLM and PagedAttention" transcript, opening paragraph: the prompt
+ * is processed at once as large matrix products; "Paged Attention" study
+ * notes (huajishe.fun), section on points to watch: prefill needs its own
+ * handling).
+ *
+ * Sequence s holds L = context_lens[s] tokens in the pool, the last
+ * C = query_start[s+1] - query_start[s] of which are the chunk (their K/V
+ * already written, e.g. by pkv_reshape_and_cache).  Query row
+ * r = query_start[s] + j (0 <= j < C) sits at position p = L - C + j:
+ *   out[r][h][:] = sum_{t <= p} softmax_t(scale * q[r][h] . k_t) * v_t,
+ * with k_t, v_t read through the block table as in decode and
+ * h / G the KV head of query head h.  Decode is the case C = 1.
+ *
+ *   out            [num_tokens][num_heads][head_dim], dtype
+ *   q              [num_tokens][num_heads][head_dim], dtype in {F16, BF16};
+ *                  the chunks of all sequences packed in order
+ *   k_pool/v_pool  see conventions, the same dtype as q
+ *   block_tables   int32 [num_seqs][max_blocks_per_seq]
+ *   context_lens   int32 [num_seqs]
+ *   query_start    int32 [num_seqs + 1], query_start[0] = 0,
+ *                  query_start[num_seqs] = num_tokens, non-decreasing
+ *   max_query_len  an upper bound of the chunk lengths (sizes the grid)
+ *   head_dim in {64, 128}; block_size in {16, 32}; G = num_heads /
+ *   num_kv_heads in {1, 2, 4, 8, 16}; scale > 0.
+ * Data-dependent problems (a chunk longer than its context, a context beyond
+ * the table, a bad block id) write NaN rows for the affected query tile and
+ * set PKV_DEVERR_CONTEXT_LEN / PKV_DEVERR_BLOCK_ID.  Scores and the output
+ * accumulate in float32; the softmax weights enter the P.V product rounded
+ * to dtype (the tensor-core operand type).  No workspace.
+ */
+pkv_status pkv_paged_attn_prefill(void* out, const void* q, pkv_dtype dtype, const void* k_pool,
+                                  const void* v_pool, const int32_t* block_tables, int max_blocks_per_seq,
+                                  const int32_t* context_lens, const int32_t* query_start, int max_query_len,
+                                  int num_seqs, int num_tokens, int num_heads, int num_kv_heads, int head_dim,
+                                  int block_size, int num_blocks, float scale, uint32_t* device_error,
+                                  void* stream);
 
 /*
  * Scatter new tokens into the pool (glossary "PagedAttention", section "How

@@ -51,6 +51,8 @@ def lib() -> ctypes.CDLL:
         L.pkv_paged_attn_decode.argtypes = [P, P, I, P, P, I, F, F, P, I, P, I, I, I, I, I, I, I, F, I,
                                             P, Z, P, P]
         L.pkv_paged_attn_decode.restype = I
+        L.pkv_paged_attn_prefill.argtypes = [P, P, I, P, P, P, I, P, P, I, I, I, I, I, I, I, I, F, P, P]
+        L.pkv_paged_attn_prefill.restype = I
         L.pkv_reshape_and_cache.argtypes = [P, P, I, P, P, I, F, F, P, I, I, I, I, I, P, P]
         L.pkv_reshape_and_cache.restype = I
         L.pkv_copy_blocks.argtypes = [P, P, Z, P, I, I, P, P]
@@ -146,6 +148,36 @@ def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_pool: torch.Tensor, 
         NB, float(scale), int(partition_size), _dev(workspace, "workspace"), ws_bytes,
         _dev(device_error, "device_error"), _stream(stream))
     _check(status, "paged_attn_decode")
+    return out
+
+
+def paged_attn_prefill(out: torch.Tensor, q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
+                       block_tables: torch.Tensor, context_lens: torch.Tensor, query_start: torch.Tensor,
+                       scale: float, *, max_query_len: int, device_error: Optional[torch.Tensor] = None,
+                       stream=None) -> torch.Tensor:
+    """out[T, H, D] = chunked causal prefill of q[T, H, D] over pools [NB, Hkv, B, D].
+
+    The chunks of all sequences are packed in q; query_start int32 [S + 1] gives
+    their row offsets, context_lens int32 [S] count each chunk's tokens (already
+    in the pool).  q, out and the pools share one 16-bit dtype.
+    """
+    T, H, D = q.shape
+    NB, Hkv, B, D2 = k_pool.shape
+    S = context_lens.numel()
+    if out.shape != q.shape or out.dtype != q.dtype or D2 != D or v_pool.shape != k_pool.shape:
+        raise ValueError("inconsistent shapes or dtypes")
+    if k_pool.dtype != q.dtype or v_pool.dtype != q.dtype:
+        raise TypeError("prefill needs q and the pools in one 16-bit dtype")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32 or query_start.dtype != torch.int32:
+        raise TypeError("block_tables, context_lens and query_start must be int32")
+    if query_start.numel() != S + 1:
+        raise ValueError("query_start must hold num_seqs + 1 offsets")
+    status = lib().pkv_paged_attn_prefill(
+        _dev(out, "out"), _dev(q, "q"), _code(q), _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"),
+        _dev(block_tables, "block_tables"), block_tables.shape[1], _dev(context_lens, "context_lens"),
+        _dev(query_start, "query_start"), int(max_query_len), S, T, H, Hkv, D, B, NB, float(scale),
+        _dev(device_error, "device_error"), _stream(stream))
+    _check(status, "paged_attn_prefill")
     return out
 
 

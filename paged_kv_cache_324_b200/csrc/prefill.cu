@@ -1,0 +1,656 @@
+// Chunked prefill over the paged KV cache on the 5th-generation tensor cores.
+//
+// Every query of a chunk attends causally to the cached tokens up to its own
+// position (Wikipedia "PagedAttention", section "Mathematical formulation",
+// token form, for each query position of the chunk); unlike decode this is a
+// dense contraction ("vLLM and PagedAttention" transcript, opening paragraph:
+// prefill maps onto large matrix products), so both products run as
+// tcgen05.mma with the accumulators in tensor memory.
+//
+// One CTA = 128 query rows (128 / G tokens x the G query heads of one KV
+// head) of one sequence, against 128-key tiles of that KV head read through
+// the block table.  Warp roles:
+//   warp 0     TMA: the Q tile once, then K and V tiles block by block (one
+//              4-D box per 16- or 32-token block and 64-column chunk) into
+//              128-byte-swizzled rings (3 K stages, 2 V stages);
+//   warp 1     allocates 512 TMEM columns; one thread issues the MMAs:
+//              S_j = Q K_j^T into one of two TMEM buffers (M=128, N=128),
+//              and O += P_j V_j (M=128, N=head_dim) once P_j is written;
+//   warps 2-5  softmax, one query row per thread (TMEM lane = row): read S_j
+//              with tcgen05.ld, mask, online softmax in base 2 with a running
+//              maximum that is only moved when the new one exceeds it by more
+//              than 2^8 (the result does not depend on the reference maximum;
+//              this only bounds the weights), write P_j as 16-bit values into
+//              a swizzled shared-memory tile (the A operand of the next MMA),
+//              and rescale O in TMEM when the maximum moves; finally O / l.
+// S_{j+1} is issued before P_j is consumed, so the tensor core works on the
+// next tile while the softmax warps work on this one.
+//
+// Keys beyond the last one any row of the CTA needs are never loaded; their V
+// rows are zeroed in shared memory (their weights are exactly 0, but 0 times
+// stale bytes could be NaN).  Every wait is bounded; a wait that gives up
+// sets PKV_DEVERR_TIMEOUT, the other roles stop at their next wait, in-flight
+// copies and MMAs are drained (bounded) and TMEM is freed before exit.
+
+#include <cmath>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "pkv_device.cuh"
+#include "pkv_host.h"
+
+namespace pkv {
+namespace {
+
+constexpr int kRows = 128;            // query rows per CTA: MMA M, one TMEM lane each
+constexpr int kKeys = 128;            // keys per tile: N of S = Q K^T, K of O += P V
+constexpr int kKStages = 3;
+constexpr int kVStages = 2;
+constexpr int kPThreads = 192;        // warp 0 TMA, warp 1 MMA, warps 2-5 softmax
+constexpr uint32_t kTmemCols = 512;   // S buffers at columns 0 and 128, O at 256
+constexpr uint32_t kTmemO = 256;
+constexpr float kMaxLag = 8.0f;       // log2 of the largest weight the lagging maximum allows
+constexpr uint32_t kChunkBytes = kRows * 128;   // 128 rows x 128 bytes: one 64-column chunk
+
+template <int D>
+struct PGeo {
+    static constexpr int kChunks = D / 64;
+    static constexpr uint32_t kTile = kChunks * kChunkBytes;   // Q, or one K or V stage
+    static constexpr uint32_t kQ = 0;
+    static constexpr uint32_t kK = kQ + kTile;
+    static constexpr uint32_t kV = kK + kKStages * kTile;
+    static constexpr uint32_t kP = kV + kVStages * kTile;
+    static constexpr uint32_t kEnd = kP + 2 * kChunkBytes;      // P: 128 rows x 128 keys x 2 bytes
+    // +1 KB to align the base; at least 120 KB so that one CTA holds an SM (TMEM is not shared)
+    static constexpr uint32_t kSmemBytes = (kEnd + 1024 > 120u * 1024u) ? kEnd + 1024 : 120u * 1024u;
+};
+
+struct PrefillArgs {
+    void* out;
+    const int32_t* block_tables;
+    const int32_t* context_lens;
+    const int32_t* query_start;
+    uint32_t* err;
+    int max_blocks_per_seq;
+    int num_tokens;
+    int num_heads;
+    int num_blocks;
+    int group;            // G = num_heads / num_kv_heads
+    float scale_log2;     // scale * log2(e)
+};
+
+// ---- tcgen05 / TMEM primitives (inline PTX) ---------------------------------------
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
+// lbo/sbo in bytes: K-major tiles use sbo = 1024 (8-row groups of 128-byte rows);
+// MN-major tiles add lbo = the distance between 64-element column chunks.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    return static_cast<uint64_t>((addr & 0x3FFFFu) >> 4) |
+           (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+           (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) |
+           (1ull << 46) |          // descriptor version for sm_100
+           (2ull << 61);           // SWIZZLE_128B
+}
+
+// Instruction descriptor of kind::f16: f32 accumulator, A and B of one 16-bit type,
+// A K-major, B K-major or MN-major, shape M x N.
+__host__ __device__ constexpr uint32_t mma_idesc(bool bf16, bool b_mn_major, int M, int N) {
+    return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+           (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, bool accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate ? 1u : 0u)
+        : "memory");
+}
+
+// Arrive once on `bar` when every MMA this thread issued so far has completed.
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+
+// tcgen05.ld delivers its registers asynchronously: the wait takes them as operands so
+// that no use of them can be scheduled before it.
+__device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, uint32_t (&r)[32]) {
+    tmem_ld32(taddr, r);
+    asm volatile(
+        "tcgen05.wait::ld.sync.aligned;"
+        : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+          "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+          "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+          "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+        :
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]),
+        "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]),
+        "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,
+                                            int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
+
+template <bool kBf16>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    if constexpr (kBf16) {
+        __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+        return *reinterpret_cast<uint32_t*>(&v);
+    } else {
+        __half2 v = __floats2half2_rn(lo, hi);
+        return *reinterpret_cast<uint32_t*>(&v);
+    }
+}
+
+// Shared flags of a CTA: a wait gave up (every role stops), a block id was bad.
+struct CtaFlags {
+    int abort;
+    int bad;
+    uint32_t tmem_base;
+};
+
+// Bounded wait that also stops when another role of the CTA already gave up.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, CtaFlags* f, uint32_t* err) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t end = global_timer_ns() + kWaitLimitNs;
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 32; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (*reinterpret_cast<volatile int*>(&f->abort)) return false;
+        if (global_timer_ns() > end) {
+            raise_error(err, PKV_DEVERR_TIMEOUT);
+            *reinterpret_cast<volatile int*>(&f->abort) = 1;
+            return false;
+        }
+    }
+}
+
+// Same, decided once for a whole warp (every lane waits; all continue only if all succeeded).
+__device__ __forceinline__ bool warp_wait_bar(uint32_t bar, uint32_t parity, CtaFlags* f, uint32_t* err) {
+    const bool ok = wait_bar(bar, parity, f, err);
+    return __all_sync(0xffffffffu, ok);
+}
+
+template <int D, int BS, bool kBf16>
+__global__ void __launch_bounds__(kPThreads, 1)
+paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
+                     const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap) {
+    using Gm = PGeo<D>;
+    constexpr int kTB = kKeys / BS;                  // blocks per key tile
+    constexpr uint32_t kBoxBytes = BS * 128;         // one block x one 64-column chunk
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t bars[2 * kKStages + 2 * kVStages + 8];
+    __shared__ CtaFlags flags;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = a.group, TQ = kRows / G;
+    const int kvh = blockIdx.y, s = blockIdx.z;
+
+    pdl_wait();   // q, the pool and the tables may come from the previous kernel on the stream
+    const int q0 = __ldg(a.query_start + s), q1 = __ldg(a.query_start + s + 1);
+    const int L = __ldg(a.context_lens + s);
+    if (q0 < 0 || q1 < q0 || q1 > a.num_tokens) {        // rows of unknown place: nothing to write
+        if (threadIdx.x == 0 && blockIdx.x == 0) raise_error(a.err, PKV_DEVERR_CONTEXT_LEN);
+        return;
+    }
+    const int C = q1 - q0;
+    const int ntq = (C + TQ - 1) / TQ;
+    if (blockIdx.x == 0 && threadIdx.x == 0 && ntq > static_cast<int>(gridDim.x))
+        raise_error(a.err, PKV_DEVERR_CONTEXT_LEN);      // longer than max_query_len: rows left unwritten
+    if (static_cast<int>(blockIdx.x) >= ntq) return;
+    if (grid_timed_out(a.err)) return;   // a wait elsewhere gave up: finish at once
+    const int t0 = (ntq - 1 - static_cast<int>(blockIdx.x)) * TQ;   // longest tiles first
+    const int rows_valid = min(TQ, C - t0);
+    const int pq_max = min(L - C + t0 + TQ - 1, L - 1);   // last key any row of this CTA attends
+
+    if (C > L || L > a.max_blocks_per_seq * BS) {         // positions undefined: NaN rows
+        if (threadIdx.x == 0) raise_error(a.err, PKV_DEVERR_CONTEXT_LEN);
+        for (int i = threadIdx.x; i < rows_valid * G * D; i += kPThreads) {
+            const int t = i / (G * D), rem = i % (G * D);
+            const size_t o = (static_cast<size_t>(q0 + t0 + t) * a.num_heads + kvh * G) * D + rem;
+            reinterpret_cast<uint16_t*>(a.out)[o] = kBf16 ? 0x7FC0u : 0x7E00u;
+        }
+        return;
+    }
+    const int ntk = pq_max / kKeys + 1;                    // key tiles this CTA needs
+    const int nblk = (pq_max + 1 + BS - 1) / BS;           // blocks holding keys 0..pq_max
+
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_addr(smem);
+    const uint32_t sQ = sbase + Gm::kQ, sK = sbase + Gm::kK, sV = sbase + Gm::kV, sP = sbase + Gm::kP;
+    const uint32_t b0 = smem_addr(bars);
+    auto k_full = [&](int i) { return b0 + 8u * i; };
+    auto k_empty = [&](int i) { return b0 + 8u * (kKStages + i); };
+    auto v_full = [&](int i) { return b0 + 8u * (2 * kKStages + i); };
+    auto v_empty = [&](int i) { return b0 + 8u * (2 * kKStages + kVStages + i); };
+    const uint32_t bar_q = b0 + 8u * (2 * kKStages + 2 * kVStages);
+    auto s_full = [&](int i) { return bar_q + 8u * (1 + i); };
+    auto s_empty = [&](int i) { return bar_q + 8u * (3 + i); };
+    const uint32_t p_full = bar_q + 8u * 5, o_done = bar_q + 8u * 6, drain = bar_q + 8u * 7;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kKStages; ++i) {
+            mbar_init(k_full(i), 1);
+            mbar_init(k_empty(i), 1);
+        }
+        for (int i = 0; i < kVStages; ++i) {
+            mbar_init(v_full(i), 1);
+            mbar_init(v_empty(i), 1);
+        }
+        mbar_init(bar_q, 1);
+        mbar_init(s_full(0), 1);
+        mbar_init(s_full(1), 1);
+        mbar_init(s_empty(0), 4);
+        mbar_init(s_empty(1), 4);
+        mbar_init(p_full, 4);
+        mbar_init(o_done, 1);
+        mbar_init(drain, 1);
+        flags.abort = 0;
+        flags.bad = 0;
+        mbar_fence_init();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_addr(&flags.tmem_base)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = flags.tmem_base;
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        const uint64_t pol = l2_policy_evict_last();      // K/V tiles are read again by the other query tiles
+        if (lane == 0) {
+            tma_prefetch_desc(&qmap);
+            tma_prefetch_desc(&kmap);
+            tma_prefetch_desc(&vmap);
+            mbar_arrive_expect_tx(bar_q, Gm::kTile);
+#pragma unroll
+            for (int c = 0; c < Gm::kChunks; ++c) tma_load_3d(sQ + c * kChunkBytes, &qmap, bar_q, c * 64, kvh * G, q0 + t0);
+        }
+        const int32_t* trow = a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq;
+        int k_issued = 0, v_issued = 0;   // tiles whose K (V) copies were issued
+        for (int j = 0; j < ntk; ++j) {
+            const int blk = j * kTB + lane;
+            const bool want = lane < kTB && blk < nblk;
+            const int pid = want ? __ldg(trow + blk) : -1;
+            const bool bad = want && (pid < 0 || pid >= a.num_blocks);
+            const unsigned ok_mask = __ballot_sync(0xffffffffu, want && !bad);
+            if (__any_sync(0xffffffffu, bad) && lane == 0) {
+                raise_error(a.err, PKV_DEVERR_BLOCK_ID);
+                flags.bad = 1;
+            }
+            const uint32_t bytes = __popc(ok_mask) * kBoxBytes * Gm::kChunks;
+            const int ks = j % kKStages, vs = j % kVStages;
+            if (j >= kKStages && !warp_wait_bar(k_empty(ks), ((j / kKStages) - 1) & 1, &flags, a.err)) break;
+            if (lane == 0) mbar_arrive_expect_tx(k_full(ks), bytes);
+            k_issued = j + 1;
+            for (int b = 0; b < kTB; ++b) {
+                const int p = __shfl_sync(0xffffffffu, pid, b);
+                if (lane == 0 && ((ok_mask >> b) & 1u)) {
+#pragma unroll
+                    for (int c = 0; c < Gm::kChunks; ++c)
+                        tma_load_4d(sK + ks * Gm::kTile + c * kChunkBytes + b * kBoxBytes, &kmap, k_full(ks), c * 64,
+                                    0, kvh, p, pol);
+                }
+            }
+            if (j >= kVStages && !warp_wait_bar(v_empty(vs), ((j / kVStages) - 1) & 1, &flags, a.err)) break;
+            if (lane == 0) mbar_arrive_expect_tx(v_full(vs), bytes);
+            v_issued = j + 1;
+            for (int b = 0; b < kTB; ++b) {
+                const int p = __shfl_sync(0xffffffffu, pid, b);
+                if (lane == 0 && ((ok_mask >> b) & 1u)) {
+#pragma unroll
+                    for (int c = 0; c < Gm::kChunks; ++c)
+                        tma_load_4d(sV + vs * Gm::kTile + c * kChunkBytes + b * kBoxBytes, &vmap, v_full(vs), c * 64,
+                                    0, kvh, p, pol);
+                }
+            }
+        }
+        // drain: the last copies of each stage must land before the CTA may exit
+        if (lane == 0) {
+            const uint64_t end = global_timer_ns() + kWaitLimitNs;
+            mbar_wait(bar_q, 0, end);
+            for (int j = max(0, k_issued - kKStages); j < k_issued; ++j)
+                mbar_wait(k_full(j % kKStages), (j / kKStages) & 1, end);
+            for (int j = max(0, v_issued - kVStages); j < v_issued; ++j)
+                mbar_wait(v_full(j % kVStages), (j / kVStages) & 1, end);
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer (one thread) ----------------
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = mma_idesc(kBf16, false, kRows, kKeys);
+            constexpr uint32_t idesc_o = mma_idesc(kBf16, true, kRows, D);
+            bool ok = wait_bar(bar_q, 0, &flags, a.err);
+            auto issue_s = [&](int j) -> bool {
+                const int ks = j % kKStages;
+                if (!wait_bar(k_full(ks), (j / kKStages) & 1, &flags, a.err)) return false;
+                if (j >= 2 && !wait_bar(s_empty(j & 1), ((j >> 1) - 1) & 1, &flags, a.err)) return false;
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < D / 16; ++k) {
+                    const uint32_t off = (k >> 2) * kChunkBytes + (k & 3) * 32;
+                    mma_f16(tmem + (j & 1) * kKeys, smem_desc(sQ + off, 16, 1024),
+                            smem_desc(sK + ks * Gm::kTile + off, 16, 1024), idesc_s, k > 0);
+                }
+                mma_commit(s_full(j & 1));
+                mma_commit(k_empty(ks));
+                return true;
+            };
+            if (ok) ok = issue_s(0);
+            for (int j = 0; ok && j < ntk; ++j) {
+                if (j + 1 < ntk && !issue_s(j + 1)) break;
+                const int vs = j % kVStages;
+                if (!wait_bar(v_full(vs), (j / kVStages) & 1, &flags, a.err)) break;
+                if (!wait_bar(p_full, j & 1, &flags, a.err)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kKeys / 16; ++kk) {
+                    mma_f16(tmem + kTmemO, smem_desc(sP + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024),
+                            smem_desc(sV + vs * Gm::kTile + kk * 16 * 128, kChunkBytes, 1024), idesc_o,
+                            j > 0 || kk > 0);
+                }
+                mma_commit(o_done);
+                mma_commit(v_empty(vs));
+            }
+            // drain: every MMA issued so far completes before TMEM is freed
+            mma_commit(drain);
+            mbar_wait(drain, 0, global_timer_ns() + kWaitLimitNs);
+        }
+        __syncwarp();
+    } else {
+        // ---------------- softmax (warps 2-5, one row per thread) ----------------
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+        const int tq = row / G;
+        const int pq = min(L - C + t0 + tq, L - 1);
+        float m_used = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < ntk; ++j) {
+            const int buf = j & 1;
+            if (!warp_wait_bar(s_full(buf), (j >> 1) & 1, &flags, a.err)) { ok = false; break; }
+            tc_fence_after();
+            float x[kKeys];
+#pragma unroll
+            for (int c = 0; c < kKeys / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32_wait(trow + buf * kKeys + c * 32, r);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(r[i]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(s_empty(buf));
+            const int kbase = j * kKeys;
+            if (kbase + kKeys - 1 > pq) {
+#pragma unroll
+                for (int c = 0; c < kKeys; ++c) x[c] = (kbase + c > pq) ? -INFINITY : x[c];
+            }
+            float mx = x[0];
+#pragma unroll
+            for (int c = 1; c < kKeys; ++c) mx = fmaxf(mx, x[c]);
+            const float m_cand = mx * a.scale_log2;
+            const bool move = m_cand > m_used + kMaxLag;
+            float alpha = 1.f;
+            if (move) {
+                alpha = exp2f(m_used - m_cand);
+                m_used = m_cand;
+            }
+            const float neg_m = -m_used;
+            uint32_t pk[kKeys / 2];
+            float sum = 0.f;
+#pragma unroll
+            for (int c = 0; c < kKeys; c += 2) {
+                const float p0 = exp2f(fmaf(x[c], a.scale_log2, neg_m));
+                const float p1 = exp2f(fmaf(x[c + 1], a.scale_log2, neg_m));
+                sum += p0 + p1;
+                pk[c / 2] = pack2<kBf16>(p0, p1);
+            }
+            l = l * alpha + sum;
+            // P and O are free once the previous P.V product has completed
+            if (j > 0 && !warp_wait_bar(o_done, (j - 1) & 1, &flags, a.err)) { ok = false; break; }
+            if (j > 0 && __any_sync(0xffffffffu, move)) {
+                tc_fence_after();
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32_wait(trow + kTmemO + c * 32, r);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                    tmem_st32(trow + kTmemO + c * 32, r);
+                }
+                tmem_wait_st();
+            }
+            // P row: keys as K, 64 keys per 128-byte chunk row, 16-byte units swizzled by row % 8
+#pragma unroll
+            for (int u = 0; u < kKeys / 8; ++u) {
+                const uint32_t addr = sP + (u >> 3) * kChunkBytes + row * 128 + (((u & 7) ^ (row & 7)) << 4);
+                sts128(addr, pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+            }
+            if (j == ntk - 1 && kbase + kKeys - 1 > pq_max) {
+                // keys past pq_max were not loaded (or are unwritten slots): zero their V rows
+                const int vs = j % kVStages;
+                if (!warp_wait_bar(v_full(vs), (j / kVStages) & 1, &flags, a.err)) { ok = false; break; }
+                if (kbase + row > pq_max) {
+#pragma unroll
+                    for (int c = 0; c < Gm::kChunks; ++c)
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            sts128(sV + vs * Gm::kTile + c * kChunkBytes + row * 128 + (((u ^ (row & 7)) & 7) << 4), 0u,
+                                   0u, 0u, 0u);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_full);
+        }
+        if (ok) ok = warp_wait_bar(o_done, (ntk - 1) & 1, &flags, a.err);
+        pdl_trigger();
+        // the output is written after the CTA-wide barrier below, which also publishes flags.bad
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        // every lane takes part in the warp-wide TMEM loads; only rows of the chunk are stored
+        const bool live = tq < rows_valid;
+        const bool nan_out = !ok || flags.bad || *reinterpret_cast<volatile int*>(&flags.abort);
+        uint16_t* orow = reinterpret_cast<uint16_t*>(a.out) +
+                         (static_cast<size_t>(q0 + t0 + (live ? tq : 0)) * a.num_heads + kvh * G + row % G) * D;
+        const float inv = 1.f / l;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32_wait(trow + kTmemO + c * 32, r);
+            if (live) {
+                uint32_t w[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    w[i] = nan_out ? (kBf16 ? 0x7FC07FC0u : 0x7E007E00u)
+                                   : pack2<kBf16>(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
+                uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        return;   // warp 1 frees TMEM after the second barrier
+    }
+    // producer and MMA warps: meet the softmax warps at both barriers
+    pdl_trigger();
+    tc_fence_before();
+    __syncthreads();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                                : "memory");
+}
+
+// 3-D map over q [num_tokens][num_heads][head_dim]: box = 64 columns x G heads x 128/G tokens,
+// which lands as 128 rows (token-major, head-minor) of 128 bytes per 64-column chunk.
+bool encode_q_map(CUtensorMap* map, const void* q, int head_dim, int num_heads, int num_tokens, int G) {
+    EncodeTiledFn enc = encode_tiled_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(num_heads),
+                                static_cast<cuuint64_t>(num_tokens)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2,
+                                   static_cast<cuuint64_t>(num_heads) * head_dim * 2};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(G), static_cast<cuuint32_t>(kRows / G)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(q), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 4-D map over a 16-bit pool [num_blocks][num_kv_heads][block_size][head_dim]: box = 64 columns x
+// one block of one KV head; the block id is the outermost coordinate.
+bool encode_pool_map16(CUtensorMap* map, const void* pool, int head_dim, int block_size, int num_kv_heads,
+                       int num_blocks) {
+    EncodeTiledFn enc = encode_tiled_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(block_size),
+                                static_cast<cuuint64_t>(num_kv_heads), static_cast<cuuint64_t>(num_blocks)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(head_dim) * 2,
+                                   static_cast<cuuint64_t>(block_size) * head_dim * 2,
+                                   static_cast<cuuint64_t>(num_kv_heads) * block_size * head_dim * 2};
+    const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(block_size), 1, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, const_cast<void*>(pool), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int BS, bool kBf16>
+pkv_status launch_prefill(const PrefillArgs& a, const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm,
+                          dim3 grid, cudaStream_t st) {
+    auto kern = paged_prefill_kernel<D, BS, kBf16>;
+    const uint32_t smem = PGeo<D>::kSmemBytes;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    return launch_pdl(kern, grid, dim3(kPThreads), smem, st, a, qm, km, vm) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+template <int D, int BS>
+pkv_status dispatch_dtype(bool bf16, const PrefillArgs& a, const CUtensorMap& qm, const CUtensorMap& km,
+                          const CUtensorMap& vm, dim3 grid, cudaStream_t st) {
+    return bf16 ? launch_prefill<D, BS, true>(a, qm, km, vm, grid, st)
+                : launch_prefill<D, BS, false>(a, qm, km, vm, grid, st);
+}
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" pkv_status pkv_paged_attn_prefill(void* out, const void* q, pkv_dtype dtype, const void* k_pool,
+                                             const void* v_pool, const int32_t* block_tables, int max_blocks_per_seq,
+                                             const int32_t* context_lens, const int32_t* query_start,
+                                             int max_query_len, int num_seqs, int num_tokens, int num_heads,
+                                             int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                             float scale, uint32_t* device_error, void* stream) {
+    using namespace pkv;
+    if (num_seqs < 0 || num_tokens < 0 || max_query_len < 0 || num_heads <= 0 || num_kv_heads <= 0 ||
+        num_blocks <= 0 || max_blocks_per_seq <= 0 || !(scale > 0.f) || !std::isfinite(scale))
+        return PKV_ERR_INVALID_ARG;
+    if (num_heads % num_kv_heads != 0) return PKV_ERR_INVALID_ARG;
+    if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
+    const int G = num_heads / num_kv_heads;
+    if ((head_dim != 64 && head_dim != 128) || (block_size != 16 && block_size != 32) ||
+        (G != 1 && G != 2 && G != 4 && G != 8 && G != 16))
+        return PKV_ERR_UNSUPPORTED;
+    if (num_seqs == 0 || num_tokens == 0 || max_query_len == 0) return PKV_OK;
+    if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens || !query_start) return PKV_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) ||
+        (reinterpret_cast<uintptr_t>(block_tables) & 3) || (reinterpret_cast<uintptr_t>(context_lens) & 3) ||
+        (reinterpret_cast<uintptr_t>(query_start) & 3) || (reinterpret_cast<uintptr_t>(device_error) & 3))
+        return PKV_ERR_ALIGNMENT;
+    const long long tiles = (static_cast<long long>(max_query_len) * G + kRows - 1) / kRows;
+    if (num_seqs > 65535 || num_kv_heads > 65535 || tiles > 0x7fffffffLL) return PKV_ERR_INVALID_ARG;
+
+    PrefillArgs a{};
+    a.out = out;
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    a.query_start = query_start;
+    a.err = device_error;
+    a.max_blocks_per_seq = max_blocks_per_seq;
+    a.num_tokens = num_tokens;
+    a.num_heads = num_heads;
+    a.num_blocks = num_blocks;
+    a.group = G;
+    a.scale_log2 = scale * 1.4426950408889634f;
+
+    alignas(64) CUtensorMap qm;
+    alignas(64) CUtensorMap km;
+    alignas(64) CUtensorMap vm;
+    if (!encode_q_map(&qm, q, head_dim, num_heads, num_tokens, G) ||
+        !encode_pool_map16(&km, k_pool, head_dim, block_size, num_kv_heads, num_blocks) ||
+        !encode_pool_map16(&vm, v_pool, head_dim, block_size, num_kv_heads, num_blocks))
+        return PKV_ERR_CUDA;
+    const dim3 grid(static_cast<unsigned>(tiles), static_cast<unsigned>(num_kv_heads), static_cast<unsigned>(num_seqs));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool bf16 = dtype == PKV_BF16;
+    if (head_dim == 128)
+        return block_size == 16 ? dispatch_dtype<128, 16>(bf16, a, qm, km, vm, grid, st)
+                                : dispatch_dtype<128, 32>(bf16, a, qm, km, vm, grid, st);
+    return block_size == 16 ? dispatch_dtype<64, 16>(bf16, a, qm, km, vm, grid, st)
+                            : dispatch_dtype<64, 32>(bf16, a, qm, km, vm, grid, st);
+}

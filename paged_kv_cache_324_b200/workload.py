@@ -369,6 +369,121 @@ def make(name: str, small: bool = False) -> DecodeWorkload:
     raise KeyError(name)
 
 
+# ---------------------------------------------------------------------------
+# chunked prefill: prior context in the cache, then a chunk of new tokens
+# ---------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class PrefillWorkload:
+    """A prefill step: each sequence holds ``context_lens - chunk_lens`` earlier tokens in the
+    cache (written by the setup scatter); the step scatters the chunk's K/V, then every chunk
+    token attends causally to the cache up to its own position."""
+    name: str
+    seed: int
+    num_seqs: int
+    num_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    num_blocks: int
+    dtype: str                   # q, K/V and output: 'f16' | 'bf16'
+    scale: np.float32
+    context_lens: np.ndarray     # int32 [S], the chunk included
+    chunk_lens: np.ndarray       # int32 [S]
+    query_start: np.ndarray      # int32 [S + 1]
+    block_tables: np.ndarray     # int32 [S, max_blocks]
+    q: np.ndarray                # uint16 [T, H, D], the chunks packed in order
+    setup: list                  # Scatter of the earlier tokens
+    step_scatter: Scatter        # the chunk's K/V
+    description: str = ""
+
+    @property
+    def num_tokens(self) -> int:
+        return int(self.query_start[-1])
+
+    @property
+    def max_query_len(self) -> int:
+        return int(self.chunk_lens.max()) if self.num_seqs else 0
+
+    @property
+    def max_blocks(self) -> int:
+        return self.block_tables.shape[1]
+
+    @property
+    def pool_shape(self):
+        return (self.num_blocks, self.num_kv_heads, self.block_size, self.head_dim)
+
+    def initial_pool(self, which: str) -> np.ndarray:
+        """Random bytes, as for decode: unwritten slots hold arbitrary bit patterns."""
+        rng = np.random.default_rng([self.seed, 1 if which == "k" else 2])
+        nbytes = int(np.prod(self.pool_shape)) * 2
+        raw = np.resize(garbage_bytes(rng, min(nbytes, 32 << 20)), nbytes)
+        return raw.view(np.uint16).reshape(self.pool_shape)
+
+
+def chunked_prefill(name, seed, H, Hkv, D, B, NB, dtype, prior_lens, chunk_lens,
+                    description="") -> PrefillWorkload:
+    """Sequences with ``prior_lens`` cached tokens each receive a chunk of ``chunk_lens`` new
+    tokens.  Blocks come from a seeded shuffle of range(NB), taken only when the last block is
+    full; tokens are written in position order, so chunks start inside partially filled blocks."""
+    rng = np.random.default_rng(seed)
+    prior = np.asarray(prior_lens, dtype=np.int64)
+    chunks = np.asarray(chunk_lens, dtype=np.int64)
+    S = len(prior)
+    alloc = BlockAllocator(rng.permutation(NB))
+    tables, ctx_slots, new_slots = [], [], []
+    for P, C in zip(prior, chunks):
+        table: List[int] = []
+        for pos in range(int(P + C)):
+            slot = alloc.slot_for_append(table, pos, B, [])
+            (ctx_slots if pos < P else new_slots).append(slot)
+        tables.append(table)
+    ck, cv = _new_values(rng, len(ctx_slots), Hkv, D, dtype)
+    nk, nv = _new_values(rng, len(new_slots), Hkv, D, dtype)
+    qs = np.zeros(S + 1, np.int32)
+    qs[1:] = np.cumsum(chunks)
+    q = normal_bits(rng, (int(qs[-1]), H, D), dtype)
+    maxb = max((len(t) for t in tables), default=1)
+    return PrefillWorkload(
+        name=name, seed=seed, num_seqs=S, num_heads=H, num_kv_heads=Hkv, head_dim=D, block_size=B,
+        num_blocks=NB, dtype=dtype, scale=np.float32(1.0 / np.sqrt(D)),
+        context_lens=(prior + chunks).astype(np.int32), chunk_lens=chunks.astype(np.int32), query_start=qs,
+        block_tables=tables_array(tables, maxb), q=q,
+        setup=[Scatter(ck, cv, np.asarray(ctx_slots, dtype=np.int64))],
+        step_scatter=Scatter(nk, nv, np.asarray(new_slots, dtype=np.int64)), description=description)
+
+
+def make_prefill(name: str = "prefill", small: bool = False) -> PrefillWorkload:
+    """The chunked-prefill workload: 16 sequences, 32 q / 8 KV heads x 128, bf16, B=16, each
+    with U{0..3072} cached tokens and a chunk of U{512..2048} new ones (small: 3 sequences)."""
+    if name != "prefill":
+        raise KeyError(name)
+    rng = np.random.default_rng(6)
+    if small:
+        prior, chunks, NB = [0, 37, 300], [200, 77, 129], 256
+    else:
+        prior, chunks, NB = rng.integers(0, 3073, size=16), rng.integers(512, 2049, size=16), 4096
+    return chunked_prefill(
+        "prefill", 6, 32, 8, 128, 16, NB, "bf16", prior, chunks,
+        f"chunked prefill: {len(prior)} sequences, 32 q / 8 KV heads, head_dim 128, bf16, B=16, "
+        + ("cached 0/37/300 + chunks 200/77/129" if small else "cached U[0,3072] + chunk U[512,2048]")
+        + f", {NB}-block pool")
+
+
+def prefill_flops(w: PrefillWorkload) -> int:
+    """Multiply-adds x 2 of Q K^T and P V over the causal pairs: 4 * D * H * sum of attended keys."""
+    L = w.context_lens.astype(np.int64)
+    C = w.chunk_lens.astype(np.int64)
+    keys = int((C * (L - C) + C * (C + 1) // 2).sum())
+    return 4 * w.head_dim * w.num_heads * keys
+
+
+def prefill_bytes(w: PrefillWorkload) -> int:
+    """Bytes a prefill call must move at least: each sequence's K/V once, q and out."""
+    kv = int(w.context_lens.astype(np.int64).sum()) * kv_bytes_per_token(1, w.num_kv_heads, w.head_dim, 2)
+    return kv + 2 * w.num_tokens * w.num_heads * w.head_dim * 2
+
+
 NAMES = ("tiny", "opt13b", "gqa", "prefix", "fp8", "fp8_b32")
 EXTRA_NAMES = ("prefix_long",)
 COMPACT_NAMES = tuple(n + "_compact" for n in NAMES if n != "prefix")

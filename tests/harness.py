@@ -90,3 +90,40 @@ def oracle_step(w: wl.DecodeWorkload, block_tables=None, context_lens=None):
                                    w.context_lens if context_lens is None else context_lens,
                                    w.scale, w.k_scale, w.v_scale)
     return {"out": out, "k_pool": kp, "v_pool": vp}
+
+
+def gpu_prefill(w, dev="cuda:0", block_tables=None, context_lens=None, query_start=None, q_bits=None):
+    """Build the cache (setup scatter), scatter the chunk's K/V, run the prefill; returns
+    (out tensor, device error word, k pool, v pool)."""
+    from paged_kv_cache_324_b200 import binding as B
+    dev = torch.device(dev)
+    kp = to_dev_bits(w.initial_pool("k"), w.dtype, dev)
+    vp = to_dev_bits(w.initial_pool("v"), w.dtype, dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    for op in list(w.setup) + [w.step_scatter]:
+        if op.slots.size:
+            B.reshape_and_cache(to_dev_bits(op.k, w.dtype, dev), to_dev_bits(op.v, w.dtype, dev), kp, vp,
+                                torch.from_numpy(op.slots).to(dev), device_error=err)
+    q = to_dev_bits(w.q if q_bits is None else q_bits, w.dtype, dev)
+    out = torch.full_like(q, float("nan"))
+    bt = w.block_tables if block_tables is None else block_tables
+    cl = w.context_lens if context_lens is None else context_lens
+    qs = w.query_start if query_start is None else query_start
+    B.paged_attn_prefill(out, q, kp, vp, torch.from_numpy(np.ascontiguousarray(bt)).to(dev),
+                         torch.from_numpy(np.ascontiguousarray(cl)).to(dev),
+                         torch.from_numpy(np.ascontiguousarray(qs)).to(dev), float(w.scale),
+                         max_query_len=w.max_query_len, device_error=err)
+    torch.cuda.synchronize()
+    return out, int(err.item()), kp, vp
+
+
+def oracle_prefill_pools(w):
+    """Host pools after the setup and chunk scatters (oracle arithmetic) and the largest |v| written."""
+    import oracle
+    kp, vp = w.initial_pool("k"), w.initial_pool("v")
+    vmax = 0.0
+    for op in list(w.setup) + [w.step_scatter]:
+        if op.slots.size:
+            oracle.reshape_and_cache(op.k, op.v, w.dtype, kp, vp, w.dtype, op.slots)
+            vmax = max(vmax, float(np.abs(oracle.decode_values(op.v, w.dtype)).max()))
+    return kp, vp, vmax

@@ -79,6 +79,29 @@ def test_decode_rejects_null_and_misaligned(lib):
     assert _decode(lib, out=ctypes.c_void_p(18)) == 5
 
 
+def _prefill(lib, **over):
+    P = ctypes.c_void_p
+    args = dict(out=P(16), q=P(16), dtype=1, k_pool=P(16), v_pool=P(16), block_tables=P(16), max_blocks=4,
+                context_lens=P(16), query_start=P(16), max_q=64, S=2, T=100, H=8, Hkv=2, D=128, B=16, NB=10,
+                scale=0.1, err=None, stream=None)
+    args.update(over)
+    return lib.pkv_paged_attn_prefill(*args.values())
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(H=6, Hkv=4), 1), (dict(S=-1), 1), (dict(scale=0.0), 1), (dict(scale=-1.0), 1),
+    (dict(scale=float("inf")), 1), (dict(max_q=-1), 1), (dict(H=0), 1),
+    (dict(dtype=2), 2), (dict(D=96), 2), (dict(B=8), 2), (dict(H=6, Hkv=2), 2), (dict(H=64, Hkv=2), 2),
+    (dict(q=None), 1), (dict(query_start=None), 1), (dict(out=ctypes.c_void_p(24)), 5),
+    (dict(query_start=ctypes.c_void_p(18)), 5),
+    (dict(T=0), 0), (dict(S=0), 0), (dict(max_q=0), 0),
+])
+def test_prefill_rejects_bad_arguments(lib, over, status):
+    """Host-side checks of pkv_paged_attn_prefill (group size 3 and 32, FP8, odd sizes, a
+    non-positive scale, null and misaligned pointers; empty problems succeed at once)."""
+    assert _prefill(lib, **over) == status
+
+
 def test_reshape_and_copy_reject_bad_arguments(lib):
     P = ctypes.c_void_p
     assert lib.pkv_reshape_and_cache(P(16), P(16), 0, P(16), P(16), 1, 1.0, 1.0, P(16), 4, 2, 128, 16, 10,

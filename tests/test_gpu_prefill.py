@@ -1,0 +1,150 @@
+"""Chunked prefill on the GPU (tcgen05 kernel, through the C ABI) against the oracle.
+
+Small cases compare every output row with the float64 oracle: MHA and GQA
+groups of 2, 4, 8 and 16, head_dim 64 and 128, blocks of 16 and 32 tokens,
+f16 and bf16, whole prompts, chunks after earlier context that start inside a
+partially filled block, single-token chunks, empty chunks, chunk lengths that
+leave ragged query and key tiles, a long context, and logits wide enough that
+the running maximum moves many times.  The full-size workload is checked on
+sampled rows (each an oracle call of its own) and on properties that hold at
+any size.  Data-dependent errors (a bad block id, a chunk longer than its
+context) must give NaN rows and the documented error bits while the other
+sequences stay correct.  A prefill of one-token chunks must agree with the
+decode kernel.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from paged_kv_cache_324_b200 import binding as B
+from paged_kv_cache_324_b200 import workload as wl
+from tests import harness as H
+from tests.parity import attention_close, prefill_close
+
+pytestmark = pytest.mark.gpu
+
+
+def oracle_out(w, kp, vp, block_tables=None, context_lens=None, query_start=None, q_bits=None):
+    return oracle.paged_attn_prefill(
+        w.q if q_bits is None else q_bits, w.dtype, kp, vp, w.dtype,
+        w.block_tables if block_tables is None else block_tables,
+        w.context_lens if context_lens is None else context_lens,
+        w.query_start if query_start is None else query_start, w.scale)
+
+
+CASES = {
+    # name: (H, Hkv, D, B, dtype, prior, chunks, NB)
+    "small_workload": None,
+    "mha_f16": (4, 4, 128, 16, "f16", [0, 130, 5], [300, 1, 64], 256),
+    "g8_b32_bf16": (16, 2, 128, 32, "bf16", [1000, 0], [150, 33], 256),
+    "d64_g2_f16": (4, 2, 64, 16, "f16", [17, 500], [90, 260], 256),
+    "g16_bf16": (32, 2, 128, 16, "bf16", [64, 3], [40, 129], 64),
+    "empty_chunk": (8, 2, 128, 16, "bf16", [50, 10, 0], [0, 20, 1], 64),
+    "long_context": (8, 2, 128, 16, "f16", [5000], [130], 512),
+    "d64_b32_bf16": (8, 8, 64, 32, "bf16", [31, 300], [97, 128], 128),
+}
+
+
+def make_case(name):
+    if name == "small_workload":
+        return wl.make_prefill(small=True)
+    Hq, Hkv, D, Bs, dt, prior, chunks, NB = CASES[name]
+    return wl.chunked_prefill(name, 100 + len(name), Hq, Hkv, D, Bs, NB, dt, prior, chunks)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_prefill_matches_oracle(name):
+    w = make_case(name)
+    out, err, _, _ = H.gpu_prefill(w)
+    assert err == 0
+    kp, vp, vmax = H.oracle_prefill_pools(w)
+    ref = oracle_out(w, kp, vp)
+    ok, rep = prefill_close(H.out_f64(out), ref, w.dtype, vmax)
+    assert ok, (name, rep)
+
+
+def test_wide_logits_move_the_running_maximum():
+    """q scaled by 6: logits spread over ~+-100, so the lagging maximum moves often."""
+    w = wl.chunked_prefill("wide", 7, 8, 2, 128, 16, 256, "bf16", [700, 0], [260, 200])
+    qf = H.out_f64(H.to_dev_bits(w.q, "bf16", "cpu")) * 6.0
+    q6 = torch.from_numpy(qf).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    out, err, _, _ = H.gpu_prefill(w, q_bits=q6)
+    assert err == 0
+    kp, vp, vmax = H.oracle_prefill_pools(w)
+    ref = oracle_out(w, kp, vp, q_bits=q6)
+    ok, rep = prefill_close(H.out_f64(out), ref, "bf16", vmax)
+    assert ok, rep
+
+
+def test_bad_block_id_gives_nan_rows_and_flag():
+    w = wl.chunked_prefill("bad", 8, 8, 2, 128, 16, 128, "f16", [40, 100], [30, 60])
+    tab = w.block_tables.copy()
+    tab[1, 2] = w.num_blocks + 5                 # a block sequence 1 needs
+    out, err, _, _ = H.gpu_prefill(w, block_tables=tab)
+    assert err & 0x1
+    o = H.out_f64(out)
+    r0, r1 = int(w.query_start[1]), int(w.query_start[2])
+    assert np.isnan(o[r0:r1]).any()              # the tiles that needed the block
+    kp, vp, vmax = H.oracle_prefill_pools(w)
+    ref = oracle_out(w, kp, vp)
+    ok, rep = prefill_close(o[:r0], ref[:r0], "f16", vmax)   # sequence 0 untouched
+    assert ok, rep
+
+
+def test_chunk_longer_than_context_is_flagged():
+    w = wl.chunked_prefill("ctx", 9, 4, 4, 128, 16, 64, "bf16", [20, 5], [10, 12])
+    lens = w.context_lens.copy()
+    lens[1] = 7                                  # chunk of 12 in a context of 7
+    out, err, _, _ = H.gpu_prefill(w, context_lens=lens)
+    assert err & 0x8
+    o = H.out_f64(out)
+    r0 = int(w.query_start[1])
+    assert np.isnan(o[r0:]).all()
+    kp, vp, vmax = H.oracle_prefill_pools(w)
+    ref = oracle_out(w, kp, vp)
+    ok, rep = prefill_close(o[:r0], ref[:r0], "bf16", vmax)
+    assert ok, rep
+
+
+def test_single_token_chunks_agree_with_the_decode_kernel():
+    """Every sequence prefills one token: the same operation as decode, two different kernels."""
+    rng = np.random.default_rng(10)
+    prior = rng.integers(0, 900, size=12)
+    w = wl.chunked_prefill("c1", 10, 32, 8, 128, 16, 1024, "bf16", prior, np.ones(12, np.int64))
+    out, err, kp, vp = H.gpu_prefill(w)
+    assert err == 0
+    dev = torch.device("cuda:0")
+    q = H.to_dev_bits(w.q, "bf16", dev)
+    dec = torch.empty_like(q)
+    B.paged_attn_decode(dec, q, kp, vp, torch.from_numpy(w.block_tables).to(dev),
+                        torch.from_numpy(w.context_lens).to(dev), float(w.scale),
+                        max_context_len=int(w.context_lens.max()))
+    torch.cuda.synchronize()
+    _, _, vmax = H.oracle_prefill_pools(w)
+    ok, rep = prefill_close(H.out_f64(out), H.out_f64(dec), "bf16", vmax)
+    assert ok, rep
+
+
+def test_full_size_sampled_rows():
+    """The full chunked-prefill workload: every output finite; sampled rows against the oracle
+    (first, last and random rows of every sequence, each an oracle call of its own)."""
+    w = wl.make_prefill()
+    out, err, _, _ = H.gpu_prefill(w)
+    assert err == 0
+    o = H.out_f64(out)
+    assert np.isfinite(o).all()
+    kp, vp, vmax = H.oracle_prefill_pools(w)
+    rng = np.random.default_rng(11)
+    rows, refs = [], []
+    for s in range(w.num_seqs):
+        q0, q1 = int(w.query_start[s]), int(w.query_start[s + 1])
+        pick = {q0, q1 - 1, *rng.integers(q0, q1, size=2).tolist()}
+        for r in sorted(pick):
+            p = int(w.context_lens[s]) - (q1 - q0) + (r - q0)
+            ref = oracle.paged_attn_prefill(w.q[r:r + 1], w.dtype, kp, vp, w.dtype, w.block_tables[s:s + 1],
+                                            np.array([p + 1], np.int32), np.array([0, 1], np.int32), w.scale)
+            rows.append(r)
+            refs.append(ref[0])
+    ok, rep = prefill_close(o[rows], np.stack(refs), w.dtype, vmax)
+    assert ok, rep
