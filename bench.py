@@ -224,6 +224,189 @@ class DeviceStep:
         self.decode_op()
 
 
+class PrefillStep:
+    """The chunked-prefill workload on one GPU: the cache built, the chunk's inputs resident."""
+
+    def __init__(self, w: wl.PrefillWorkload, dev):
+        import torch
+        from paged_kv_cache_324_b200 import binding as B
+        self.w, self.dev, self.B = w, dev, B
+        self.stream = torch.cuda.current_stream(dev)
+        t16 = {"f16": torch.float16, "bf16": torch.bfloat16}
+
+        def up(bits):
+            return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(t16[w.dtype])
+
+        self.k_pool, self.v_pool = up(w.initial_pool("k")), up(w.initial_pool("v"))
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+        for op in w.setup:
+            if op.slots.size:
+                B.reshape_and_cache(up(op.k), up(op.v), self.k_pool, self.v_pool, torch.from_numpy(op.slots).to(dev),
+                                    device_error=self.err)
+        sc = w.step_scatter
+        self.host = {"q": w.q, "k_new": sc.k, "v_new": sc.v, "slots": sc.slots, "tables": w.block_tables,
+                     "lens": w.context_lens, "qstart": w.query_start}
+        self.d = {"q": up(w.q), "k_new": up(sc.k), "v_new": up(sc.v), "slots": torch.from_numpy(sc.slots).to(dev),
+                  "tables": torch.from_numpy(w.block_tables).to(dev), "lens": torch.from_numpy(w.context_lens).to(dev),
+                  "qstart": torch.from_numpy(w.query_start).to(dev)}
+        self.out = torch.empty_like(self.d["q"])
+        torch.cuda.synchronize(dev)
+        assert int(self.err.item()) == 0, "setup raised a device error"
+
+    def scatter_op(self):
+        self.B.reshape_and_cache(self.d["k_new"], self.d["v_new"], self.k_pool, self.v_pool, self.d["slots"],
+                                 device_error=self.err, stream=self.stream)
+
+    def prefill_op(self):
+        w = self.w
+        self.B.paged_attn_prefill(self.out, self.d["q"], self.k_pool, self.v_pool, self.d["tables"], self.d["lens"],
+                                  self.d["qstart"], float(w.scale), max_query_len=w.max_query_len,
+                                  device_error=self.err, stream=self.stream)
+
+    def step(self):
+        self.scatter_op()
+        self.prefill_op()
+
+
+PREFILL_METRIC = "paged prefill attention TFLOP/s (causal chunk over the paged cache)"
+
+
+def tensor_peak():
+    try:
+        d = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        return float(d["bf16_tflops"]), float(d["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 1590.0, 1400.0, "fallback"
+
+
+def run_prefill(args, rank, world, local_rank):
+    """The chunked-prefill step (scatter of the chunk's K/V, then the prefill) timed like decode."""
+    import torch
+    dist_on = world > 1
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = wl.make_prefill()
+    ps = PrefillStep(w, dev)
+    flops = wl.prefill_flops(w)
+    for _ in range(args.warmup):
+        ps.step()
+    barrier_sync(torch, dist_on)
+    K = args.steps
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        barrier_sync(torch, dist_on)
+        start.record()
+        for _ in range(K):
+            ps.step()
+        end.record()
+        barrier_sync(torch, dist_on)
+    ms_step = max_over_ranks(torch, start.elapsed_time(end), dist_on) / K
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    barrier_sync(torch, dist_on)
+    for i in range(K):
+        ev[i][0].record()
+        ps.scatter_op()
+        ev[i][1].record()
+        ps.prefill_op()
+        ev[i][2].record()
+    barrier_sync(torch, dist_on)
+    assert int(ps.err.item()) == 0, "device error during the timed region"
+    pf_ms = sum(ev[i][1].elapsed_time(ev[i][2]) for i in range(K)) / K
+    sc_ms = sum(ev[i][0].elapsed_time(ev[i][1]) for i in range(K)) / K
+    total_flops = sum_over_ranks(torch, float(flops), dist_on)
+    value = total_flops / (ms_step * 1e-3) / 1e12
+
+    pinned = {k: torch.from_numpy(np.ascontiguousarray(v).view(np.int16) if v.dtype == np.uint16
+                                  else np.ascontiguousarray(v)).pin_memory() for k, v in ps.host.items()}
+    dq = {k: (ps.d[k].view(torch.int16) if ps.d[k].dtype in (torch.float16, torch.bfloat16) else ps.d[k])
+          for k in pinned}
+    out_host = torch.empty(ps.out.shape, dtype=ps.out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step():
+        for k, v in pinned.items():
+            dq[k].copy_(v, non_blocking=True)
+        ps.step()
+        out_host.copy_(ps.out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    barrier_sync(torch, dist_on)
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record()
+    for _ in range(K):
+        e2e_step()
+    e2.record()
+    barrier_sync(torch, dist_on)
+    e2e_ms = max_over_ranks(torch, s2.elapsed_time(e2), dist_on) / K
+    peak, peak_sus, kind = tensor_peak()
+    achieved = flops / (pf_ms * 1e-3) / 1e12
+    line = {
+        "metric": PREFILL_METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype + " operands, f32 accumulate",
+        "data": "synthetic (seeded N(0,1) q/K/V; random-byte pool content in unwritten slots)",
+        "config": {"workload": w.description, "name": w.name, "num_seqs": w.num_seqs, "num_tokens": w.num_tokens,
+                   "num_heads": w.num_heads, "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
+                   "block_size": w.block_size, "num_blocks": w.num_blocks,
+                   "total_context_tokens": int(w.context_lens.sum()), "flops_per_step": flops,
+                   "step": "reshape_and_cache (the chunk's K/V) + paged_attn_prefill",
+                   "l2": "no flush: the step reads %.0f MB of K/V and q, %.0f MB of output are written; the "
+                         "kernel is bound by the tensor cores, not HBM" % (wl.prefill_bytes(w) / 1e6,
+                                                                           w.num_tokens * w.num_heads * w.head_dim * 2 / 1e6),
+                   "parallelism": f"dp{world}" if world > 1 else "single GPU"},
+        "tokens_per_s": round(sum_over_ranks(torch, float(w.num_tokens), dist_on) / (ms_step * 1e-3), 1),
+        "kernel_ms": {"paged_attn_prefill": round(pf_ms, 5), "reshape_and_cache": round(sc_ms, 5)},
+        "roofline": {"bound": "tensor", "kernel": "paged_prefill_kernel", "achieved": round(achieved, 2),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "frac_of_sustained": round(achieved / peak_sus, 4), "traffic": None,
+                     "flops_per_launch": flops,
+                     "flops_counted": "4 * head_dim * num_heads * causal (query, key) pairs",
+                     "peak_kind": f"{kind} (cuBLAS bf16, burst; sustained {peak_sus})"},
+        "e2e": {"value": round(total_flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 2 * K,
+        "timing": ("value: CUDA events around K back-to-back steps; kernel_ms and roofline: CUDA events "
+                   "around each call in a second run of K steps"),
+        "clocks": clk.report(),
+    }
+    return line, w
+
+
+class PrefillOracleRunner:
+    """The float64 oracle's prefill on the host's cores, holding the workload's pools (built once)."""
+
+    def __init__(self, w: wl.PrefillWorkload):
+        import oracle
+        self.o, self.w = oracle, w
+        self.kp, self.vp = w.initial_pool("k"), w.initial_pool("v")
+        for op in list(w.setup) + [w.step_scatter]:
+            if op.slots.size:
+                oracle.reshape_and_cache(op.k, op.v, w.dtype, self.kp, self.vp, w.dtype, op.slots)
+        self.rng = np.random.default_rng(12)
+        self.cores = os.cpu_count() or 1
+
+    def sample(self, budget_s: float, slice_rows: int = 64):
+        """Slices of ``slice_rows`` consecutive query rows of random chunks, each over its full
+        causal prefix, until the budget is spent (at least one); returns (rows, flops, seconds)."""
+        w, o = self.w, self.o
+        rows, flops, t0 = 0, 0, time.perf_counter()
+        while True:
+            s = int(self.rng.integers(0, w.num_seqs))
+            q0, q1 = int(w.query_start[s]), int(w.query_start[s + 1])
+            n = min(slice_rows, q1 - q0)
+            r0 = int(self.rng.integers(q0, q1 - n + 1))
+            L = int(w.context_lens[s]) - (q1 - q0) + (r0 - q0) + n
+            o.paged_attn_prefill(w.q[r0:r0 + n], w.dtype, self.kp, self.vp, w.dtype, w.block_tables[s:s + 1],
+                                 np.array([L], np.int32), np.array([0, n], np.int32), w.scale, threads=self.cores)
+            rows += n
+            flops += 4 * w.head_dim * w.num_heads * (n * (L - n) + n * (n + 1) // 2)
+            el = time.perf_counter() - t0
+            if el >= budget_s:
+                return rows, flops, el
+
+
 def barrier_sync(torch, dist_on):
     if dist_on:
         import torch.distributed as dist
@@ -444,7 +627,9 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--config", default="opt13b", choices=list(wl.NAMES) + list(wl.EXTRA_NAMES) + list(wl.COMPACT_NAMES))
+    ap.add_argument("--config", default="opt13b",
+                    choices=list(wl.NAMES) + list(wl.EXTRA_NAMES) + list(wl.COMPACT_NAMES) + ["prefill"],
+                    help="a decode workload, or 'prefill' (chunked prefill, reported in TFLOP/s)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--prefix-aware", action="store_true",
                     help="decode with pkv_paged_attn_decode_shared_prefix (shared prompts read once per unit)")
@@ -457,6 +642,34 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference" and args.config == "prefill":
+        if rank != 0:
+            return
+        w = wl.make_prefill()
+        r = PrefillOracleRunner(w)
+        cores = r.cores
+        per_step = min(30.0, 150.0 / (args.steps + args.warmup))
+        slice_rows = 64 if per_step >= 5.0 else 1      # one row over ~2k keys takes tens of ms
+        rates, times = [], []
+        for i in range(args.warmup + args.steps):
+            rows, flops, el = r.sample(per_step, slice_rows)
+            if i >= args.warmup:
+                rates.append(flops / el)
+                times.append(el)
+        value = sum(rates) / len(rates) / 1e12
+        sample = (f"{slice_rows}-row slices of random chunks (float64 prefill, each row over its full causal "
+                  f"prefix), ~{per_step:.2f} s per step, {len(times)} timed steps")
+        line = {"metric": PREFILL_METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * sum(times) / len(times), 3),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "impl": "reference",
+                "dtype": "f64", "data": "synthetic", "config": {"workload": w.description, "name": w.name},
+                "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                                 "sample": sample},
+                "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
 
     if args.impl == "reference":
         if rank != 0:
@@ -499,6 +712,18 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
+        if args.config == "prefill":
+            line, w = run_prefill(args, rank, world, local_rank)
+            if rank == 0 and world == 1:
+                r = PrefillOracleRunner(w)
+                rows, flops, el = r.sample(args.cpu_budget)
+                line["cpu_baseline"] = {"value": round(flops / el / 1e12, 6), "unit": "TFLOP/s", "cores": r.cores,
+                                        "kind": "oracle",
+                                        "sample": f"{rows} query rows (64-row slices of random chunks, each over "
+                                                  f"its full causal prefix, float64), {el:.1f} s"}
+            if rank == 0:
+                print(json.dumps(line), flush=True)
+            return
         line, w = run_ours(args, rank, world, local_rank)
         if rank == 0 and world == 1:
             n, nbytes, el, cores = cpu_oracle_sample(w, args.cpu_budget)
