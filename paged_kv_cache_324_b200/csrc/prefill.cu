@@ -12,11 +12,13 @@
 // the block table.  Warp roles:
 //   warp 0     TMA: the Q tile once, then K and V tiles block by block (one
 //              4-D box per 16- or 32-token block and 64-column chunk) into
-//              128-byte-swizzled rings (3 K stages, 2 V stages);
+//              128-byte-swizzled rings (2 K stages, 2 V stages);
 //   warp 1     allocates 512 TMEM columns; one thread issues the MMAs:
 //              S_j = Q K_j^T into one of two TMEM buffers (M=128, N=128),
 //              and O += P_j V_j (M=128, N=head_dim) once P_j is written;
-//   warps 2-5  softmax, one query row per thread (TMEM lane = row): read S_j
+//   warps 2-9  softmax, two warps per TMEM lane quarter: each thread takes
+//              64 of one row's 128 keys (TMEM lane = row); the two halves of a
+//              row exchange their maxima through shared memory.  Read S_j
 //              with tcgen05.ld, mask, online softmax in base 2 with a running
 //              maximum that is only moved when the new one exceeds it by more
 //              than 2^8 (the result does not depend on the reference maximum;
@@ -47,9 +49,10 @@ namespace {
 
 constexpr int kRows = 128;            // query rows per CTA: MMA M, one TMEM lane each
 constexpr int kKeys = 128;            // keys per tile: N of S = Q K^T, K of O += P V
-constexpr int kKStages = 3;
+constexpr int kKStages = 2;
 constexpr int kVStages = 2;
-constexpr int kPThreads = 192;        // warp 0 TMA, warp 1 MMA, warps 2-5 softmax
+constexpr int kPThreads = 320;        // warp 0 TMA, warp 1 MMA, warps 2-9 softmax
+constexpr int kSoftmaxWarps = 8;      // two per TMEM lane quarter: each takes 64 of a row's 128 keys
 constexpr uint32_t kTmemCols = 512;   // S buffers at columns 0 and 128, O at 256
 constexpr uint32_t kTmemO = 256;
 constexpr float kMaxLag = 8.0f;       // log2 of the largest weight the lagging maximum allows
@@ -152,6 +155,39 @@ __device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, uint32_t (&r)[32]
         : "memory");
 }
 
+__device__ __forceinline__ void tmem_ld64_wait(uint32_t taddr, uint32_t (&r)[64]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+          "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+          "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+          "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+          "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "r"(taddr));
+    asm volatile(
+        "tcgen05.wait::ld.sync.aligned;"
+        : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+          "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+          "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+          "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]),
+          "+r"(r[32]), "+r"(r[33]), "+r"(r[34]), "+r"(r[35]), "+r"(r[36]), "+r"(r[37]), "+r"(r[38]), "+r"(r[39]),
+          "+r"(r[40]), "+r"(r[41]), "+r"(r[42]), "+r"(r[43]), "+r"(r[44]), "+r"(r[45]), "+r"(r[46]), "+r"(r[47]),
+          "+r"(r[48]), "+r"(r[49]), "+r"(r[50]), "+r"(r[51]), "+r"(r[52]), "+r"(r[53]), "+r"(r[54]), "+r"(r[55]),
+          "+r"(r[56]), "+r"(r[57]), "+r"(r[58]), "+r"(r[59]), "+r"(r[60]), "+r"(r[61]), "+r"(r[62]), "+r"(r[63])
+        :
+        : "memory");
+}
+
+// 2^x with the multi-function unit's approximation (subnormal results flush to zero).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
@@ -234,8 +270,10 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
     constexpr int kTB = kKeys / BS;                  // blocks per key tile
     constexpr uint32_t kBoxBytes = BS * 128;         // one block x one 64-column chunk
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t bars[2 * kKStages + 2 * kVStages + 8];
+    __shared__ __align__(8) uint64_t bars[2 * kKStages + 2 * kVStages + 8 + 4];
     __shared__ CtaFlags flags;
+    __shared__ float red[2][2][kRows];   // [tile parity][half][row]: partial row maxima
+    __shared__ float red_l[2][kRows];    // [half][row]: partial row sums at the end
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = a.group, TQ = kRows / G;
@@ -282,6 +320,7 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
     auto s_full = [&](int i) { return bar_q + 8u * (1 + i); };
     auto s_empty = [&](int i) { return bar_q + 8u * (3 + i); };
     const uint32_t p_full = bar_q + 8u * 5, o_done = bar_q + 8u * 6, drain = bar_q + 8u * 7;
+    auto xchg = [&](int quarter) { return bar_q + 8u * (8 + quarter); };   // the two warps of a lane quarter
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kKStages; ++i) {
@@ -295,9 +334,10 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
         mbar_init(bar_q, 1);
         mbar_init(s_full(0), 1);
         mbar_init(s_full(1), 1);
-        mbar_init(s_empty(0), 4);
-        mbar_init(s_empty(1), 4);
-        mbar_init(p_full, 4);
+        mbar_init(s_empty(0), kSoftmaxWarps);
+        mbar_init(s_empty(1), kSoftmaxWarps);
+        mbar_init(p_full, kSoftmaxWarps);
+        for (int i = 0; i < 4; ++i) mbar_init(xchg(i), 2);
         mbar_init(o_done, 1);
         mbar_init(drain, 1);
         flags.abort = 0;
@@ -418,86 +458,92 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
         }
         __syncwarp();
     } else {
-        // ---------------- softmax (warps 2-5, one row per thread) ----------------
+        // ---------------- softmax (warps 2-9: row = TMEM lane, half = which 64 keys) ----------------
         const int quarter = warp & 3;
+        const int half = (warp - 2) >> 2;
         const int row = quarter * 32 + lane;
         const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
         const int tq = row / G;
         const int pq = min(L - C + t0 + tq, L - 1);
+        constexpr int kHalf = kKeys / 2;
+        constexpr int kOCols = D / 2;                        // O columns this thread rescales and stores
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; j < ntk; ++j) {
             const int buf = j & 1;
             if (!warp_wait_bar(s_full(buf), (j >> 1) & 1, &flags, a.err)) { ok = false; break; }
             tc_fence_after();
-            float x[kKeys];
+            float x[kHalf];
+            {
+                uint32_t r[kHalf];
+                tmem_ld64_wait(trow + buf * kKeys + half * kHalf, r);
 #pragma unroll
-            for (int c = 0; c < kKeys / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32_wait(trow + buf * kKeys + c * 32, r);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(r[i]);
+                for (int i = 0; i < kHalf; ++i) x[i] = __uint_as_float(r[i]);
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(s_empty(buf));
-            const int kbase = j * kKeys;
-            if (kbase + kKeys - 1 > pq) {
+            const int kbase = j * kKeys + half * kHalf;
+            if (kbase + kHalf - 1 > pq) {
 #pragma unroll
-                for (int c = 0; c < kKeys; ++c) x[c] = (kbase + c > pq) ? -INFINITY : x[c];
+                for (int c = 0; c < kHalf; ++c) x[c] = (kbase + c > pq) ? -INFINITY : x[c];
             }
             float mx = x[0];
 #pragma unroll
-            for (int c = 1; c < kKeys; ++c) mx = fmaxf(mx, x[c]);
+            for (int c = 1; c < kHalf; ++c) mx = fmaxf(mx, x[c]);
+            // the row's maximum over both halves: exchange through shared memory
+            red[buf][half][row] = mx;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(xchg(quarter));
+            if (!warp_wait_bar(xchg(quarter), j & 1, &flags, a.err)) { ok = false; break; }
+            mx = fmaxf(mx, red[buf][half ^ 1][row]);
             const float m_cand = mx * a.scale_log2;
             const bool move = m_cand > m_used + kMaxLag;
             float alpha = 1.f;
             if (move) {
-                alpha = exp2f(m_used - m_cand);
+                alpha = ex2(m_used - m_cand);
                 m_used = m_cand;
             }
             const float neg_m = -m_used;
-            uint32_t pk[kKeys / 2];
+            uint32_t pk[kHalf / 2];
             float sum = 0.f;
 #pragma unroll
-            for (int c = 0; c < kKeys; c += 2) {
-                const float p0 = exp2f(fmaf(x[c], a.scale_log2, neg_m));
-                const float p1 = exp2f(fmaf(x[c + 1], a.scale_log2, neg_m));
+            for (int c = 0; c < kHalf; c += 2) {
+                const float p0 = ex2(fmaf(x[c], a.scale_log2, neg_m));
+                const float p1 = ex2(fmaf(x[c + 1], a.scale_log2, neg_m));
                 sum += p0 + p1;
                 pk[c / 2] = pack2<kBf16>(p0, p1);
             }
-            l = l * alpha + sum;
+            l = l * alpha + sum;                             // this half's share of the row sum
             // P and O are free once the previous P.V product has completed
             if (j > 0 && !warp_wait_bar(o_done, (j - 1) & 1, &flags, a.err)) { ok = false; break; }
             if (j > 0 && __any_sync(0xffffffffu, move)) {
                 tc_fence_after();
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
+                for (int c = 0; c < kOCols / 32; ++c) {
                     uint32_t r[32];
-                    tmem_ld32_wait(trow + kTmemO + c * 32, r);
+                    tmem_ld32_wait(trow + kTmemO + half * kOCols + c * 32, r);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                    tmem_st32(trow + kTmemO + c * 32, r);
+                    tmem_st32(trow + kTmemO + half * kOCols + c * 32, r);
                 }
                 tmem_wait_st();
             }
-            // P row: keys as K, 64 keys per 128-byte chunk row, 16-byte units swizzled by row % 8
+            // this half's 64 keys are P's 64-key chunk `half`: one 128-byte row, units swizzled by row % 8
 #pragma unroll
-            for (int u = 0; u < kKeys / 8; ++u) {
-                const uint32_t addr = sP + (u >> 3) * kChunkBytes + row * 128 + (((u & 7) ^ (row & 7)) << 4);
+            for (int u = 0; u < 8; ++u) {
+                const uint32_t addr = sP + half * kChunkBytes + row * 128 + ((u ^ (row & 7)) << 4);
                 sts128(addr, pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
             }
-            if (j == ntk - 1 && kbase + kKeys - 1 > pq_max) {
+            if (j == ntk - 1 && j * kKeys + kKeys - 1 > pq_max) {
                 // keys past pq_max were not loaded (or are unwritten slots): zero their V rows
                 const int vs = j % kVStages;
                 if (!warp_wait_bar(v_full(vs), (j / kVStages) & 1, &flags, a.err)) { ok = false; break; }
-                if (kbase + row > pq_max) {
+                if (half < Gm::kChunks && j * kKeys + row > pq_max) {
 #pragma unroll
-                    for (int c = 0; c < Gm::kChunks; ++c)
-#pragma unroll
-                        for (int u = 0; u < 8; ++u)
-                            sts128(sV + vs * Gm::kTile + c * kChunkBytes + row * 128 + (((u ^ (row & 7)) & 7) << 4), 0u,
-                                   0u, 0u, 0u);
+                    for (int u = 0; u < 8; ++u)
+                        sts128(sV + vs * Gm::kTile + half * kChunkBytes + row * 128 + ((u ^ (row & 7)) << 4), 0u, 0u,
+                               0u, 0u);
                 }
             }
             fence_proxy_async_smem();
@@ -506,6 +552,7 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
             if (lane == 0) mbar_arrive(p_full);
         }
         if (ok) ok = warp_wait_bar(o_done, (ntk - 1) & 1, &flags, a.err);
+        red_l[half][row] = l;                                // read back after the barrier below
         pdl_trigger();
         // the output is written after the CTA-wide barrier below, which also publishes flags.bad
         tc_fence_before();
@@ -515,12 +562,13 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
         const bool live = tq < rows_valid;
         const bool nan_out = !ok || flags.bad || *reinterpret_cast<volatile int*>(&flags.abort);
         uint16_t* orow = reinterpret_cast<uint16_t*>(a.out) +
-                         (static_cast<size_t>(q0 + t0 + (live ? tq : 0)) * a.num_heads + kvh * G + row % G) * D;
-        const float inv = 1.f / l;
+                         (static_cast<size_t>(q0 + t0 + (live ? tq : 0)) * a.num_heads + kvh * G + row % G) * D +
+                         half * kOCols;
+        const float inv = 1.f / (red_l[0][row] + red_l[1][row]);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < kOCols / 32; ++c) {
             uint32_t r[32];
-            tmem_ld32_wait(trow + kTmemO + c * 32, r);
+            tmem_ld32_wait(trow + kTmemO + half * kOCols + c * 32, r);
             if (live) {
                 uint32_t w[16];
 #pragma unroll
