@@ -10,9 +10,10 @@
 // One CTA = 128 query rows (128 / G tokens x the G query heads of one KV
 // head) of one sequence, against 128-key tiles of that KV head read through
 // the block table.  Warp roles:
-//   warp 0     TMA: the Q tile once, then K and V tiles block by block (one
-//              4-D box per 16- or 32-token block and 64-column chunk) into
-//              128-byte-swizzled rings (2 K stages, 2 V stages);
+//   warps 0,10 TMA: warp 0 the Q tile once, then K tiles, warp 10 V tiles,
+//              block by block (one 4-D box per 16- or 32-token block and
+//              64-column chunk) into 128-byte-swizzled rings of two stages,
+//              each warp reading its table entries one tile ahead;
 //   warp 1     allocates 512 TMEM columns; one thread issues the MMAs:
 //              S_j = Q K_j^T into one of two TMEM buffers (M=128, N=128),
 //              and O += P_j V_j (M=128, N=head_dim) once P_j is written;
@@ -49,9 +50,10 @@ namespace {
 
 constexpr int kRows = 128;            // query rows per CTA: MMA M, one TMEM lane each
 constexpr int kKeys = 128;            // keys per tile: N of S = Q K^T, K of O += P V
-constexpr int kKStages = 2;
+constexpr int kKStages = 2;           // the producers' ring arithmetic assumes two stages each
 constexpr int kVStages = 2;
-constexpr int kPThreads = 320;        // warp 0 TMA, warp 1 MMA, warps 2-9 softmax
+constexpr int kPThreads = 352;        // warp 0 TMA (Q, K), warp 1 MMA, warps 2-9 softmax, warp 10 TMA (V)
+constexpr int kVWarp = 10;
 constexpr int kSoftmaxWarps = 8;      // two per TMEM lane quarter: each takes 64 of a row's 128 keys
 constexpr uint32_t kTmemCols = 512;   // S buffers at columns 0 and 128, O at 256
 constexpr uint32_t kTmemO = 256;
@@ -356,10 +358,11 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
     tc_fence_after();
     const uint32_t tmem = flags.tmem_base;
 
-    if (warp == 0) {
-        // ---------------- TMA producer ----------------
+    if (warp == 0 || warp == kVWarp) {
+        // ---------------- TMA producers: warp 0 loads Q and K, warp 10 loads V ----------------
+        const bool is_k = warp == 0;
         const uint64_t pol = l2_policy_evict_last();      // K/V tiles are read again by the other query tiles
-        if (lane == 0) {
+        if (is_k && lane == 0) {
             tma_prefetch_desc(&qmap);
             tma_prefetch_desc(&kmap);
             tma_prefetch_desc(&vmap);
@@ -367,53 +370,45 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
 #pragma unroll
             for (int c = 0; c < Gm::kChunks; ++c) tma_load_3d(sQ + c * kChunkBytes, &qmap, bar_q, c * 64, kvh * G, q0 + t0);
         }
+        const CUtensorMap* map = is_k ? &kmap : &vmap;
+        const uint32_t ring = is_k ? sK : sV;
         const int32_t* trow = a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq;
-        int k_issued = 0, v_issued = 0;   // tiles whose K (V) copies were issued
+        int issued = 0;                                   // tiles whose copies were issued
+        // table entries are read one tile ahead so that their latency hides behind the copies
+        int pid_next = (lane < kTB && lane < nblk) ? __ldg(trow + lane) : -1;
         for (int j = 0; j < ntk; ++j) {
-            const int blk = j * kTB + lane;
-            const bool want = lane < kTB && blk < nblk;
-            const int pid = want ? __ldg(trow + blk) : -1;
+            const int pid = pid_next;
+            const int nb = (j + 1) * kTB + lane;
+            pid_next = (j + 1 < ntk && lane < kTB && nb < nblk) ? __ldg(trow + nb) : -1;
+            const bool want = lane < kTB && j * kTB + lane < nblk;
             const bool bad = want && (pid < 0 || pid >= a.num_blocks);
             const unsigned ok_mask = __ballot_sync(0xffffffffu, want && !bad);
-            if (__any_sync(0xffffffffu, bad) && lane == 0) {
+            if (is_k && __any_sync(0xffffffffu, bad) && lane == 0) {
                 raise_error(a.err, PKV_DEVERR_BLOCK_ID);
                 flags.bad = 1;
             }
             const uint32_t bytes = __popc(ok_mask) * kBoxBytes * Gm::kChunks;
-            const int ks = j % kKStages, vs = j % kVStages;
-            if (j >= kKStages && !warp_wait_bar(k_empty(ks), ((j / kKStages) - 1) & 1, &flags, a.err)) break;
-            if (lane == 0) mbar_arrive_expect_tx(k_full(ks), bytes);
-            k_issued = j + 1;
+            const int st = j % 2;                          // both rings have two stages
+            const uint32_t full = is_k ? k_full(st) : v_full(st), empty = is_k ? k_empty(st) : v_empty(st);
+            if (j >= 2 && !warp_wait_bar(empty, ((j / 2) - 1) & 1, &flags, a.err)) break;
+            if (lane == 0) mbar_arrive_expect_tx(full, bytes);
+            issued = j + 1;
             for (int b = 0; b < kTB; ++b) {
                 const int p = __shfl_sync(0xffffffffu, pid, b);
                 if (lane == 0 && ((ok_mask >> b) & 1u)) {
 #pragma unroll
                     for (int c = 0; c < Gm::kChunks; ++c)
-                        tma_load_4d(sK + ks * Gm::kTile + c * kChunkBytes + b * kBoxBytes, &kmap, k_full(ks), c * 64,
-                                    0, kvh, p, pol);
-                }
-            }
-            if (j >= kVStages && !warp_wait_bar(v_empty(vs), ((j / kVStages) - 1) & 1, &flags, a.err)) break;
-            if (lane == 0) mbar_arrive_expect_tx(v_full(vs), bytes);
-            v_issued = j + 1;
-            for (int b = 0; b < kTB; ++b) {
-                const int p = __shfl_sync(0xffffffffu, pid, b);
-                if (lane == 0 && ((ok_mask >> b) & 1u)) {
-#pragma unroll
-                    for (int c = 0; c < Gm::kChunks; ++c)
-                        tma_load_4d(sV + vs * Gm::kTile + c * kChunkBytes + b * kBoxBytes, &vmap, v_full(vs), c * 64,
-                                    0, kvh, p, pol);
+                        tma_load_4d(ring + st * Gm::kTile + c * kChunkBytes + b * kBoxBytes, map, full, c * 64, 0, kvh,
+                                    p, pol);
                 }
             }
         }
         // drain: the last copies of each stage must land before the CTA may exit
         if (lane == 0) {
             const uint64_t end = global_timer_ns() + kWaitLimitNs;
-            mbar_wait(bar_q, 0, end);
-            for (int j = max(0, k_issued - kKStages); j < k_issued; ++j)
-                mbar_wait(k_full(j % kKStages), (j / kKStages) & 1, end);
-            for (int j = max(0, v_issued - kVStages); j < v_issued; ++j)
-                mbar_wait(v_full(j % kVStages), (j / kVStages) & 1, end);
+            if (is_k) mbar_wait(bar_q, 0, end);
+            for (int j = max(0, issued - 2); j < issued; ++j)
+                mbar_wait(is_k ? k_full(j % 2) : v_full(j % 2), (j / 2) & 1, end);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer (one thread) ----------------
@@ -460,7 +455,7 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
     } else {
         // ---------------- softmax (warps 2-9: row = TMEM lane, half = which 64 keys) ----------------
         const int quarter = warp & 3;
-        const int half = (warp - 2) >> 2;
+        const int half = (warp - 2) >> 2;                   // warps 2-5: keys 0-63, warps 6-9: keys 64-127
         const int row = quarter * 32 + lane;
         const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
         const int tq = row / G;
@@ -488,9 +483,13 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
 #pragma unroll
                 for (int c = 0; c < kHalf; ++c) x[c] = (kbase + c > pq) ? -INFINITY : x[c];
             }
-            float mx = x[0];
+            float mp[8];                                      // eight independent chains, then a tree
 #pragma unroll
-            for (int c = 1; c < kHalf; ++c) mx = fmaxf(mx, x[c]);
+            for (int i = 0; i < 8; ++i) mp[i] = x[i];
+#pragma unroll
+            for (int c = 8; c < kHalf; ++c) mp[c & 7] = fmaxf(mp[c & 7], x[c]);
+            float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
             // the row's maximum over both halves: exchange through shared memory
             red[buf][half][row] = mx;
             __syncwarp();
@@ -506,14 +505,15 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
             }
             const float neg_m = -m_used;
             uint32_t pk[kHalf / 2];
-            float sum = 0.f;
+            float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int c = 0; c < kHalf; c += 2) {
                 const float p0 = ex2(fmaf(x[c], a.scale_log2, neg_m));
                 const float p1 = ex2(fmaf(x[c + 1], a.scale_log2, neg_m));
-                sum += p0 + p1;
+                sp[(c >> 1) & 7] += p0 + p1;
                 pk[c / 2] = pack2<kBf16>(p0, p1);
             }
+            const float sum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
             l = l * alpha + sum;                             // this half's share of the row sum
             // P and O are free once the previous P.V product has completed
             if (j > 0 && !warp_wait_bar(o_done, (j - 1) & 1, &flags, a.err)) { ok = false; break; }
