@@ -54,6 +54,16 @@ NCU_TRAFFIC = {
 }
 
 
+# the same for the prefill kernel (sha256 prefix of prefill.cu), on the prefill workload
+PREFILL_TRAFFIC = {"bytes_per_launch": 569_860_352, "kernel_sha": "92b4d97290f49bc4",
+                   "capture": "profiles/paged_prefill_kernel_prefill.md"}
+
+
+def prefill_source_sha() -> str:
+    p = os.path.join(ROOT, "paged_kv_cache_324_b200", "csrc", "prefill.cu")
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+
+
 def decode_source_sha() -> str:
     p = os.path.join(ROOT, "paged_kv_cache_324_b200", "csrc", "decode.cu")
     return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
@@ -360,7 +370,9 @@ def run_prefill(args, rank, world, local_rank):
         "kernel_ms": {"paged_attn_prefill": round(pf_ms, 5), "reshape_and_cache": round(sc_ms, 5)},
         "roofline": {"bound": "tensor", "kernel": "paged_prefill_kernel", "achieved": round(achieved, 2),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                     "frac_of_sustained": round(achieved / peak_sus, 4), "traffic": None,
+                     "frac_of_sustained": round(achieved / peak_sus, 4),
+                     "traffic": (PREFILL_TRAFFIC["bytes_per_launch"]
+                                 if PREFILL_TRAFFIC["kernel_sha"] == prefill_source_sha() else None),
                      "flops_per_launch": flops,
                      "flops_counted": "4 * head_dim * num_heads * causal (query, key) pairs",
                      "peak_kind": f"{kind} (cuBLAS bf16, burst; sustained {peak_sus})"},
