@@ -419,6 +419,119 @@ class PrefillOracleRunner:
                 return rows, flops, el
 
 
+SWAP_METRIC = "block swap GB/s over the host link (GPU pool <-> pinned host pool, both directions)"
+
+
+def run_swap(args, rank, world, local_rank):
+    """Preemption by swapping: each step moves a group's blocks GPU -> pinned host (pkv_swap_blocks)
+    and another group's blocks host -> GPU.  Pools of the OPT-13B layer shape."""
+    import torch
+    from paged_kv_cache_324_b200 import binding as B
+    dist_on = world > 1
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    NB, NH, Hkv, Bs, D, n = 16384, 4096, 40, 16, 128, 1024     # 1024 blocks = 16 sequences of 1,024 tokens
+    rng = np.random.default_rng(7)
+    kp = torch.empty((NB, Hkv, Bs, D), dtype=torch.float16, device=dev).normal_()
+    vp = torch.empty_like(kp).normal_()
+    hk = torch.empty((NH, Hkv, Bs, D), dtype=torch.float16).pin_memory()
+    hv = torch.empty_like(hk).pin_memory()
+    block_bytes = Hkv * Bs * D * 2
+    out_pairs = np.stack([rng.choice(NB, n, replace=False), rng.choice(NH // 2, n, replace=False)], axis=1)
+    in_pairs = np.stack([NH // 2 + rng.choice(NH // 2, n, replace=False), rng.choice(NB, n, replace=False)], axis=1)
+    host_pairs = {"out": out_pairs.astype(np.int64), "in": in_pairs.astype(np.int64)}
+    dpairs = {k: torch.from_numpy(v).to(dev) for k, v in host_pairs.items()}
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    step_bytes = 2 * 2 * n * block_bytes                         # K and V, out and in
+
+    def step():
+        B.swap_blocks(kp, vp, hk, hv, dpairs["out"], device_error=err)
+        B.swap_blocks(hk, hv, kp, vp, dpairs["in"], device_error=err)
+
+    for _ in range(args.warmup):
+        step()
+    K = args.steps
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        barrier_sync(torch, dist_on)
+        start.record()
+        for _ in range(K):
+            step()
+        end.record()
+        barrier_sync(torch, dist_on)
+    ms_step = max_over_ranks(torch, start.elapsed_time(end), dist_on) / K
+    assert int(err.item()) == 0, "device error during the timed region"
+    # per direction, and the copy engines' rate for the same bytes (the link's measured peak here)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    ev[0].record()
+    for _ in range(K):
+        B.swap_blocks(kp, vp, hk, hv, dpairs["out"], device_error=err)
+    ev[1].record()
+    for _ in range(K):
+        B.swap_blocks(hk, hv, kp, vp, dpairs["in"], device_error=err)
+    ev[2].record()
+    torch.cuda.synchronize()
+    out_ms, in_ms = ev[0].elapsed_time(ev[1]) / K, ev[1].elapsed_time(ev[2]) / K
+    nbytes = n * block_bytes
+    big_d, big_h = torch.empty(nbytes, dtype=torch.uint8, device=dev), torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    ce = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    for _ in range(2):
+        big_h.copy_(big_d, non_blocking=True)
+        big_d.copy_(big_h, non_blocking=True)
+    ce[0].record()
+    for _ in range(4):
+        big_h.copy_(big_d, non_blocking=True)
+    ce[1].record()
+    for _ in range(4):
+        big_d.copy_(big_h, non_blocking=True)
+    ce[2].record()
+    torch.cuda.synchronize()
+    d2h = nbytes / (ce[0].elapsed_time(ce[1]) / 4 * 1e-3) / 1e9
+    h2d = nbytes / (ce[1].elapsed_time(ce[2]) / 4 * 1e-3) / 1e9
+    peak = step_bytes / ((step_bytes / 2) / (d2h * 1e9) + (step_bytes / 2) / (h2d * 1e9)) / 1e9
+    value = sum_over_ranks(torch, float(step_bytes), dist_on) / (ms_step * 1e-3) / 1e9
+    achieved = step_bytes / (ms_step * 1e-3) / 1e9
+    # end to end: the step's pairs come from pinned host memory each step
+    pin = {k: torch.from_numpy(v).pin_memory() for k, v in host_pairs.items()}
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record()
+    for _ in range(K):
+        for k in pin:
+            dpairs[k].copy_(pin[k], non_blocking=True)
+        step()
+        err_h = err.to("cpu", non_blocking=True)
+    e2.record()
+    barrier_sync(torch, dist_on)
+    e2e_ms = max_over_ranks(torch, s2.elapsed_time(e2), dist_on) / K
+    line = {
+        "metric": SWAP_METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16 (bytes moved as is)",
+        "data": "synthetic (N(0,1) pools; random distinct block pairs)",
+        "config": {"workload": f"swap out {n} blocks GPU -> pinned host and {n} blocks host -> GPU per step; "
+                               f"pools [{NB} | {NH}, {Hkv}, {Bs}, {D}] f16 (OPT-13B layer shape)",
+                   "name": "swap", "blocks_per_direction": n, "block_bytes_per_pool": block_bytes,
+                   "step": "pkv_swap_blocks (out) + pkv_swap_blocks (in)",
+                   "l2": "no flush: each step moves %.0f MB, more than the 126 MB L2" % (step_bytes / 1e6),
+                   "parallelism": f"dp{world}" if world > 1 else "single GPU"},
+        "kernel_ms": {"swap_out": round(out_ms, 5), "swap_in": round(in_ms, 5)},
+        "roofline": {"bound": "link", "kernel": "swap_blocks_kernel", "achieved": round(achieved, 2),
+                     "peak": round(peak, 2), "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "bytes_per_step": step_bytes,
+                     "peak_kind": f"measured in this run: copy engines on one {nbytes >> 20} MiB pinned buffer, "
+                                  f"device->host {d2h:.1f} GB/s, host->device {h2d:.1f} GB/s, combined for "
+                                  f"equal bytes each way",
+                     "per_direction_gbs": {"out": round(nbytes * 2 / (out_ms * 1e-3) / 1e9, 2),
+                                           "in": round(nbytes * 2 / (in_ms * 1e-3) / 1e9, 2)}},
+        "e2e": {"value": round(step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s", "ms_per_step": round(e2e_ms, 5),
+                "h2d_bytes_per_step": sum(v.nbytes for v in host_pairs.values()), "d2h_bytes_per_step": 4},
+        "gpu_launches": 2 * K,
+        "timing": "value: CUDA events around K back-to-back steps",
+        "clocks": clk.report(),
+    }
+    return line
+
+
 def barrier_sync(torch, dist_on):
     if dist_on:
         import torch.distributed as dist
@@ -640,8 +753,8 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--config", default="opt13b",
-                    choices=list(wl.NAMES) + list(wl.EXTRA_NAMES) + list(wl.COMPACT_NAMES) + ["prefill"],
-                    help="a decode workload, or 'prefill' (chunked prefill, reported in TFLOP/s)")
+                    choices=list(wl.NAMES) + list(wl.EXTRA_NAMES) + list(wl.COMPACT_NAMES) + ["prefill", "swap"],
+                    help="a decode workload, 'prefill' (chunked prefill, TFLOP/s) or 'swap' (block swap, GB/s)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--prefix-aware", action="store_true",
                     help="decode with pkv_paged_attn_decode_shared_prefix (shared prompts read once per unit)")
@@ -654,6 +767,38 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference" and args.config == "swap":
+        if rank != 0:
+            return
+        # the oracle's block swap (memcpy per block) between two host pools of the same shape
+        import oracle
+        NB, NH, Hkv, Bs, D, n = 16384, 4096, 40, 16, 128, 1024
+        rng = np.random.default_rng(7)
+        gk = np.zeros((NB, Hkv, Bs, D), np.uint16)
+        gv = np.zeros_like(gk)
+        hk = np.zeros((NH, Hkv, Bs, D), np.uint16)
+        hv = np.zeros_like(hk)
+        out_p = np.stack([rng.choice(NB, n, replace=False), rng.choice(NH // 2, n, replace=False)], axis=1)
+        in_p = np.stack([NH // 2 + rng.choice(NH // 2, n, replace=False), rng.choice(NB, n, replace=False)], axis=1)
+        step_bytes = 2 * 2 * n * gk[0].nbytes
+        times = []
+        for i in range(args.warmup + args.steps):
+            t0 = time.perf_counter()
+            oracle.swap_blocks(gk, gv, hk, hv, out_p)
+            oracle.swap_blocks(hk, hv, gk, gv, in_p)
+            if i >= args.warmup:
+                times.append(time.perf_counter() - t0)
+        value = step_bytes / (sum(times) / len(times)) / 1e9
+        line = {"metric": SWAP_METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * sum(times) / len(times), 3),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "impl": "reference",
+                "dtype": "bytes", "data": "synthetic", "config": {"workload": "swap", "name": "swap"},
+                "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                 "sample": f"the whole step (memcpy per block, host memory only), {len(times)} steps"},
+                "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
 
     if args.impl == "reference" and args.config == "prefill":
         if rank != 0:
@@ -724,6 +869,28 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
+        if args.config == "swap":
+            line = run_swap(args, rank, world, local_rank)
+            if rank == 0 and world == 1:
+                import oracle
+                n, NB, NH = 1024, 16384, 4096
+                gk = np.zeros((NB, 40, 16, 128), np.uint16)
+                hk = np.zeros((NH, 40, 16, 128), np.uint16)
+                rng = np.random.default_rng(7)
+                pairs = np.stack([rng.choice(NB, n, replace=False), rng.choice(NH, n, replace=False)], axis=1)
+                t0, steps = time.perf_counter(), 0
+                while time.perf_counter() - t0 < max(args.cpu_budget, 0.5) or steps == 0:
+                    oracle.swap_blocks(gk, gk, hk, hk, pairs)
+                    oracle.swap_blocks(hk, hk, gk, gk, pairs[:, ::-1])
+                    steps += 1
+                el = time.perf_counter() - t0
+                line["cpu_baseline"] = {"value": round(steps * 2 * 2 * n * gk[0].nbytes / el / 1e9, 3), "unit": "GB/s",
+                                        "cores": 1, "kind": "oracle",
+                                        "sample": f"{steps} whole step(s) between two host pools (memcpy per block), "
+                                                  f"{el:.1f} s"}
+            if rank == 0:
+                print(json.dumps(line), flush=True)
+            return
         if args.config == "prefill":
             line, w = run_prefill(args, rank, world, local_rank)
             if rank == 0 and world == 1:

@@ -301,6 +301,24 @@ pkv_status pkv_copy_blocks(void* k_pool, void* v_pool, size_t block_bytes,
                            uint32_t* device_error, void* stream);
 
 /*
+ * Block swap between two pools of the same layout ("vLLM and PagedAttention"
+ * transcript, on preemption: a group's KV data moves to CPU memory and comes
+ * back later): for every pair i,
+ *   dst_k_pool[pairs[i][1]] := src_k_pool[pairs[i][0]] and the same for V,
+ * block_bytes = num_kv_heads * block_size * head_dim * element size, a
+ * multiple of 16.  Each pool is device memory or host memory pinned and
+ * mapped by CUDA (cudaHostAlloc, or torch's pin_memory) -- the kernel reads or
+ * writes it across the link directly; pageable host memory is rejected with
+ * PKV_ERR_INVALID_ARG.  pairs is int64 [num_pairs][2] (src block, dst block),
+ * device or mapped host memory; pkv_bm_swap produces it.  Pairs naming a
+ * block outside [0, src_num_blocks) / [0, dst_num_blocks) are skipped and set
+ * PKV_DEVERR_PAIR.  Destinations must be distinct.
+ */
+pkv_status pkv_swap_blocks(const void* src_k_pool, const void* src_v_pool, int src_num_blocks,
+                           void* dst_k_pool, void* dst_v_pool, int dst_num_blocks, size_t block_bytes,
+                           const int64_t* pairs, int num_pairs, uint32_t* device_error, void* stream);
+
+/*
  * Host-side block manager (no GPU involved): the bookkeeping that produces block
  * tables, slot mappings and copy-on-write pairs for the kernels above
  * (glossary "PagedAttention", sections "How paging works" and "Sharing blocks
@@ -340,6 +358,36 @@ pkv_status pkv_bm_block_tables(pkv_block_manager* m, const int64_t* seq_ids, int
                                int max_blocks, int32_t pad, int32_t* context_lens);
 int pkv_bm_ref_count(pkv_block_manager* m, int32_t block);          /* -1 if out of range */
 int64_t pkv_bm_sequence_length(pkv_block_manager* m, int64_t seq_id);  /* -1 if unknown */
+
+/* Prefix caching by block content (glossary, section "Sharing blocks across
+ * sequences": hashing whole blocks extends sharing across requests; "Paged
+ * Attention" study notes, section on prefix caching: look up by hash, then
+ * confirm the prefix matches).  pkv_bm_cache_sequence registers the full blocks
+ * covering tokens[0 .. num_tokens) of an existing sequence (num_tokens <= its
+ * length) under a hash chained over each block's token ids and its
+ * predecessor's hash.  pkv_bm_add_sequence_cached creates a sequence for a
+ * prompt of num_tokens token ids: its leading full blocks that hit the cache --
+ * same tokens, same predecessor, confirmed exactly, at most (num_tokens - 1) /
+ * block_size blocks so that at least one token is left to compute -- are shared
+ * (reference counts), and *num_cached_tokens receives their token count (the
+ * sequence's length); the caller appends and prefills the rest.  Registered
+ * blocks that no sequence holds stay cached until the free list runs dry, then
+ * the one released longest ago is reused (pkv_bm_num_free counts them as free).
+ * pkv_bm_num_cached: registered blocks. */
+pkv_status pkv_bm_add_sequence_cached(pkv_block_manager* m, int64_t seq_id, const int32_t* tokens, int num_tokens,
+                                      int* num_cached_tokens);
+pkv_status pkv_bm_cache_sequence(pkv_block_manager* m, int64_t seq_id, const int32_t* tokens, int num_tokens);
+int pkv_bm_num_cached(pkv_block_manager* m);
+
+/* Move sequences between two managers with the same block size (e.g. a GPU
+ * pool's and a host pool's, for preemption by swapping): every distinct block
+ * the n sequences use in `from` gets one block in `to`; the sequences leave
+ * `from` (their references drop there) and appear in `to` with the same
+ * lengths and correspondingly shared blocks.  The (from block, to block) pairs,
+ * int64 [max_pairs][2], feed pkv_swap_blocks; *num_pairs receives their count.
+ * PKV_ERR_OUT_OF_BLOCKS if `to` is short of blocks (nothing changes). */
+pkv_status pkv_bm_swap(pkv_block_manager* from, pkv_block_manager* to, const int64_t* seq_ids, int n,
+                       int64_t* pairs, int max_pairs, int* num_pairs);
 
 /*
  * Diagnostic for the failure handling above (no counterpart on the pages): runs one

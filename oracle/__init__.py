@@ -2,8 +2,9 @@
 
 Python access to the float64 CPU oracle in ``pagedkv_oracle.c``: the plain
 definition of paged decode attention (gather through the block table, then
-textbook two-pass softmax) and of chunked prefill over the same cache, the scatter of new tokens into the pool, the
-block copy used for copy-on-write, and the number-format codecs.
+textbook two-pass softmax) and of chunked prefill over the same cache, the
+scatter of new tokens into the pool, the block copy used for copy-on-write,
+the block swap between two pools, and the number-format codecs.
 
 Only the test suite, ``__graft_entry__.smoke()`` and the benchmark's CPU
 baseline leg may import this package.  It shares no code with the CUDA
@@ -64,6 +65,8 @@ def _load():
         lib.orc_reshape_and_cache.restype = I
         lib.orc_copy_blocks.argtypes = [P, P, Z, P, I, I]
         lib.orc_copy_blocks.restype = I
+        lib.orc_swap_blocks.argtypes = [P, P, I, P, P, I, Z, P, I]
+        lib.orc_swap_blocks.restype = I
         lib.orc_gather.argtypes = [P, P, I, P, I, I, I, I, I, I, I]
         lib.orc_gather.restype = I
         lib.orc_decode_array.argtypes = [P, P, I, Z]
@@ -179,6 +182,15 @@ def copy_blocks(k_pool, v_pool, pairs) -> None:
     block_bytes = k_pool[0].nbytes
     _check(_load().orc_copy_blocks(_ptr(k_pool), _ptr(v_pool), block_bytes, _ptr(pairs),
                                    pairs.shape[0], NB))
+
+
+def swap_blocks(src_k, src_v, dst_k, dst_v, pairs) -> None:
+    """dst[d] := src[s] (K and V, whole blocks) for each row (s, d) of pairs, in place in dst."""
+    pairs = np.ascontiguousarray(pairs, dtype=np.int64).reshape(-1, 2)
+    assert src_k.shape[1:] == dst_k.shape[1:] and src_k.dtype == dst_k.dtype
+    _check(_load().orc_swap_blocks(_ptr(np.ascontiguousarray(src_k)), _ptr(np.ascontiguousarray(src_v)),
+                                   src_k.shape[0], _ptr(dst_k), _ptr(dst_v), dst_k.shape[0], src_k[0].nbytes,
+                                   _ptr(pairs), pairs.shape[0]))
 
 
 def gather(pool, kv_dtype, table, length, kvh=0) -> np.ndarray:

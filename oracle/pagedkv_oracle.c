@@ -425,6 +425,29 @@ int orc_copy_blocks(void* k_pool, void* v_pool, size_t block_bytes,
     return ORC_OK;
 }
 
+/*
+ * Swap between two pools ([PT], on preemption: a group's KV data moves to CPU
+ * memory and is brought back later): for each pair (s, d),
+ *   dst_k[d] := src_k[s] and dst_v[d] := src_v[s], whole blocks, bit for bit.
+ */
+int orc_swap_blocks(const void* src_k, const void* src_v, int src_blocks, void* dst_k, void* dst_v,
+                    int dst_blocks, size_t block_bytes, const int64_t* pairs, int num_pairs)
+{
+    if (num_pairs < 0 || src_blocks <= 0 || dst_blocks <= 0 || block_bytes == 0)
+        return ORC_BAD_ARG;
+    for (int i = 0; i < num_pairs; ++i) {
+        int64_t s = pairs[2 * i], d = pairs[2 * i + 1];
+        if (s < 0 || s >= src_blocks || d < 0 || d >= dst_blocks)
+            return ORC_BAD_BLOCK;
+    }
+    for (int i = 0; i < num_pairs; ++i) {
+        int64_t s = pairs[2 * i], d = pairs[2 * i + 1];
+        memcpy((char*)dst_k + (size_t)d * block_bytes, (const char*)src_k + (size_t)s * block_bytes, block_bytes);
+        memcpy((char*)dst_v + (size_t)d * block_bytes, (const char*)src_v + (size_t)s * block_bytes, block_bytes);
+    }
+    return ORC_OK;
+}
+
 /* ---------------------------------------------------------------------- */
 /* Gather through the table ([UL]: pool[block_table].reshape(-1, d)[:len]) */
 /* ---------------------------------------------------------------------- */

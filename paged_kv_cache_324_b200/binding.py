@@ -57,6 +57,8 @@ def lib() -> ctypes.CDLL:
         L.pkv_reshape_and_cache.restype = I
         L.pkv_copy_blocks.argtypes = [P, P, Z, P, I, I, P, P]
         L.pkv_copy_blocks.restype = I
+        L.pkv_swap_blocks.argtypes = [P, P, I, P, P, I, Z, P, I, P, P]
+        L.pkv_swap_blocks.restype = I
         L.pkv_selftest_bounded_wait.argtypes = [P, ctypes.c_uint, P]
         L.pkv_selftest_bounded_wait.restype = I
         _lib = L
@@ -210,6 +212,28 @@ def copy_blocks(k_pool: torch.Tensor, v_pool: torch.Tensor, pairs: torch.Tensor,
     _check(status, "copy_blocks")
 
 
+def swap_blocks(src_k: torch.Tensor, src_v: torch.Tensor, dst_k: torch.Tensor, dst_v: torch.Tensor,
+                pairs: torch.Tensor, *, device_error: Optional[torch.Tensor] = None, stream=None) -> None:
+    """dst[d] := src[s] (K and V pools [NB, Hkv, B, D], whole blocks) for each row (s, d) of pairs
+    (int64 [n, 2], on the GPU).  Either side may be pinned host memory (``pin_memory()``)."""
+    if pairs.dtype != torch.int64 or (pairs.numel() and pairs.shape[-1] != 2):
+        raise TypeError("pairs must be int64 [n, 2]")
+    if src_k.shape[1:] != dst_k.shape[1:] or src_k.dtype != dst_k.dtype or src_v.shape != src_k.shape \
+            or dst_v.shape != dst_k.shape:
+        raise ValueError("pools of one layout and dtype")
+    for t, name in ((src_k, "src_k"), (src_v, "src_v"), (dst_k, "dst_k"), (dst_v, "dst_v")):
+        if not t.is_cuda and not t.is_pinned():
+            raise ValueError(f"{name} must be on the GPU or in pinned host memory")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    block_bytes = src_k[0].numel() * src_k.element_size()
+    status = lib().pkv_swap_blocks(
+        ctypes.c_void_p(src_k.data_ptr()), ctypes.c_void_p(src_v.data_ptr()), src_k.shape[0],
+        ctypes.c_void_p(dst_k.data_ptr()), ctypes.c_void_p(dst_v.data_ptr()), dst_k.shape[0], block_bytes,
+        _dev(pairs, "pairs"), pairs.numel() // 2, _dev(device_error, "device_error"), _stream(stream))
+    _check(status, "swap_blocks")
+
+
 def selftest_bounded_wait(device_error: torch.Tensor, timeout_us: int, stream=None) -> None:
     """Run one bounded wait that nothing completes; it sets DEVERR_TIMEOUT in device_error."""
     _check(lib().pkv_selftest_bounded_wait(_dev(device_error, "device_error"), int(timeout_us), _stream(stream)),
@@ -235,6 +259,10 @@ class BlockManager:
         L.pkv_bm_ref_count.argtypes = [P, I32]
         L.pkv_bm_sequence_length.argtypes = [P, I64]
         L.pkv_bm_sequence_length.restype = I64
+        L.pkv_bm_num_cached.argtypes = [P]
+        L.pkv_bm_add_sequence_cached.argtypes = [P, I64, P, I, P]
+        L.pkv_bm_cache_sequence.argtypes = [P, I64, P, I]
+        L.pkv_bm_swap.argtypes = [P, P, P, I, P, I, P]
         self._L, self._np = L, np
         order = None
         if free_order is not None:
@@ -296,6 +324,40 @@ class BlockManager:
 
     def sequence_length(self, seq_id: int) -> int:
         return self._L.pkv_bm_sequence_length(self._h, seq_id)
+
+    # prefix caching by block content
+    @property
+    def num_cached(self) -> int:
+        return self._L.pkv_bm_num_cached(self._h)
+
+    def add_sequence_cached(self, seq_id: int, tokens) -> int:
+        """A new sequence for a prompt of token ids; returns how many of its leading tokens
+        are already cached (whole blocks, shared), which is the sequence's length."""
+        np = self._np
+        t = np.ascontiguousarray(tokens, dtype=np.int32)
+        n = ctypes.c_int(0)
+        self._ok(self._L.pkv_bm_add_sequence_cached(self._h, seq_id, t.ctypes.data_as(ctypes.c_void_p), t.size,
+                                                    ctypes.byref(n)), "add_sequence_cached")
+        return n.value
+
+    def cache_sequence(self, seq_id: int, tokens):
+        """Register the full blocks holding tokens[0 .. len(tokens)) of the sequence."""
+        np = self._np
+        t = np.ascontiguousarray(tokens, dtype=np.int32)
+        self._ok(self._L.pkv_bm_cache_sequence(self._h, seq_id, t.ctypes.data_as(ctypes.c_void_p), t.size),
+                 "cache_sequence")
+
+    def swap_to(self, other: "BlockManager", seq_ids):
+        """Move the sequences to ``other``; returns the (block here, block there) pairs, int64 [k, 2]."""
+        np = self._np
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        cap = max(1, sum(-(-max(self.sequence_length(int(i)), 0) // self.block_size) for i in ids))
+        pairs = np.empty((cap, 2), np.int64)
+        k = ctypes.c_int(0)
+        P = ctypes.c_void_p
+        self._ok(self._L.pkv_bm_swap(self._h, other._h, ids.ctypes.data_as(P), ids.size, pairs.ctypes.data_as(P),
+                                     cap, ctypes.byref(k)), "swap")
+        return pairs[:k.value].copy()
 
 
 def find_shared_prefixes(block_tables, context_lens, block_size: int, unit_width: int):

@@ -164,3 +164,124 @@ def test_bad_arguments(BM):
         m.append_slots([1, 1])                          # one token per sequence per call
     with pytest.raises(PagedKVError):
         m.free_sequence(5)
+
+
+# --------------------------------------------------------------------------
+# prefix caching by block content, and swapping between two managers
+# --------------------------------------------------------------------------
+
+def _fill(m, seq, n):
+    """Append n tokens to seq one at a time; returns the slots."""
+    return [int(m.append_slots([seq])[0][0]) for _ in range(n)]
+
+
+def test_prefix_cache_shares_whole_matching_blocks(BM):
+    m = BM(64, 4, np.random.default_rng(1).permutation(64))
+    a = np.arange(100, 122)                                  # 22 tokens: 5 full blocks + 2
+    m.add_sequence(0)
+    _fill(m, 0, len(a))
+    m.cache_sequence(0, a)
+    assert m.num_cached == 5
+    b = np.concatenate([a[:13], [999], a[14:]])               # differs inside block 3
+    got = m.add_sequence_cached(1, b)
+    assert got == 12                                          # blocks 0-2 match, block 3 does not
+    ta, _ = m.block_tables([0], 8)
+    tb, lb = m.block_tables([1], 8)
+    assert tb[0, :3].tolist() == ta[0, :3].tolist() and tb[0, 3] == -1 and lb[0] == 12
+    assert all(m.ref_count(int(x)) == 2 for x in ta[0, :3]) and m.ref_count(int(ta[0, 3])) == 1
+    # the rest of the prompt is appended into fresh blocks
+    _fill(m, 1, len(b) - got)
+    tb, lb = m.block_tables([1], 8)
+    assert lb[0] == len(b) and tb[0, 3] not in ta[0].tolist()
+
+
+def test_prefix_cache_leaves_one_token_to_compute(BM):
+    m = BM(32, 4)
+    a = np.arange(12)                                         # exactly 3 blocks
+    m.add_sequence(0)
+    _fill(m, 0, 12)
+    m.cache_sequence(0, a)
+    assert m.add_sequence_cached(1, a) == 8                   # not all 12: the last token is computed
+    assert m.add_sequence_cached(2, a[:1]) == 0
+    assert m.add_sequence_cached(3, np.arange(13)) == 12
+
+
+def test_idle_cached_blocks_are_reused_then_evicted_oldest_first(BM):
+    m = BM(6, 2, np.arange(6))
+    m.add_sequence(0)
+    _fill(m, 0, 4)                                            # blocks 0, 1
+    m.cache_sequence(0, [5, 6, 7, 8])
+    m.add_sequence(1)
+    _fill(m, 1, 4)                                            # blocks 2, 3
+    m.cache_sequence(1, [1, 2, 3, 4])
+    m.free_sequence(0)                                        # blocks 0, 1 idle first
+    m.free_sequence(1)                                        # then 2, 3
+    assert m.num_free == 6 and m.num_cached == 4
+    assert m.add_sequence_cached(2, [5, 6, 7, 8, 9]) == 4     # hit on idle blocks
+    t, _ = m.block_tables([2], 4)
+    assert t[0, :2].tolist() == [0, 1] and m.ref_count(0) == 1
+    m.add_sequence(3)
+    _fill(m, 3, 6)                                            # free 4, 5, then evicts idle 2 (oldest idle)
+    t, _ = m.block_tables([3], 4)
+    assert t[0, :3].tolist() == [4, 5, 2]
+    assert m.num_cached == 3                                  # block 2's entry is gone
+    assert m.add_sequence_cached(4, [1, 2, 3, 4, 0]) == 0     # its first block was evicted: no hit
+
+
+def test_stale_child_of_a_recycled_block_does_not_match(BM):
+    m = BM(4, 2, np.arange(4))
+    m.add_sequence(0)
+    _fill(m, 0, 4)                                            # blocks 0 (tokens 1,2), 1 (tokens 3,4)
+    m.cache_sequence(0, [1, 2, 3, 4])
+    m.free_sequence(0)
+    m.add_sequence(1)
+    _fill(m, 1, 6)                                            # 2, 3, then evicts 0 and reuses it
+    m.cache_sequence(1, [1, 2, 9, 9, 7, 7])                   # block 2 now holds tokens 1,2 again
+    # block 1 (tokens 3,4) still names block 0 of the old generation as its predecessor
+    m.free_sequence(1)
+    got = m.add_sequence_cached(2, [1, 2, 3, 4, 5])
+    t, _ = m.block_tables([2], 4)
+    assert got == 2 and t[0, 0] == 2                          # only the first block matches
+
+
+def test_swap_moves_a_group_and_its_shared_blocks(BM):
+    gpu = BM(40, 4, np.random.default_rng(2).permutation(40))
+    host = BM(20, 4, np.arange(20))
+    gpu.add_sequence(0)
+    _fill(gpu, 0, 9)                                          # 3 blocks, the last partial
+    gpu.fork(0, 1)
+    gpu.fork(0, 2)
+    _fill(gpu, 1, 1)                                          # copy-on-write of the partial block
+    gpu.add_sequence(3)
+    _fill(gpu, 3, 5)
+    before, lens0 = gpu.block_tables([0, 1, 2, 3], 4)
+    free0 = gpu.num_free
+    pairs = gpu.swap_to(host, [1, 2])                         # the group of samples 1 and 2
+    distinct = set(before[1, :3].tolist()) | set(before[2, :3].tolist())
+    assert len(pairs) == len(distinct) == 4                   # 2 shared full + 1 shared partial + 1 copy
+    assert set(pairs[:, 0].tolist()) == distinct
+    assert gpu.sequence_length(1) == -1 and host.sequence_length(1) == 10 and host.sequence_length(2) == 9
+    ht, _ = host.block_tables([1, 2], 4)
+    m = dict(pairs.tolist())
+    assert ht[0, :3].tolist() == [m[b] for b in before[1, :3]]
+    assert ht[1, :3].tolist() == [m[b] for b in before[2, :3]]
+    assert host.ref_count(m[int(before[1, 0])]) == 2          # shared by both swapped samples
+    assert gpu.num_free == free0 + 1                          # only the private copy left the GPU pool
+    # and back, into whatever blocks the GPU manager has free now
+    back = host.swap_to(gpu, [1, 2])
+    assert len(back) == 4 and host.num_free == 20
+    t2, lens2 = gpu.block_tables([1, 2], 4)
+    assert lens2.tolist() == lens0[1:3].tolist()
+
+
+def test_swap_is_all_or_nothing(BM):
+    from paged_kv_cache_324_b200.binding import PagedKVError
+    gpu = BM(10, 4)
+    host = BM(1, 4)
+    gpu.add_sequence(0)
+    _fill(gpu, 0, 8)                                          # 2 blocks, host has 1
+    with pytest.raises(PagedKVError) as e:
+        gpu.swap_to(host, [0])
+    assert e.value.status == 6 and gpu.sequence_length(0) == 8 and host.num_free == 1
+    with pytest.raises(PagedKVError):
+        gpu.swap_to(host, [5])                                # unknown sequence

@@ -481,3 +481,28 @@ def test_tolerance_rejects_planted_mistakes(name):
     for what, (tab, ln) in mistakes.items():
         bad = oracle.paged_attn_decode(w.q, w.q_dtype, kp, vp, w.kv_dtype, tab, ln, w.scale, **args)
         assert not attention_close(bad, ref, w.kv_dtype, w.q_dtype)[0], what
+
+
+def test_swap_blocks_round_trip_and_untouched_blocks():
+    """Swap-out then swap-in through another pool restores the blocks bit for bit; blocks
+    that no pair names are unchanged on both sides; a pair outside either pool is rejected."""
+    rng = np.random.default_rng(70)
+    gk = wl.garbage_bytes(rng, 12 * 2 * 16 * 8 * 2).view(np.uint16).reshape(12, 2, 16, 8)
+    gv = wl.garbage_bytes(rng, gk.nbytes).view(np.uint16).reshape(gk.shape)
+    hk = wl.garbage_bytes(rng, 5 * gk[0].nbytes).view(np.uint16).reshape(5, 2, 16, 8)
+    hv = wl.garbage_bytes(rng, hk.nbytes).view(np.uint16).reshape(hk.shape)
+    gk0, gv0, hk0, hv0 = gk.copy(), gv.copy(), hk.copy(), hv.copy()
+    out = np.array([[3, 0], [7, 4], [11, 1]])
+    oracle.swap_blocks(gk, gv, hk, hv, out)
+    for s, d in out:
+        assert np.array_equal(hk[d], gk0[s]) and np.array_equal(hv[d], gv0[s])
+    for d in (2, 3):
+        assert np.array_equal(hk[d], hk0[d]) and np.array_equal(hv[d], hv0[d])
+    assert np.array_equal(gk, gk0) and np.array_equal(gv, gv0)            # the source is only read
+    gk[[3, 7, 11]] = 0                                                     # the GPU blocks are reused meanwhile
+    back = np.array([[0, 9], [4, 2], [1, 5]])                              # swap in to other blocks
+    oracle.swap_blocks(hk, hv, gk, gv, back)
+    for (s_out, _), (_, d_in) in zip(out, back):
+        assert np.array_equal(gk[d_in], gk0[s_out]) and np.array_equal(gv[d_in], gv0[s_out])
+    with pytest.raises(oracle.OracleError):
+        oracle.swap_blocks(gk, gv, hk, hv, np.array([[0, 5]]))             # destination beyond the host pool
