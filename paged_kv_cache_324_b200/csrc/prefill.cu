@@ -7,27 +7,35 @@
 // prefill maps onto large matrix products), so both products run as
 // tcgen05.mma with the accumulators in tensor memory.
 //
-// One CTA = 128 query rows (128 / G tokens x the G query heads of one KV
-// head) of one sequence, against 128-key tiles of that KV head read through
-// the block table.  Warp roles:
-//   warps 0,10 TMA: warp 0 the Q tile once, then K tiles, warp 10 V tiles,
-//              block by block (one 4-D box per 16- or 32-token block and
-//              64-column chunk) into 128-byte-swizzled rings of two stages,
-//              each warp reading its table entries one tile ahead;
-//   warp 1     allocates 512 TMEM columns; one thread issues the MMAs:
-//              S_j = Q K_j^T into one of two TMEM buffers (M=128, N=128),
-//              and O += P_j V_j (M=128, N=head_dim) once P_j is written;
-//   warps 2-9  softmax, two warps per TMEM lane quarter: each thread takes
-//              64 of one row's 128 keys (TMEM lane = row); the two halves of a
-//              row exchange their maxima through shared memory.  Read S_j
-//              with tcgen05.ld, mask, online softmax in base 2 with a running
-//              maximum that is only moved when the new one exceeds it by more
-//              than 2^8 (the result does not depend on the reference maximum;
-//              this only bounds the weights), write P_j as 16-bit values into
-//              a swizzled shared-memory tile (the A operand of the next MMA),
-//              and rescale O in TMEM when the maximum moves; finally O / l.
-// S_{j+1} is issued before P_j is consumed, so the tensor core works on the
-// next tile while the softmax warps work on this one.
+// One CTA = two tiles of 128 query rows (tile A, then tile B: 128 / G tokens
+// each, x the G query heads of one KV head) of one sequence, against 128-key
+// tiles of that KV head read through the block table.  Both query tiles use
+// every K/V tile the CTA loads, which halves the K/V bytes per FLOP of a
+// one-tile CTA.  Warp roles:
+//   warps 0,10 TMA: warp 0 both Q tiles once, then K tiles into a 3-stage
+//              ring, warp 10 V tiles into a 2-stage ring, block by block (one
+//              4-D box per 16- or 32-token block and 64-column chunk,
+//              128-byte swizzle), each reading its table entries one tile
+//              ahead;
+//   warp 1     allocates all 512 TMEM columns (S_A, S_B, O_A, O_B); one thread
+//              issues the MMAs in the order
+//                PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), PV_A(j+1), ...
+//              S = Q K^T (M=128, N=128, both operands K-major in shared
+//              memory) and O += P V (M=128, N=head_dim; P read from tensor
+//              memory, V an MN-major shared-memory operand).  The MMAs of a CTA
+//              execute in issue order, which is what lets P overwrite the S it
+//              came from and S_X(j+1) overwrite P_X(j) once PV_X(j) has read it;
+//   warps 2-5  softmax of tile A, warps 6-9 of tile B: one query row per
+//              thread (TMEM lane = row).  Read S (two 64-column halves, the
+//              first read twice to keep the registers down), mask, online
+//              softmax in base 2 with a running maximum that is only moved when
+//              the new one exceeds it by more than 2^8 (the result does not
+//              depend on the reference maximum; the lag only bounds the
+//              weights), write P as packed 16-bit pairs into the upper half of
+//              the same S columns with tcgen05.st, and rescale O in TMEM when
+//              the maximum moves; finally O / l.
+// While tile A's softmax works on S_A(j+1), the tensor core computes PV_B(j)
+// and S_B(j+1), and the other way round.
 //
 // Keys beyond the last one any row of the CTA needs are never loaded; their V
 // rows are zeroed in shared memory (their weights are exactly 0, but 0 times
@@ -48,27 +56,28 @@
 namespace pkv {
 namespace {
 
-constexpr int kRows = 128;            // query rows per CTA: MMA M, one TMEM lane each
-constexpr int kKeys = 128;            // keys per tile: N of S = Q K^T, K of O += P V
-constexpr int kKStages = 2;           // the producers' ring arithmetic assumes two stages each
+constexpr int kRows = 128;            // query rows per tile: MMA M, one TMEM lane each
+constexpr int kTiles = 2;             // query tiles per CTA
+constexpr int kKeys = 128;            // keys per K/V tile: N of S = Q K^T, K of O += P V
+constexpr int kKStages = 2;
 constexpr int kVStages = 2;
-constexpr int kPThreads = 352;        // warp 0 TMA (Q, K), warp 1 MMA, warps 2-9 softmax, warp 10 TMA (V)
-constexpr int kVWarp = 10;
-constexpr int kSoftmaxWarps = 8;      // two per TMEM lane quarter: each takes 64 of a row's 128 keys
-constexpr uint32_t kTmemCols = 512;   // S buffers at columns 0 and 128, O at 256
-constexpr uint32_t kTmemO = 256;
+constexpr int kHalves = 2;            // softmax warps per TMEM lane quarter and tile: each takes 64 of 128 keys
+constexpr int kTileWarps = 4 * kHalves;
+constexpr int kVWarp = 2 + kTiles * kTileWarps;
+constexpr int kPThreads = 32 * (kVWarp + 1);   // warp 0 TMA (Q, K), warp 1 MMA, softmax, last warp TMA (V)
+constexpr uint32_t kTmemCols = 512;   // S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512)
+constexpr uint32_t kTmemS = 0, kTmemO = 256, kTmemP = 64;   // P_X: the upper half of S_X, packed pairs
 constexpr float kMaxLag = 8.0f;       // log2 of the largest weight the lagging maximum allows
 constexpr uint32_t kChunkBytes = kRows * 128;   // 128 rows x 128 bytes: one 64-column chunk
 
 template <int D>
 struct PGeo {
     static constexpr int kChunks = D / 64;
-    static constexpr uint32_t kTile = kChunks * kChunkBytes;   // Q, or one K or V stage
+    static constexpr uint32_t kTile = kChunks * kChunkBytes;   // one Q tile, or one K or V stage
     static constexpr uint32_t kQ = 0;
-    static constexpr uint32_t kK = kQ + kTile;
+    static constexpr uint32_t kK = kQ + kTiles * kTile;
     static constexpr uint32_t kV = kK + kKStages * kTile;
-    static constexpr uint32_t kP = kV + kVStages * kTile;
-    static constexpr uint32_t kEnd = kP + 2 * kChunkBytes;      // P: 128 rows x 128 keys x 2 bytes
+    static constexpr uint32_t kEnd = kV + kVStages * kTile;
     // +1 KB to align the base; at least 120 KB so that one CTA holds an SM (TMEM is not shared)
     static constexpr uint32_t kSmemBytes = (kEnd + 1024 > 120u * 1024u) ? kEnd + 1024 : 120u * 1024u;
 };
@@ -123,6 +132,17 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b,
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a), "l"(b), "r"(idesc), "r"(accumulate ? 1u : 0u)
+        : "memory");
+}
+
+// The same with A read from tensor memory (lane = row, two 16-bit K elements per column).
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                           bool accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate ? 1u : 0u)
         : "memory");
 }
 
@@ -201,6 +221,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,
@@ -272,13 +301,12 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
     constexpr int kTB = kKeys / BS;                  // blocks per key tile
     constexpr uint32_t kBoxBytes = BS * 128;         // one block x one 64-column chunk
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t bars[2 * kKStages + 2 * kVStages + 8 + 4];
+    __shared__ __align__(8) uint64_t bars[2 * kKStages + 2 * kVStages + 8 + kTiles * 4];
     __shared__ CtaFlags flags;
-    __shared__ float red[2][2][kRows];   // [tile parity][half][row]: partial row maxima
-    __shared__ float red_l[2][kRows];    // [half][row]: partial row sums at the end
+    __shared__ float red[2][kTiles][kHalves][kRows];   // [tile parity][query tile][half][row]: partial maxima
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int G = a.group, TQ = kRows / G;
+    const int G = a.group, TQ = kRows / G;           // tokens per query tile
     const int kvh = blockIdx.y, s = blockIdx.z;
 
     pdl_wait();   // q, the pool and the tables may come from the previous kernel on the stream
@@ -289,40 +317,47 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
         return;
     }
     const int C = q1 - q0;
-    const int ntq = (C + TQ - 1) / TQ;
-    if (blockIdx.x == 0 && threadIdx.x == 0 && ntq > static_cast<int>(gridDim.x))
+    const int ncta = (C + kTiles * TQ - 1) / (kTiles * TQ);
+    if (blockIdx.x == 0 && threadIdx.x == 0 && ncta > static_cast<int>(gridDim.x))
         raise_error(a.err, PKV_DEVERR_CONTEXT_LEN);      // longer than max_query_len: rows left unwritten
-    if (static_cast<int>(blockIdx.x) >= ntq) return;
+    if (static_cast<int>(blockIdx.x) >= ncta) return;
     if (grid_timed_out(a.err)) return;   // a wait elsewhere gave up: finish at once
-    const int t0 = (ntq - 1 - static_cast<int>(blockIdx.x)) * TQ;   // longest tiles first
-    const int rows_valid = min(TQ, C - t0);
-    const int pq_max = min(L - C + t0 + TQ - 1, L - 1);   // last key any row of this CTA attends
+    const int t0 = (ncta - 1 - static_cast<int>(blockIdx.x)) * kTiles * TQ;   // longest tiles first
+    const int rows_cta = min(kTiles * TQ, C - t0);                              // tokens of this CTA
 
     if (C > L || L > a.max_blocks_per_seq * BS) {         // positions undefined: NaN rows
         if (threadIdx.x == 0) raise_error(a.err, PKV_DEVERR_CONTEXT_LEN);
-        for (int i = threadIdx.x; i < rows_valid * G * D; i += kPThreads) {
+        for (int i = threadIdx.x; i < rows_cta * G * D; i += kPThreads) {
             const int t = i / (G * D), rem = i % (G * D);
             const size_t o = (static_cast<size_t>(q0 + t0 + t) * a.num_heads + kvh * G) * D + rem;
             reinterpret_cast<uint16_t*>(a.out)[o] = kBf16 ? 0x7FC0u : 0x7E00u;
         }
         return;
     }
-    const int ntk = pq_max / kKeys + 1;                    // key tiles this CTA needs
+    const bool has_b = rows_cta > TQ;
+    // last key each tile's rows attend; key tiles each tile needs; the CTA loads the larger range
+    const int pq_max_a = min(L - C + t0 + TQ - 1, L - 1);
+    const int pq_max_b = min(L - C + t0 + 2 * TQ - 1, L - 1);
+    const int ntk_a = pq_max_a / kKeys + 1;
+    const int ntk_b = has_b ? pq_max_b / kKeys + 1 : 0;
+    const int ntk = max(ntk_a, ntk_b);
+    const int pq_max = has_b ? pq_max_b : pq_max_a;
     const int nblk = (pq_max + 1 + BS - 1) / BS;           // blocks holding keys 0..pq_max
 
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_addr(smem);
-    const uint32_t sQ = sbase + Gm::kQ, sK = sbase + Gm::kK, sV = sbase + Gm::kV, sP = sbase + Gm::kP;
+    const uint32_t sQ = sbase + Gm::kQ, sK = sbase + Gm::kK, sV = sbase + Gm::kV;
     const uint32_t b0 = smem_addr(bars);
     auto k_full = [&](int i) { return b0 + 8u * i; };
     auto k_empty = [&](int i) { return b0 + 8u * (kKStages + i); };
     auto v_full = [&](int i) { return b0 + 8u * (2 * kKStages + i); };
     auto v_empty = [&](int i) { return b0 + 8u * (2 * kKStages + kVStages + i); };
     const uint32_t bar_q = b0 + 8u * (2 * kKStages + 2 * kVStages);
-    auto s_full = [&](int i) { return bar_q + 8u * (1 + i); };
-    auto s_empty = [&](int i) { return bar_q + 8u * (3 + i); };
-    const uint32_t p_full = bar_q + 8u * 5, o_done = bar_q + 8u * 6, drain = bar_q + 8u * 7;
-    auto xchg = [&](int quarter) { return bar_q + 8u * (8 + quarter); };   // the two warps of a lane quarter
+    auto s_full = [&](int t) { return bar_q + 8u * (1 + t); };    // per query tile
+    auto p_full = [&](int t) { return bar_q + 8u * (3 + t); };
+    auto o_done = [&](int t) { return bar_q + 8u * (5 + t); };    // the tile's last P.V product completed
+    const uint32_t drain = bar_q + 8u * 7;
+    auto xchg = [&](int t, int quarter) { return bar_q + 8u * (8 + t * 4 + quarter); };   // the halves of a row
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kKStages; ++i) {
@@ -334,13 +369,12 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
             mbar_init(v_empty(i), 1);
         }
         mbar_init(bar_q, 1);
-        mbar_init(s_full(0), 1);
-        mbar_init(s_full(1), 1);
-        mbar_init(s_empty(0), kSoftmaxWarps);
-        mbar_init(s_empty(1), kSoftmaxWarps);
-        mbar_init(p_full, kSoftmaxWarps);
-        for (int i = 0; i < 4; ++i) mbar_init(xchg(i), 2);
-        mbar_init(o_done, 1);
+        for (int t = 0; t < kTiles; ++t) {
+            mbar_init(s_full(t), 1);
+            mbar_init(p_full(t), kTileWarps);
+            mbar_init(o_done(t), 1);
+            for (int q = 0; q < 4; ++q) mbar_init(xchg(t, q), kHalves);
+        }
         mbar_init(drain, 1);
         flags.abort = 0;
         flags.bad = 0;
@@ -361,14 +395,18 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
     if (warp == 0 || warp == kVWarp) {
         // ---------------- TMA producers: warp 0 loads Q and K, warp 10 loads V ----------------
         const bool is_k = warp == 0;
+        const int nst = is_k ? kKStages : kVStages;
         const uint64_t pol = l2_policy_evict_last();      // K/V tiles are read again by the other query tiles
         if (is_k && lane == 0) {
             tma_prefetch_desc(&qmap);
             tma_prefetch_desc(&kmap);
             tma_prefetch_desc(&vmap);
-            mbar_arrive_expect_tx(bar_q, Gm::kTile);
+            mbar_arrive_expect_tx(bar_q, kTiles * Gm::kTile);
 #pragma unroll
-            for (int c = 0; c < Gm::kChunks; ++c) tma_load_3d(sQ + c * kChunkBytes, &qmap, bar_q, c * 64, kvh * G, q0 + t0);
+            for (int t = 0; t < kTiles; ++t)
+#pragma unroll
+                for (int c = 0; c < Gm::kChunks; ++c)
+                    tma_load_3d(sQ + t * Gm::kTile + c * kChunkBytes, &qmap, bar_q, c * 64, kvh * G, q0 + t0 + t * TQ);
         }
         const CUtensorMap* map = is_k ? &kmap : &vmap;
         const uint32_t ring = is_k ? sK : sV;
@@ -388,9 +426,9 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
                 flags.bad = 1;
             }
             const uint32_t bytes = __popc(ok_mask) * kBoxBytes * Gm::kChunks;
-            const int st = j % 2;                          // both rings have two stages
+            const int st = j % nst;
             const uint32_t full = is_k ? k_full(st) : v_full(st), empty = is_k ? k_empty(st) : v_empty(st);
-            if (j >= 2 && !warp_wait_bar(empty, ((j / 2) - 1) & 1, &flags, a.err)) break;
+            if (j >= nst && !warp_wait_bar(empty, ((j / nst) - 1) & 1, &flags, a.err)) break;
             if (lane == 0) mbar_arrive_expect_tx(full, bytes);
             issued = j + 1;
             for (int b = 0; b < kTB; ++b) {
@@ -407,45 +445,60 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
         if (lane == 0) {
             const uint64_t end = global_timer_ns() + kWaitLimitNs;
             if (is_k) mbar_wait(bar_q, 0, end);
-            for (int j = max(0, issued - 2); j < issued; ++j)
-                mbar_wait(is_k ? k_full(j % 2) : v_full(j % 2), (j / 2) & 1, end);
+            for (int j = max(0, issued - nst); j < issued; ++j)
+                mbar_wait(is_k ? k_full(j % nst) : v_full(j % nst), (j / nst) & 1, end);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer (one thread) ----------------
         if (lane == 0) {
             constexpr uint32_t idesc_s = mma_idesc(kBf16, false, kRows, kKeys);
             constexpr uint32_t idesc_o = mma_idesc(kBf16, true, kRows, D);
-            bool ok = wait_bar(bar_q, 0, &flags, a.err);
-            auto issue_s = [&](int j) -> bool {
+            int k_waited = -1;                            // the last key tile whose arrival was awaited
+            auto issue_s = [&](int t, int j) -> bool {    // S_t(j) = Q_t K_j^T into S_t
                 const int ks = j % kKStages;
-                if (!wait_bar(k_full(ks), (j / kKStages) & 1, &flags, a.err)) return false;
-                if (j >= 2 && !wait_bar(s_empty(j & 1), ((j >> 1) - 1) & 1, &flags, a.err)) return false;
+                if (k_waited < j) {
+                    if (!wait_bar(k_full(ks), (j / kKStages) & 1, &flags, a.err)) return false;
+                    k_waited = j;
+                }
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
                     const uint32_t off = (k >> 2) * kChunkBytes + (k & 3) * 32;
-                    mma_f16(tmem + (j & 1) * kKeys, smem_desc(sQ + off, 16, 1024),
+                    mma_f16(tmem + kTmemS + t * kKeys, smem_desc(sQ + t * Gm::kTile + off, 16, 1024),
                             smem_desc(sK + ks * Gm::kTile + off, 16, 1024), idesc_s, k > 0);
                 }
-                mma_commit(s_full(j & 1));
-                mma_commit(k_empty(ks));
+                mma_commit(s_full(t));
                 return true;
             };
-            if (ok) ok = issue_s(0);
-            for (int j = 0; ok && j < ntk; ++j) {
-                if (j + 1 < ntk && !issue_s(j + 1)) break;
-                const int vs = j % kVStages;
-                if (!wait_bar(v_full(vs), (j / kVStages) & 1, &flags, a.err)) break;
-                if (!wait_bar(p_full, j & 1, &flags, a.err)) break;
+            auto issue_pv = [&](int t, int j) -> bool {   // O_t += P_t V_j, P_t from tensor memory
+                if (!wait_bar(p_full(t), j & 1, &flags, a.err)) return false;
                 tc_fence_after();
+                const int vs = j % kVStages;
 #pragma unroll
                 for (int kk = 0; kk < kKeys / 16; ++kk) {
-                    mma_f16(tmem + kTmemO, smem_desc(sP + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024),
-                            smem_desc(sV + vs * Gm::kTile + kk * 16 * 128, kChunkBytes, 1024), idesc_o,
-                            j > 0 || kk > 0);
+                    mma_f16_ts(tmem + kTmemO + t * 128, tmem + kTmemS + t * kKeys + kTmemP + kk * 8,
+                               smem_desc(sV + vs * Gm::kTile + kk * 16 * 128, kChunkBytes, 1024), idesc_o,
+                               j > 0 || kk > 0);
                 }
-                mma_commit(o_done);
-                mma_commit(v_empty(vs));
+                if (j == (t == 0 ? ntk_a : ntk_b) - 1) mma_commit(o_done(t));
+                return true;
+            };
+            bool ok = wait_bar(bar_q, 0, &flags, a.err);
+            if (ok) ok = issue_s(0, 0);
+            if (ok && ntk_b > 0) ok = issue_s(1, 0);
+            if (ok) mma_commit(k_empty(0));
+            for (int j = 0; ok && j < ntk; ++j) {
+                if (!wait_bar(v_full(j % kVStages), (j / kVStages) & 1, &flags, a.err)) break;
+#pragma unroll
+                for (int t = 0; t < kTiles; ++t) {
+                    const int nt = t == 0 ? ntk_a : ntk_b;
+                    if (!ok || j >= nt) continue;
+                    ok = issue_pv(t, j);                       // reads P_t(j) ...
+                    if (ok && j + 1 < nt) ok = issue_s(t, j + 1);   // ... before S_t(j+1) overwrites it
+                }
+                if (!ok) break;
+                mma_commit(v_empty(j % kVStages));
+                if (j + 1 < ntk) mma_commit(k_empty((j + 1) % kKStages));
             }
             // drain: every MMA issued so far completes before TMEM is freed
             mma_commit(drain);
@@ -453,49 +506,46 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
         }
         __syncwarp();
     } else {
-        // ---------------- softmax (warps 2-9: row = TMEM lane, half = which 64 keys) ----------------
+        // ---------------- softmax: row = TMEM lane, half = which 64 of the row's keys ----------------
+        const int t = (warp - 2) / kTileWarps;
+        const int half = ((warp - 2) % kTileWarps) >> 2;
         const int quarter = warp & 3;
-        const int half = (warp - 2) >> 2;                   // warps 2-5: keys 0-63, warps 6-9: keys 64-127
         const int row = quarter * 32 + lane;
-        const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-        const int tq = row / G;
+        const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);   // this warp's lanes
+        const uint32_t tS = tl + kTmemS + t * kKeys, tO = tl + kTmemO + t * 128;
+        constexpr int kOCols = D / kHalves;                // O columns this thread rescales and stores
+        const int tq = t * TQ + row / G;                  // token of this row within the CTA
         const int pq = min(L - C + t0 + tq, L - 1);
-        constexpr int kHalf = kKeys / 2;
-        constexpr int kOCols = D / 2;                        // O columns this thread rescales and stores
+        const int my_ntk = t == 0 ? ntk_a : ntk_b;
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
-        for (int j = 0; j < ntk; ++j) {
-            const int buf = j & 1;
-            if (!warp_wait_bar(s_full(buf), (j >> 1) & 1, &flags, a.err)) { ok = false; break; }
+        for (int j = 0; j < my_ntk; ++j) {
+            // S_t(j) complete means PV_t(j-1) has completed too (issue order): P and O are free
+            if (!warp_wait_bar(s_full(t), j & 1, &flags, a.err)) { ok = false; break; }
             tc_fence_after();
-            float x[kHalf];
+            const int kbase = j * kKeys + half * 64;
+            const bool mask = kbase + 63 > pq;
+            float x[64];
             {
-                uint32_t r[kHalf];
-                tmem_ld64_wait(trow + buf * kKeys + half * kHalf, r);
+                uint32_t r[64];
+                tmem_ld64_wait(tS + half * 64, r);
 #pragma unroll
-                for (int i = 0; i < kHalf; ++i) x[i] = __uint_as_float(r[i]);
+                for (int i = 0; i < 64; ++i) x[i] = (mask && kbase + i > pq) ? -INFINITY : __uint_as_float(r[i]);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(s_empty(buf));
-            const int kbase = j * kKeys + half * kHalf;
-            if (kbase + kHalf - 1 > pq) {
-#pragma unroll
-                for (int c = 0; c < kHalf; ++c) x[c] = (kbase + c > pq) ? -INFINITY : x[c];
-            }
-            float mp[8];                                      // eight independent chains, then a tree
+            float mp[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) mp[i] = x[i];
 #pragma unroll
-            for (int c = 8; c < kHalf; ++c) mp[c & 7] = fmaxf(mp[c & 7], x[c]);
+            for (int c = 8; c < 64; ++c) mp[c & 7] = fmaxf(mp[c & 7], x[c]);
             float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
                              fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
-            // the row's maximum over both halves: exchange through shared memory
-            red[buf][half][row] = mx;
+            // the row's maximum over both halves; after this exchange both halves have read their S,
+            // so P may be written over the S columns of keys 64-127
+            red[j & 1][t][half][row] = mx;
             __syncwarp();
-            if (lane == 0) mbar_arrive(xchg(quarter));
-            if (!warp_wait_bar(xchg(quarter), j & 1, &flags, a.err)) { ok = false; break; }
-            mx = fmaxf(mx, red[buf][half ^ 1][row]);
+            if (lane == 0) mbar_arrive(xchg(t, quarter));
+            if (!warp_wait_bar(xchg(t, quarter), j & 1, &flags, a.err)) { ok = false; break; }
+            mx = fmaxf(mx, red[j & 1][t][half ^ 1][row]);
             const float m_cand = mx * a.scale_log2;
             const bool move = m_cand > m_used + kMaxLag;
             float alpha = 1.f;
@@ -504,39 +554,34 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
                 m_used = m_cand;
             }
             const float neg_m = -m_used;
-            uint32_t pk[kHalf / 2];
             float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int c = 0; c < kHalf; c += 2) {
-                const float p0 = ex2(fmaf(x[c], a.scale_log2, neg_m));
-                const float p1 = ex2(fmaf(x[c + 1], a.scale_log2, neg_m));
-                sp[(c >> 1) & 7] += p0 + p1;
-                pk[c / 2] = pack2<kBf16>(p0, p1);
+            for (int h = 0; h < 2; ++h) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int c = 0; c < 32; c += 2) {
+                    const float p0 = ex2(fmaf(x[32 * h + c], a.scale_log2, neg_m));
+                    const float p1 = ex2(fmaf(x[32 * h + c + 1], a.scale_log2, neg_m));
+                    sp[(c >> 1) & 7] += p0 + p1;
+                    pk[c / 2] = pack2<kBf16>(p0, p1);
+                }
+                tmem_st16(tS + kTmemP + half * 32 + h * 16, pk);
             }
-            const float sum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
-            l = l * alpha + sum;                             // this half's share of the row sum
-            // P and O are free once the previous P.V product has completed
-            if (j > 0 && !warp_wait_bar(o_done, (j - 1) & 1, &flags, a.err)) { ok = false; break; }
+            l = l * alpha + (((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7])));
             if (j > 0 && __any_sync(0xffffffffu, move)) {
-                tc_fence_after();
 #pragma unroll
                 for (int c = 0; c < kOCols / 32; ++c) {
                     uint32_t r[32];
-                    tmem_ld32_wait(trow + kTmemO + half * kOCols + c * 32, r);
+                    tmem_ld32_wait(tO + half * kOCols + c * 32, r);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                    tmem_st32(trow + kTmemO + half * kOCols + c * 32, r);
+                    tmem_st32(tO + half * kOCols + c * 32, r);
                 }
-                tmem_wait_st();
             }
-            // this half's 64 keys are P's 64-key chunk `half`: one 128-byte row, units swizzled by row % 8
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const uint32_t addr = sP + half * kChunkBytes + row * 128 + ((u ^ (row & 7)) << 4);
-                sts128(addr, pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-            }
+            tmem_wait_st();
             if (j == ntk - 1 && j * kKeys + kKeys - 1 > pq_max) {
-                // keys past pq_max were not loaded (or are unwritten slots): zero their V rows
+                // keys past pq_max were not loaded (or are unwritten slots): zero their V rows (each half its
+                // 64-column chunk).  When both query tiles reach this tile they write the same zeros.
                 const int vs = j % kVStages;
                 if (!warp_wait_bar(v_full(vs), (j / kVStages) & 1, &flags, a.err)) { ok = false; break; }
                 if (half < Gm::kChunks && j * kKeys + row > pq_max) {
@@ -545,30 +590,31 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
                         sts128(sV + vs * Gm::kTile + half * kChunkBytes + row * 128 + ((u ^ (row & 7)) << 4), 0u, 0u,
                                0u, 0u);
                 }
+                fence_proxy_async_smem();
             }
-            fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full);
+            if (lane == 0) mbar_arrive(p_full(t));
         }
-        if (ok) ok = warp_wait_bar(o_done, (ntk - 1) & 1, &flags, a.err);
-        red_l[half][row] = l;                                // read back after the barrier below
+        if (ok && my_ntk > 0) ok = warp_wait_bar(o_done(t), 0, &flags, a.err);
         pdl_trigger();
+        // partial row sums: the parity buffer the last exchange did not use is free by now
+        red[my_ntk & 1][t][half][row] = l;
         // the output is written after the CTA-wide barrier below, which also publishes flags.bad
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
         // every lane takes part in the warp-wide TMEM loads; only rows of the chunk are stored
-        const bool live = tq < rows_valid;
+        const bool live = tq < rows_cta;
         const bool nan_out = !ok || flags.bad || *reinterpret_cast<volatile int*>(&flags.abort);
         uint16_t* orow = reinterpret_cast<uint16_t*>(a.out) +
                          (static_cast<size_t>(q0 + t0 + (live ? tq : 0)) * a.num_heads + kvh * G + row % G) * D +
                          half * kOCols;
-        const float inv = 1.f / (red_l[0][row] + red_l[1][row]);
+        const float inv = 1.f / (red[my_ntk & 1][t][0][row] + red[my_ntk & 1][t][1][row]);
 #pragma unroll
         for (int c = 0; c < kOCols / 32; ++c) {
             uint32_t r[32];
-            tmem_ld32_wait(trow + kTmemO + half * kOCols + c * 32, r);
+            tmem_ld32_wait(tO + half * kOCols + c * 32, r);
             if (live) {
                 uint32_t w[16];
 #pragma unroll
@@ -670,7 +716,7 @@ extern "C" pkv_status pkv_paged_attn_prefill(void* out, const void* q, pkv_dtype
         (reinterpret_cast<uintptr_t>(block_tables) & 3) || (reinterpret_cast<uintptr_t>(context_lens) & 3) ||
         (reinterpret_cast<uintptr_t>(query_start) & 3) || (reinterpret_cast<uintptr_t>(device_error) & 3))
         return PKV_ERR_ALIGNMENT;
-    const long long tiles = (static_cast<long long>(max_query_len) * G + kRows - 1) / kRows;
+    const long long tiles = (static_cast<long long>(max_query_len) * G + kTiles * kRows - 1) / (kTiles * kRows);
     if (num_seqs > 65535 || num_kv_heads > 65535 || tiles > 0x7fffffffLL) return PKV_ERR_INVALID_ARG;
 
     PrefillArgs a{};
