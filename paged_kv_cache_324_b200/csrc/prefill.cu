@@ -203,6 +203,31 @@ __device__ __forceinline__ void tmem_ld64_wait(uint32_t taddr, uint32_t (&r)[64]
         : "memory");
 }
 
+// Paired fp32 arithmetic (one instruction for two lanes of work) and a three-input maximum.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{.reg .b64 pa, pb, pc, pd;\n\t"
+        "mov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %5};\n\tmov.b64 pc, {%6, %7};\n\t"
+        "fma.rn.f32x2 pd, pa, pb, pc;\n\tmov.b64 {%0, %1}, pd;}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    float2 d;
+    asm("{.reg .b64 pa, pb, pd;\n\t"
+        "mov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %5};\n\t"
+        "add.rn.f32x2 pd, pa, pb;\n\tmov.b64 {%0, %1}, pd;}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // 2^x with the multi-function unit's approximation (subnormal results flush to zero).
 __device__ __forceinline__ float ex2(float x) {
     float y;
@@ -529,16 +554,20 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
             {
                 uint32_t r[64];
                 tmem_ld64_wait(tS + half * 64, r);
+                if (mask) {                                   // only tiles that cross this row's position
 #pragma unroll
-                for (int i = 0; i < 64; ++i) x[i] = (mask && kbase + i > pq) ? -INFINITY : __uint_as_float(r[i]);
+                    for (int i = 0; i < 64; ++i) x[i] = kbase + i > pq ? -INFINITY : __uint_as_float(r[i]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) x[i] = __uint_as_float(r[i]);
+                }
             }
-            float mp[8];
+            float mp[8];                                      // eight chains of three-input maxima, then a tree
 #pragma unroll
-            for (int i = 0; i < 8; ++i) mp[i] = x[i];
-#pragma unroll
-            for (int c = 8; c < 64; ++c) mp[c & 7] = fmaxf(mp[c & 7], x[c]);
-            float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+            for (int i = 0; i < 8; ++i)
+                mp[i] = fmaxf(max3f(max3f(x[i], x[i + 8], x[i + 16]), x[i + 24], x[i + 32]),
+                              max3f(x[i + 40], x[i + 48], x[i + 56]));
+            float mx = max3f(max3f(mp[0], mp[1], mp[2]), max3f(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
             // the row's maximum over both halves; after this exchange both halves have read their S,
             // so P may be written over the S columns of keys 64-127
             red[j & 1][t][half][row] = mx;
@@ -553,21 +582,23 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
                 alpha = ex2(m_used - m_cand);
                 m_used = m_cand;
             }
-            const float neg_m = -m_used;
-            float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nm2 = make_float2(-m_used, -m_used);
+            float2 sp[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                            make_float2(0.f, 0.f)};
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int c = 0; c < 32; c += 2) {
-                    const float p0 = ex2(fmaf(x[32 * h + c], a.scale_log2, neg_m));
-                    const float p1 = ex2(fmaf(x[32 * h + c + 1], a.scale_log2, neg_m));
-                    sp[(c >> 1) & 7] += p0 + p1;
-                    pk[c / 2] = pack2<kBf16>(p0, p1);
+                    const float2 e = fma2(make_float2(x[32 * h + c], x[32 * h + c + 1]), sc2, nm2);
+                    const float2 p = make_float2(ex2(e.x), ex2(e.y));
+                    sp[(c >> 1) & 3] = add2(sp[(c >> 1) & 3], p);
+                    pk[c / 2] = pack2<kBf16>(p.x, p.y);
                 }
                 tmem_st16(tS + kTmemP + half * 32 + h * 16, pk);
             }
-            l = l * alpha + (((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7])));
+            const float2 s01 = add2(add2(sp[0], sp[1]), add2(sp[2], sp[3]));
+            l = l * alpha + (s01.x + s01.y);
             if (j > 0 && __any_sync(0xffffffffu, move)) {
 #pragma unroll
                 for (int c = 0; c < kOCols / 32; ++c) {
