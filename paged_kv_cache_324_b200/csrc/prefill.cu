@@ -19,7 +19,8 @@
 //              ahead;
 //   warp 1     allocates all 512 TMEM columns (S_A, S_B, O_A, O_B); one thread
 //              issues the MMAs in the order
-//                PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), PV_A(j+1), ...
+//                S_A(0), PV_A(0), S_A(1), S_B(0), PV_B(0), S_B(1), PV_A(1), S_A(2), ...
+//              (tile B half a period behind tile A)
 //              S = Q K^T (M=128, N=128, both operands K-major in shared
 //              memory) and O += P V (M=128, N=head_dim; P read from tensor
 //              memory, V an MN-major shared-memory operand).  The MMAs of a CTA
@@ -508,22 +509,29 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
                 if (j == (t == 0 ? ntk_a : ntk_b) - 1) mma_commit(o_done(t));
                 return true;
             };
+            int v_waited = -1;
+            auto pv_then_s = [&](int t, int j) -> bool {   // PV_t(j), then S_t(j+1) over the P it read
+                if (v_waited < j) {
+                    if (!wait_bar(v_full(j % kVStages), (j / kVStages) & 1, &flags, a.err)) return false;
+                    v_waited = j;
+                }
+                if (!issue_pv(t, j)) return false;
+                return j + 1 < (t == 0 ? ntk_a : ntk_b) ? issue_s(t, j + 1) : true;
+            };
+            // Tile B runs half a period behind tile A, so that each tile's softmax overlaps the other
+            // tile's P.V and S products: S_A(0), PV_A(0) S_A(1), S_B(0), then for each j
+            // PV_B(j) S_B(j+1), PV_A(j+1) S_A(j+2).
             bool ok = wait_bar(bar_q, 0, &flags, a.err);
             if (ok) ok = issue_s(0, 0);
-            if (ok && ntk_b > 0) ok = issue_s(1, 0);
+            if (ok) ok = pv_then_s(0, 0);
+            if (ok && has_b) ok = issue_s(1, 0);
             if (ok) mma_commit(k_empty(0));
             for (int j = 0; ok && j < ntk; ++j) {
-                if (!wait_bar(v_full(j % kVStages), (j / kVStages) & 1, &flags, a.err)) break;
-#pragma unroll
-                for (int t = 0; t < kTiles; ++t) {
-                    const int nt = t == 0 ? ntk_a : ntk_b;
-                    if (!ok || j >= nt) continue;
-                    ok = issue_pv(t, j);                       // reads P_t(j) ...
-                    if (ok && j + 1 < nt) ok = issue_s(t, j + 1);   // ... before S_t(j+1) overwrites it
-                }
+                if (has_b && j < ntk_b) ok = pv_then_s(1, j);
                 if (!ok) break;
-                mma_commit(v_empty(j % kVStages));
-                if (j + 1 < ntk) mma_commit(k_empty((j + 1) % kKStages));
+                mma_commit(v_empty(j % kVStages));                   // V_j: PV_A(j) and PV_B(j) issued
+                if (j + 1 < ntk) mma_commit(k_empty((j + 1) % kKStages));   // K_{j+1}: both S issued
+                if (j + 1 < ntk_a) ok = pv_then_s(0, j + 1);
             }
             // drain: every MMA issued so far completes before TMEM is freed
             mma_commit(drain);
