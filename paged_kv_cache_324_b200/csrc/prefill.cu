@@ -247,13 +247,10 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-        "%14, %15, %16};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-        : "memory");
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
 }
 
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
@@ -591,21 +588,20 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
                 m_used = m_cand;
             }
             const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nm2 = make_float2(-m_used, -m_used);
-            float2 sp[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                            make_float2(0.f, 0.f)};
+            float2 sp[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t pk[16];
+            for (int h = 0; h < 4; ++h) {                    // 16 keys (8 packed words) at a time
+                uint32_t pk[8];
 #pragma unroll
-                for (int c = 0; c < 32; c += 2) {
-                    const float2 e = fma2(make_float2(x[32 * h + c], x[32 * h + c + 1]), sc2, nm2);
+                for (int c = 0; c < 16; c += 2) {
+                    const float2 e = fma2(make_float2(x[16 * h + c], x[16 * h + c + 1]), sc2, nm2);
                     const float2 p = make_float2(ex2(e.x), ex2(e.y));
-                    sp[(c >> 1) & 3] = add2(sp[(c >> 1) & 3], p);
+                    sp[(c >> 1) & 1] = add2(sp[(c >> 1) & 1], p);
                     pk[c / 2] = pack2<kBf16>(p.x, p.y);
                 }
-                tmem_st16(tS + kTmemP + half * 32 + h * 16, pk);
+                tmem_st8(tS + kTmemP + half * 32 + h * 8, pk);
             }
-            const float2 s01 = add2(add2(sp[0], sp[1]), add2(sp[2], sp[3]));
+            const float2 s01 = add2(sp[0], sp[1]);
             l = l * alpha + (s01.x + s01.y);
             if (j > 0 && __any_sync(0xffffffffu, move)) {
 #pragma unroll
