@@ -55,7 +55,7 @@ NCU_TRAFFIC = {
 
 
 # the same for the prefill kernel (sha256 prefix of prefill.cu), on the prefill workload
-PREFILL_TRAFFIC = {"bytes_per_launch": 569_860_352, "kernel_sha": "92b4d97290f49bc4",
+PREFILL_TRAFFIC = {"bytes_per_launch": 568_925_952, "kernel_sha": "d284513126c47679",
                    "capture": "profiles/paged_prefill_kernel_prefill.md"}
 
 
