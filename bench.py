@@ -55,7 +55,7 @@ NCU_TRAFFIC = {
 
 
 # the same for the prefill kernel (sha256 prefix of prefill.cu), on the prefill workload
-PREFILL_TRAFFIC = {"bytes_per_launch": 568_925_952, "kernel_sha": "d284513126c47679",
+PREFILL_TRAFFIC = {"bytes_per_launch": 568_925_952, "kernel_sha": "538588bfa1f1bfab",
                    "capture": "profiles/paged_prefill_kernel_prefill.md"}
 
 

@@ -11,12 +11,11 @@
 // each, x the G query heads of one KV head) of one sequence, against 128-key
 // tiles of that KV head read through the block table.  Both query tiles use
 // every K/V tile the CTA loads, which halves the K/V bytes per FLOP of a
-// one-tile CTA.  Warp roles:
-//   warps 0,10 TMA: warp 0 both Q tiles once, then K tiles into a 3-stage
-//              ring, warp 10 V tiles into a 2-stage ring, block by block (one
-//              4-D box per 16- or 32-token block and 64-column chunk,
-//              128-byte swizzle), each reading its table entries one tile
-//              ahead;
+// one-tile CTA.  Warp roles (19 warps):
+//   warps 0,18 TMA: warp 0 both Q tiles once, then K tiles, warp 18 V tiles,
+//              each into a 2-stage ring, block by block (one 4-D box per 16-
+//              or 32-token block and 64-column chunk, 128-byte swizzle), each
+//              reading its table entries one tile ahead;
 //   warp 1     allocates all 512 TMEM columns (S_A, S_B, O_A, O_B); one thread
 //              issues the MMAs in the order
 //                S_A(0), PV_A(0), S_A(1), S_B(0), PV_B(0), S_B(1), PV_A(1), S_A(2), ...
@@ -26,15 +25,16 @@
 //              memory, V an MN-major shared-memory operand).  The MMAs of a CTA
 //              execute in issue order, which is what lets P overwrite the S it
 //              came from and S_X(j+1) overwrite P_X(j) once PV_X(j) has read it;
-//   warps 2-5  softmax of tile A, warps 6-9 of tile B: one query row per
-//              thread (TMEM lane = row).  Read S (two 64-column halves, the
-//              first read twice to keep the registers down), mask, online
-//              softmax in base 2 with a running maximum that is only moved when
-//              the new one exceeds it by more than 2^8 (the result does not
-//              depend on the reference maximum; the lag only bounds the
-//              weights), write P as packed 16-bit pairs into the upper half of
-//              the same S columns with tcgen05.st, and rescale O in TMEM when
-//              the maximum moves; finally O / l.
+//   warps 2-9  softmax of tile A, warps 10-17 of tile B, two warps per TMEM
+//              lane quarter: each thread takes one query row (TMEM lane = row)
+//              and 64 of its 128 keys, the two halves of a row exchanging their
+//              maxima through shared memory.  Read S, mask, online softmax in
+//              base 2 with a running maximum that is only moved when the new
+//              one exceeds it by more than 2^8 (the result does not depend on
+//              the reference maximum; the lag only bounds the weights), write P
+//              as packed 16-bit pairs into the upper half of the same S columns
+//              with tcgen05.st, and rescale O in TMEM when the maximum moves;
+//              finally O / l.
 // While tile A's softmax works on S_A(j+1), the tensor core computes PV_B(j)
 // and S_B(j+1), and the other way round.
 //
@@ -416,7 +416,7 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
     const uint32_t tmem = flags.tmem_base;
 
     if (warp == 0 || warp == kVWarp) {
-        // ---------------- TMA producers: warp 0 loads Q and K, warp 10 loads V ----------------
+        // ---------------- TMA producers: warp 0 loads Q and K, the last warp loads V ----------------
         const bool is_k = warp == 0;
         const int nst = is_k ? kKStages : kVStages;
         const uint64_t pol = l2_policy_evict_last();      // K/V tiles are read again by the other query tiles
