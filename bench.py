@@ -45,11 +45,11 @@ FALLBACK_HBM_GBS = 6650.0
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by workload, valid only
 # for the decode kernel source it was measured on (sha256 prefix of decode.cu).
 NCU_TRAFFIC = {
-    "opt13b": {"bytes_per_launch": 1_316_705_536, "kernel_sha": "50dd0cd8f2ba18ba",
+    "opt13b": {"bytes_per_launch": 1_316_705_536, "kernel_sha": "05714f1368298826",
                "capture": "profiles/paged_decode_kernel_opt13b.md (opt13b_compact: same sequences)"},
-    "gqa": {"bytes_per_launch": 1_224_799_136, "kernel_sha": "50dd0cd8f2ba18ba",
+    "gqa": {"bytes_per_launch": 1_224_799_136, "kernel_sha": "05714f1368298826",
             "capture": "profiles/paged_decode_kernel_gqa.md (gqa_compact: same sequences)"},
-    "fp8": {"bytes_per_launch": 1_118_479_160, "kernel_sha": "50dd0cd8f2ba18ba",
+    "fp8": {"bytes_per_launch": 1_118_479_160, "kernel_sha": "05714f1368298826",
             "capture": "profiles/paged_decode_kernel_fp8.md (fp8_compact: same sequences, 512-token partitions)"},
 }
 

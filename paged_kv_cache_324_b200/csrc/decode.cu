@@ -1016,11 +1016,23 @@ namespace pkv {
 namespace {
 // The prefix pass is partitioned on its own: it has one work unit per (unit, KV head)
 // and partition, so its partitions shrink until the SMs have enough of them.
+//
+// Automatic choice: a whole prefix per CTA needs no merge of prefix partitions, so a prefix is only
+// split while the (unit, KV head) pairs would leave more than a quarter of the CTA slots empty.  The
+// slots are those of the 16-row instance (two CTAs per SM), which units of 16 / G sequences use.
 int prefix_partition(int num_units, int num_kv_heads, int head_dim, pkv_dtype kv_dtype, int block_size,
                      int max_prefix_len, int partition_size) {
     if (max_prefix_len <= 0) return block_size;
-    return pkv_decode_partition_size(num_units > 0 ? num_units : 1, num_kv_heads, head_dim, kv_dtype, block_size,
-                                     max_prefix_len, partition_size);
+    if (partition_size > 0)
+        return pkv_decode_partition_size(num_units > 0 ? num_units : 1, num_kv_heads, head_dim, kv_dtype,
+                                         block_size, max_prefix_len, partition_size);
+    const long long slots = 2LL * num_sms();
+    const long long pairs = static_cast<long long>(num_units > 0 ? num_units : 1) * num_kv_heads;
+    const int nblk = (max_prefix_len + block_size - 1) / block_size;
+    const int max_split = nblk / 4 > 1 ? nblk / 4 : 1;   // at least four blocks per partition
+    int k = 1;
+    while (k < max_split && pairs * k * 4 < slots * 3) ++k;
+    return (nblk + k - 1) / k * block_size;
 }
 }  // namespace
 }  // namespace pkv
