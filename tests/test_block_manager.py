@@ -285,3 +285,168 @@ def test_swap_is_all_or_nothing(BM):
     assert e.value.status == 6 and gpu.sequence_length(0) == 8 and host.num_free == 1
     with pytest.raises(PagedKVError):
         gpu.swap_to(host, [5])                                # unknown sequence
+
+
+class _ModelManager:
+    """An independent Python statement of the manager's rules, for randomized comparison:
+    FIFO free list; a new block only when the last is full; fork shares; copy on write for a
+    shared partial last block (the last holder writes in place); full blocks registered under
+    their token content chained on their predecessor, hits confirmed exactly (tokens, the
+    predecessor block and its generation); registered blocks without holders stay cached and are
+    reused oldest-released first when the free list is empty."""
+
+    def __init__(self, n, bs, order):
+        self.bs = bs
+        self.free = list(order)
+        self.ref = [0] * n
+        self.seqs = {}
+        self.key_of = {}          # block -> (content key)
+        self.cache = {}           # content key -> block
+        self.gen = [0] * n
+        self.idle = []            # cached blocks with no holder, oldest first
+
+    def _take(self):
+        if self.free:
+            b = self.free.pop(0)
+        else:
+            b = self.idle.pop(0)
+            self._uncache(b)
+        self.ref[b] = 1
+        return b
+
+    def _uncache(self, b):
+        k = self.key_of.pop(b)
+        if self.cache.get(k) == b:
+            del self.cache[k]
+        self.gen[b] += 1
+
+    def _release(self, b):
+        self.ref[b] -= 1
+        if self.ref[b] == 0:
+            (self.idle if b in self.key_of else self.free).append(b)
+
+    def _acquire(self, b):
+        if b in self.idle:
+            self.idle.remove(b)
+        self.ref[b] += 1
+
+    def available(self):
+        return len(self.free) + len(self.idle)
+
+    def append(self, ids):
+        need, copied = 0, {}
+        for s in ids:
+            blocks, L = self.seqs[s]
+            if L % self.bs == 0:
+                need += 1
+            else:
+                last = blocks[-1]
+                if self.ref[last] - copied.get(last, 0) > 1:
+                    copied[last] = copied.get(last, 0) + 1
+                    need += 1
+        if need > self.available():
+            return None
+        slots, pairs = [], []
+        for s in ids:
+            blocks, L = self.seqs[s]
+            off = L % self.bs
+            if off == 0:
+                blocks.append(self._take())
+            elif self.ref[blocks[-1]] > 1:
+                fresh = self._take()
+                pairs.append((blocks[-1], fresh))
+                self.ref[blocks[-1]] -= 1
+                blocks[-1] = fresh
+            slots.append(blocks[-1] * self.bs + off)
+            self.seqs[s] = (blocks, L + 1)
+        return slots, pairs
+
+    def fork(self, p, c):
+        blocks, L = self.seqs[p]
+        for b in blocks:
+            self._acquire(b)
+        self.seqs[c] = (list(blocks), L)
+
+    def free_seq(self, s):
+        for b in self.seqs.pop(s)[0]:
+            self._release(b)
+
+    def cache_seq(self, s, toks):
+        blocks, _ = self.seqs[s]
+        prev, prev_gen = -1, 0
+        for j in range(len(toks) // self.bs):
+            b = blocks[j]
+            key = (tuple(toks[j * self.bs:(j + 1) * self.bs]), prev, prev_gen)
+            if b not in self.key_of and key not in self.cache:
+                self.key_of[b] = key
+                self.cache[key] = b
+            prev, prev_gen = b, self.gen[b]
+
+    def add_cached(self, s, toks):
+        got, prev, prev_gen = [], -1, 0
+        for j in range((len(toks) - 1) // self.bs if len(toks) else 0):
+            key = (tuple(toks[j * self.bs:(j + 1) * self.bs]), prev, prev_gen)
+            b = self.cache.get(key)
+            if b is None:
+                break
+            got.append(b)
+            prev, prev_gen = b, self.gen[b]
+        for b in got:
+            self._acquire(b)
+        self.seqs[s] = (got, len(got) * self.bs)
+        return len(got) * self.bs
+
+
+def test_randomized_against_a_python_model(BM):
+    """Random add / cached add / append / fork / register / free sequences: the library and the
+    model give the same slots, copy pairs, cached-token counts, tables and free counts."""
+    from paged_kv_cache_324_b200.binding import PagedKVError
+    rng = np.random.default_rng(31)
+    NB, B = 48, 4
+    order = rng.permutation(NB)
+    m = BM(NB, B, order)
+    py = _ModelManager(NB, B, order.tolist())
+    toks = {}                                    # tokens written per sequence
+    vocab = 3                                    # small, so prompts repeat and the cache hits
+    nxt = 0
+    for step in range(1500):
+        live = sorted(py.seqs)
+        op = rng.integers(0, 6)
+        if op == 0 or not live:
+            prompt = rng.integers(0, vocab, size=int(rng.integers(1, 14))).tolist()
+            got = m.add_sequence_cached(nxt, prompt)
+            assert got == py.add_cached(nxt, prompt)
+            toks[nxt] = prompt[:got]
+            nxt += 1
+        elif op == 1:
+            p = int(rng.choice(live))
+            m.fork(p, nxt)
+            py.fork(p, nxt)
+            toks[nxt] = list(toks[p])
+            nxt += 1
+        elif op == 2 and len(live) > 2:
+            s = int(rng.choice(live))
+            m.free_sequence(s)
+            py.free_seq(s)
+            del toks[s]
+        elif op == 3:
+            s = int(rng.choice(live))
+            m.cache_sequence(s, toks[s])
+            py.cache_seq(s, toks[s])
+        else:
+            ids = [int(x) for x in rng.choice(live, size=min(len(live), int(rng.integers(1, 4))), replace=False)]
+            want = py.append(ids)
+            if want is None:
+                with pytest.raises(PagedKVError):
+                    m.append_slots(ids)
+                continue
+            slots, pairs = m.append_slots(ids)
+            assert slots.tolist() == want[0] and [tuple(p) for p in pairs.tolist()] == want[1]
+            for s in ids:
+                toks[s].append(int(rng.integers(0, vocab)))
+        assert m.num_free == py.available()
+    live = sorted(py.seqs)
+    tabs, lens = m.block_tables(live, 16)
+    for i, s in enumerate(live):
+        blocks, L = py.seqs[s]
+        assert tabs[i, :len(blocks)].tolist() == blocks and lens[i] == L
