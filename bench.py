@@ -349,7 +349,8 @@ def run_prefill(args, rank, world, local_rank):
         e2e_step()
     e2.record()
     barrier_sync(torch, dist_on)
-    e2e_ms = max_over_ranks(torch, s2.elapsed_time(e2), dist_on) / K
+    e2e_serial_ms = max_over_ranks(torch, s2.elapsed_time(e2), dist_on) / K
+    e2e_ms = pipelined_e2e_ms(torch, dev, ps, pinned, args.warmup, K, dist_on)
     peak, peak_sus, kind = tensor_peak()
     achieved = flops / (pf_ms * 1e-3) / 1e12
     line = {
@@ -377,7 +378,10 @@ def run_prefill(args, rank, world, local_rank):
                      "flops_counted": "4 * head_dim * num_heads * causal (query, key) pairs",
                      "peak_kind": f"{kind} (cuBLAS bf16, burst; sustained {peak_sus})"},
         "e2e": {"value": round(total_flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-                "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "overlap": PIPELINE_NOTE,
+                "serial_value": round(total_flops / (e2e_serial_ms * 1e-3) / 1e12, 2),
+                "serial_ms_per_step": round(e2e_serial_ms, 5)},
         "gpu_launches": 2 * K,
         "timing": ("value: CUDA events around K back-to-back steps; kernel_ms and roofline: CUDA events "
                    "around each call in a second run of K steps"),
@@ -532,6 +536,63 @@ def run_swap(args, rank, world, local_rank):
     return line
 
 
+def pipelined_e2e_ms(torch, dev, step_obj, pinned, warmup, K, dist_on) -> float:
+    """Milliseconds per step of the end-to-end loop as a serving engine runs it: two sets of input
+    and output buffers and one copy stream per direction, so that step i+1's inputs cross the
+    link while step i computes and step i-1's output comes back.  Every step still copies all of
+    its inputs in (from the pinned host tensors in `pinned`) and its output back.  `step_obj`
+    has `d` (device inputs by the same keys), `out`, `stream` and `step()`."""
+    import copy as _copy
+    second = _copy.copy(step_obj)
+    second.d = {k: v.clone() for k, v in step_obj.d.items()}
+    second.out = torch.empty_like(step_obj.out)
+    sets = [step_obj, second]
+
+    def as_bits(t):
+        return t.view(torch.int16) if t.dtype in (torch.float16, torch.bfloat16) else t
+
+    dst = [{k: as_bits(x.d[k]) for k in pinned} for x in sets]
+    out_host = [torch.empty(step_obj.out.shape, dtype=step_obj.out.dtype).pin_memory() for _ in sets]
+    comp, s_in, s_out = step_obj.stream, torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_ready = [torch.cuda.Event() for _ in range(2)]
+    ev_free = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+
+    def run(n):
+        for i in range(n):
+            b = i % 2
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_free[b])             # the set's previous step and read-back are done
+                for k, v in pinned.items():
+                    dst[b][k].copy_(v, non_blocking=True)
+                ev_ready[b].record(s_in)
+            comp.wait_event(ev_ready[b])
+            sets[b].step()
+            ev_done[b].record(comp)
+            with torch.cuda.stream(s_out):                  # a read-back must not hold up the next inputs
+                s_out.wait_event(ev_done[b])
+                out_host[b].copy_(sets[b].out, non_blocking=True)
+                ev_free[b].record(s_out)
+        comp.wait_stream(s_in)
+        comp.wait_stream(s_out)
+
+    run(max(warmup, 2))
+    barrier_sync(torch, dist_on)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(comp)
+    s_in.wait_event(s)
+    s_out.wait_event(s)
+    run(K)
+    e.record(comp)
+    barrier_sync(torch, dist_on)
+    return max_over_ranks(torch, s.elapsed_time(e), dist_on) / K
+
+
+PIPELINE_NOTE = ("two buffer sets and one copy stream per direction: step i+1's inputs are copied in, and "
+                 "step i-1's output copied back, while step i computes")
+
+
 def barrier_sync(torch, dist_on):
     if dist_on:
         import torch.distributed as dist
@@ -646,52 +707,8 @@ def run_ours(args, rank, world, local_rank):
     barrier_sync(torch, dist_on)
     e2e_serial_ms = max_over_ranks(torch, s2.elapsed_time(e2), dist_on) / K
 
-    # the same, pipelined as a serving loop would run it: two sets of input and output buffers and
-    # a copy stream, so that step i+1's inputs cross the link while step i computes; every step
-    # still copies all of its inputs in and its output back inside the timed region
-    import copy as _copy
-    ds2 = _copy.copy(ds)
-    ds2.d = {k: v.clone() for k, v in ds.d.items()}
-    ds2.out = torch.empty_like(ds.out)
-    sets = [ds, ds2]
-    dqs = [dq, {k: (ds2.d[k].view(torch.int16) if ds2.d[k].dtype in (torch.float16, torch.bfloat16) else ds2.d[k])
-                for k in pinned}]
-    outs_host = [out_host, torch.empty(ds.out.shape, dtype=ds.out.dtype).pin_memory()]
-    # one stream per direction: a read-back must not hold up the next step's inputs
-    comp, s_in, s_out = ds.stream, torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    ev_ready = [torch.cuda.Event() for _ in range(2)]
-    ev_free = [torch.cuda.Event() for _ in range(2)]
-    ev_done = [torch.cuda.Event() for _ in range(2)]
-
-    def pipelined(n):
-        for i in range(n):
-            b = i % 2
-            with torch.cuda.stream(s_in):
-                if i >= 2:
-                    s_in.wait_event(ev_free[b])             # the set's previous step and read-back are done
-                for k, v in pinned.items():
-                    dqs[b][k].copy_(v, non_blocking=True)
-                ev_ready[b].record(s_in)
-            comp.wait_event(ev_ready[b])
-            sets[b].step()
-            ev_done[b].record(comp)
-            with torch.cuda.stream(s_out):
-                s_out.wait_event(ev_done[b])
-                outs_host[b].copy_(sets[b].out, non_blocking=True)
-                ev_free[b].record(s_out)
-        comp.wait_stream(s_in)
-        comp.wait_stream(s_out)
-
-    pipelined(max(args.warmup, 2))
-    barrier_sync(torch, dist_on)
-    s3, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s3.record(comp)
-    s_in.wait_event(s3)
-    s_out.wait_event(s3)
-    pipelined(K)
-    e3.record(comp)
-    barrier_sync(torch, dist_on)
-    e2e_ms = max_over_ranks(torch, s3.elapsed_time(e3), dist_on) / K
+    # the same, pipelined as a serving loop runs it
+    e2e_ms = pipelined_e2e_ms(torch, dev, ds, pinned, args.warmup, K, dist_on)
     e2e_value = total_bytes / (e2e_ms * 1e-3) / 1e9
     e2e_serial_value = total_bytes / (e2e_serial_ms * 1e-3) / 1e9
 
@@ -738,8 +755,7 @@ def run_ours(args, rank, world, local_rank):
                      "peak_kind": f"{peak_kind} (copy, burst)"},
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "ms_per_step": round(e2e_ms, 5),
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "overlap": "two buffer sets and one copy stream per direction: step i+1's inputs are copied "
-                           "in, and step i-1's output copied back, while step i computes",
+                "overlap": PIPELINE_NOTE,
                 "serial_value": round(e2e_serial_value, 2), "serial_ms_per_step": round(e2e_serial_ms, 5)},
         "gpu_launches": ds.launches_per_step() * K,
         "timing": ("value: CUDA events around K back-to-back steps; kernel_ms and roofline: CUDA events "
