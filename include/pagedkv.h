@@ -1,5 +1,5 @@
 /*
- * pagedkv.h -- C ABI of the B200 (sm_100a) paged KV-cache decode library.
+ * pagedkv.h -- C ABI of the B200 (sm_100a) paged KV-cache library.
  *
  * The KV cache of every sequence is split into fixed-size blocks that sit
  * anywhere in one shared physical pool and are reached through a
@@ -21,10 +21,17 @@
  * and the prefill of a chunk of new tokens over the same cache
  * (pkv_paged_attn_prefill: every query of the chunk attends causally, the
  * dense phase of the "vLLM and PagedAttention" transcript's opening
- * paragraph), on the 5th-generation tensor cores.
+ * paragraph), on the 5th-generation tensor cores.  Around them: a decode
+ * that reads shared prompt blocks once per group of sequences
+ * (pkv_paged_attn_decode_shared_prefix), block swapping between the device
+ * pool and pinned host memory (pkv_swap_blocks), and a host-side block
+ * manager with copy-on-write, prefix caching by block content and swap
+ * bookkeeping (pkv_bm_*).
  *
  * Conventions shared by every entry point
- *   - All pointers except scalars are DEVICE pointers, owned by the caller.
+ *   - All pointers except scalars are DEVICE pointers, owned by the caller
+ *     (exceptions, stated where they apply: the block manager's arrays are
+ *     host memory; pkv_swap_blocks also takes pinned, mapped host pools).
  *     The library allocates nothing and keeps no per-call state; calls are
  *     asynchronous on `stream` (a cudaStream_t passed as void*, NULL = the
  *     legacy default stream) and nothing synchronises.
