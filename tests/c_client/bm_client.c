@@ -1,0 +1,70 @@
+/*
+ * A plain C client of the library's C ABI (no Python): drives the host-side
+ * block manager through the glossary "PagedAttention" worked example (section
+ * "How paging works": 40 tokens, blocks of 16, free list 41, 7, 19, 2, 33 ->
+ * block table 41, 7, 19) and the copy-on-write rule of its section "Sharing
+ * blocks across sequences", and checks status strings.  Prints "ok" and exits
+ * 0 when every check holds.
+ */
+#include <stdio.h>
+#include <stdlib.h>
+
+#include "pagedkv.h"
+
+#define CHECK(c)                                                 \
+    do {                                                         \
+        if (!(c)) {                                              \
+            fprintf(stderr, "check failed: %s (line %d)\n", #c, __LINE__); \
+            return 1;                                            \
+        }                                                        \
+    } while (0)
+
+int main(void) {
+    CHECK(pkv_version() >= 100);
+    CHECK(pkv_status_string(PKV_OK) != NULL);
+
+    /* the worked example: a 64-block pool whose free list starts 41, 7, 19, 2, 33 */
+    int32_t order[64];
+    int n = 0;
+    const int32_t head[5] = {41, 7, 19, 2, 33};
+    for (int i = 0; i < 5; ++i) order[n++] = head[i];
+    for (int b = 0; b < 64; ++b) {
+        int used = 0;
+        for (int i = 0; i < 5; ++i) used |= head[i] == b;
+        if (!used) order[n++] = b;
+    }
+    pkv_block_manager* m = pkv_bm_create(64, 16, order);
+    CHECK(m != NULL);
+    CHECK(pkv_bm_add_sequence(m, 0) == PKV_OK);
+    int64_t id = 0, slot = 0, pairs[2];
+    int np = 0;
+    for (int t = 0; t < 40; ++t) {
+        CHECK(pkv_bm_append_slots(m, &id, 1, &slot, pairs, 1, &np) == PKV_OK);
+        CHECK(np == 0);
+    }
+    int32_t table[4], len = 0;
+    CHECK(pkv_bm_block_tables(m, &id, 1, table, 4, -1, &len) == PKV_OK);
+    CHECK(table[0] == 41 && table[1] == 7 && table[2] == 19 && table[3] == -1 && len == 40);
+    CHECK(3 * 16 - len == 8);                        /* unused slots under paging */
+    CHECK(slot == 19 * 16 + 39 % 16);                /* the 40th token's slot */
+
+    /* fork, then the child's first token: the shared partial block is copied for the writer */
+    CHECK(pkv_bm_fork(m, 0, 1) == PKV_OK);
+    CHECK(pkv_bm_ref_count(m, 19) == 2);
+    int64_t child = 1;
+    CHECK(pkv_bm_append_slots(m, &child, 1, &slot, pairs, 1, &np) == PKV_OK);
+    CHECK(np == 1 && pairs[0] == 19 && pairs[1] == 2);  /* the next free block in FIFO order */
+    CHECK(pkv_bm_ref_count(m, 19) == 1 && pkv_bm_ref_count(m, 41) == 2);
+    /* the parent is now the only holder of block 19: it writes in place */
+    CHECK(pkv_bm_append_slots(m, &id, 1, &slot, pairs, 1, &np) == PKV_OK);
+    CHECK(np == 0 && slot == 19 * 16 + 40 % 16);
+
+    CHECK(pkv_bm_free_sequence(m, 0) == PKV_OK);
+    CHECK(pkv_bm_free_sequence(m, 1) == PKV_OK);
+    CHECK(pkv_bm_num_free(m) == 64);
+    CHECK(pkv_bm_add_sequence(m, 1) == PKV_OK);
+    CHECK(pkv_bm_add_sequence(m, 1) == PKV_ERR_INVALID_ARG);
+    pkv_bm_destroy(m);
+    printf("ok\n");
+    return 0;
+}
