@@ -13,10 +13,18 @@ Prints one JSON line (rank 0).  ``value`` is algorithmic bytes per step
 and the copies' bytes) divided by the device time per step, summed over
 ranks; inputs are resident in HBM and larger than L2.  ``e2e`` is the same
 metric with the step's inputs copied from pinned host memory and the output
-copied back inside the timed region.  ``--impl reference`` times the CPU
-oracle (float64) on the host's cores on a bounded sample of the same workload.
-Under torchrun each rank runs its own batch (weak scaling, no collective on
-the data path); the time is the maximum over ranks.
+copied back inside the timed region, pipelined over two buffer sets and a copy
+stream per direction (``e2e.serial_value``: one after the other).
+``--impl reference`` times the CPU oracle (float64) on the host's cores on a
+bounded sample of the same workload.  Under torchrun each rank runs its own
+batch (weak scaling, no collective on the data path); the time is the maximum
+over ranks.
+
+Other configurations: the other decode workloads by name (``--prefix-aware``
+decodes shared prompts with the shared-prefix call); ``--config prefill``
+(a chunk's scatter + the tensor-core prefill, in TFLOP/s against the measured
+bf16 throughput); ``--config swap`` (blocks out to pinned host memory and back,
+in GB/s against the copy engines' rate measured in the same run).
 """
 from __future__ import annotations
 
