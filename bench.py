@@ -444,6 +444,7 @@ def run_swap(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     NB, NH, Hkv, Bs, D, n = 16384, 4096, 40, 16, 128, 1024     # 1024 blocks = 16 sequences of 1,024 tokens
     rng = np.random.default_rng(7)
+    torch.manual_seed(7)
     kp = torch.empty((NB, Hkv, Bs, D), dtype=torch.float16, device=dev).normal_()
     vp = torch.empty_like(kp).normal_()
     hk = torch.empty((NH, Hkv, Bs, D), dtype=torch.float16).pin_memory()
