@@ -274,6 +274,29 @@ pkv_status pkv_paged_attn_prefill(void* out, const void* q, pkv_dtype dtype, con
                                   void* stream);
 
 /*
+ * Chunked prefill over an FP8_E4M3 cache (glossary, section "Related methods":
+ * an 8-bit KV cache), same result definition as pkv_paged_attn_prefill with
+ * k_t = e4m3(K byte) * k_scale and v_t = e4m3(V byte) * v_scale.  A gather
+ * kernel widens the blocks each sequence's queries can reach into 16-bit
+ * pools inside `workspace` (one row of max_blocks_per_seq blocks per
+ * sequence; K exactly, V times v_scale rounded once to q_dtype), then the
+ * tensor-core prefill runs on them with scale * k_scale.  Arguments as for
+ * pkv_paged_attn_prefill, except: q_dtype in {F16, BF16} is also the output
+ * type; the pools hold E4M3 bytes; k_scale, v_scale > 0; workspace: device
+ * memory of at least pkv_prefill_fp8_workspace_bytes() bytes, 256-byte
+ * aligned.  A bad block id yields PKV_DEVERR_BLOCK_ID and NaN rows.
+ */
+size_t pkv_prefill_fp8_workspace_bytes(int num_seqs, int max_blocks_per_seq, int num_kv_heads, int head_dim,
+                                       int block_size);
+pkv_status pkv_paged_attn_prefill_fp8(void* out, const void* q, pkv_dtype q_dtype, const void* k_pool,
+                                      const void* v_pool, float k_scale, float v_scale, const int32_t* block_tables,
+                                      int max_blocks_per_seq, const int32_t* context_lens,
+                                      const int32_t* query_start, int max_query_len, int num_seqs, int num_tokens,
+                                      int num_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                      float scale, void* workspace, size_t workspace_bytes, uint32_t* device_error,
+                                      void* stream);
+
+/*
  * Scatter new tokens into the pool (glossary "PagedAttention", section "How
  * paging works").  For every token t with slot = slot_mapping[t] >= 0 and
  * every KV head h:

@@ -53,6 +53,11 @@ def lib() -> ctypes.CDLL:
         L.pkv_paged_attn_decode.restype = I
         L.pkv_paged_attn_prefill.argtypes = [P, P, I, P, P, P, I, P, P, I, I, I, I, I, I, I, I, F, P, P]
         L.pkv_paged_attn_prefill.restype = I
+        L.pkv_prefill_fp8_workspace_bytes.argtypes = [I, I, I, I, I]
+        L.pkv_prefill_fp8_workspace_bytes.restype = Z
+        L.pkv_paged_attn_prefill_fp8.argtypes = [P, P, I, P, P, F, F, P, I, P, P, I, I, I, I, I, I, I, I, F, P, Z,
+                                                 P, P]
+        L.pkv_paged_attn_prefill_fp8.restype = I
         L.pkv_reshape_and_cache.argtypes = [P, P, I, P, P, I, F, F, P, I, I, I, I, I, P, P]
         L.pkv_reshape_and_cache.restype = I
         L.pkv_copy_blocks.argtypes = [P, P, Z, P, I, I, P, P]
@@ -180,6 +185,34 @@ def paged_attn_prefill(out: torch.Tensor, q: torch.Tensor, k_pool: torch.Tensor,
         _dev(query_start, "query_start"), int(max_query_len), S, T, H, Hkv, D, B, NB, float(scale),
         _dev(device_error, "device_error"), _stream(stream))
     _check(status, "paged_attn_prefill")
+    return out
+
+
+def paged_attn_prefill_fp8(out: torch.Tensor, q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
+                           block_tables: torch.Tensor, context_lens: torch.Tensor, query_start: torch.Tensor,
+                           scale: float, k_scale: float, v_scale: float, *, max_query_len: int,
+                           workspace: Optional[torch.Tensor] = None, device_error: Optional[torch.Tensor] = None,
+                           stream=None) -> torch.Tensor:
+    """Chunked prefill as paged_attn_prefill over E4M3 pools (uint8 [NB, Hkv, B, D]) with per-tensor
+    scales; q and out are f16 or bf16.  ``workspace`` (uint8) is allocated with torch if not given."""
+    T, H, D = q.shape
+    NB, Hkv, B, D2 = k_pool.shape
+    S = context_lens.numel()
+    if out.shape != q.shape or out.dtype != q.dtype or D2 != D or v_pool.shape != k_pool.shape:
+        raise ValueError("inconsistent shapes or dtypes")
+    if k_pool.dtype != torch.uint8 or v_pool.dtype != torch.uint8:
+        raise TypeError("the pools hold E4M3 bytes (uint8)")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32 or query_start.dtype != torch.int32:
+        raise TypeError("block_tables, context_lens and query_start must be int32")
+    need = lib().pkv_prefill_fp8_workspace_bytes(S, block_tables.shape[1], Hkv, D, B)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    status = lib().pkv_paged_attn_prefill_fp8(
+        _dev(out, "out"), _dev(q, "q"), _code(q), _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"), float(k_scale),
+        float(v_scale), _dev(block_tables, "block_tables"), block_tables.shape[1], _dev(context_lens, "context_lens"),
+        _dev(query_start, "query_start"), int(max_query_len), S, T, H, Hkv, D, B, NB, float(scale),
+        _dev(workspace, "workspace"), workspace.numel(), _dev(device_error, "device_error"), _stream(stream))
+    _check(status, "paged_attn_prefill_fp8")
     return out
 
 

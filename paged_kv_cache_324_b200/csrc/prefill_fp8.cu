@@ -1,0 +1,176 @@
+// pkv_paged_attn_prefill_fp8: chunked prefill over an E4M3 cache (Ultralytics glossary
+// "PagedAttention", section "Related methods": an 8-bit KV cache).
+//
+// Prefill is bound by the tensor cores, not by the cache bytes (each K/V tile is used by
+// 2 x 128 query rows), so the FP8 case reuses the 16-bit tensor-core kernel: a gather kernel
+// first widens the blocks each sequence's queries can reach into a 16-bit workspace pool laid
+// out one row of max_blocks_per_seq blocks per sequence, with a block table of its own.  E4M3
+// values are exactly representable in f16 and bf16, so K is widened exactly and its scale is
+// folded into the softmax scale; V is multiplied by its scale and rounded once to the query's
+// type.  A block id outside the pool becomes an out-of-range entry of the workspace table, which
+// the prefill kernel reports (PKV_DEVERR_BLOCK_ID) with NaN rows, as for a 16-bit cache.
+
+#include <cmath>
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "pkv_device.cuh"
+#include "pkv_host.h"
+
+namespace pkv {
+namespace {
+
+constexpr int kWidenThreads = 256;
+
+// Two E4M3 values (low byte first) -> two f16 values in one word (exact).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t x) {
+    uint32_t h;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(x));
+    return h;
+}
+
+template <bool kBf16>
+__device__ __forceinline__ uint32_t scaled_pair(uint32_t f16x2, float s) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&f16x2));
+    if constexpr (kBf16) {
+        const __nv_bfloat162 b = __floats2bfloat162_rn(f.x * s, f.y * s);
+        return *reinterpret_cast<const uint32_t*>(&b);
+    } else {
+        const __half2 h = __floats2half2_rn(f.x * s, f.y * s);
+        return *reinterpret_cast<const uint32_t*>(&h);
+    }
+}
+
+// 16 E4M3 bytes -> 16 values of the query's type, times `s` (s = 1 for K: exact).
+template <bool kBf16, bool kScale>
+__device__ __forceinline__ void widen16(const uint4& x, float s, uint4& lo, uint4& hi) {
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t a = e4m3x2_to_f16x2(static_cast<uint16_t>(w[i] & 0xffffu));
+        const uint32_t b = e4m3x2_to_f16x2(static_cast<uint16_t>(w[i] >> 16));
+        if constexpr (!kScale && !kBf16) {
+            o[2 * i] = a;
+            o[2 * i + 1] = b;
+        } else {
+            o[2 * i] = scaled_pair<kBf16>(a, kScale ? s : 1.f);
+            o[2 * i + 1] = scaled_pair<kBf16>(b, kScale ? s : 1.f);
+        }
+    }
+    lo = make_uint4(o[0], o[1], o[2], o[3]);
+    hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+// Flat index over (sequence s, table slot j, 16-byte vector of the block): block s * maxb + j of
+// the workspace pools receives the widened block block_tables[s][j], for j < ceil(L_s / B).
+template <bool kBf16>
+__global__ void __launch_bounds__(kWidenThreads)
+widen_blocks_kernel(const uint4* __restrict__ k_pool, const uint4* __restrict__ v_pool, uint4* __restrict__ wk,
+                    uint4* __restrict__ wv, int32_t* __restrict__ wtab, const int32_t* __restrict__ tables,
+                    const int32_t* __restrict__ lens, int num_seqs, int maxb, long long vec_per_block,
+                    int block_size, int num_blocks, float v_scale, uint32_t* err) {
+    pdl_trigger();
+    pdl_wait();   // the pool may still be written by the previous kernel (the chunk's scatter)
+    const long long total = static_cast<long long>(num_seqs) * maxb * vec_per_block;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long blk = i / vec_per_block;
+        const long long e = i - blk * vec_per_block;
+        const int s = static_cast<int>(blk / maxb), j = static_cast<int>(blk - static_cast<long long>(s) * maxb);
+        const int L = __ldg(lens + s);
+        const long long cap = static_cast<long long>(maxb) * block_size;
+        const int nb = L <= 0 ? 0 : static_cast<int>((min(static_cast<long long>(L), cap) + block_size - 1) / block_size);
+        if (j >= nb) continue;
+        const int pid = __ldg(tables + blk);
+        const bool bad = pid < 0 || pid >= num_blocks;
+        if (e == 0) {
+            wtab[blk] = bad ? -1 : static_cast<int32_t>(blk);
+            if (bad) raise_error(err, PKV_DEVERR_BLOCK_ID);
+        }
+        if (bad) continue;
+        const long long src = static_cast<long long>(pid) * vec_per_block + e;
+        uint4 lo, hi;
+        widen16<kBf16, false>(k_pool[src], 1.f, lo, hi);
+        wk[2 * i] = lo;
+        wk[2 * i + 1] = hi;
+        widen16<kBf16, true>(v_pool[src], v_scale, lo, hi);
+        wv[2 * i] = lo;
+        wv[2 * i + 1] = hi;
+    }
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" size_t pkv_prefill_fp8_workspace_bytes(int num_seqs, int max_blocks_per_seq, int num_kv_heads,
+                                                  int head_dim, int block_size) {
+    if (num_seqs <= 0 || max_blocks_per_seq <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0) return 0;
+    const size_t blocks = static_cast<size_t>(num_seqs) * max_blocks_per_seq;
+    const size_t pool = blocks * num_kv_heads * block_size * head_dim * 2;
+    return 2 * pkv::align256(pool) + pkv::align256(blocks * sizeof(int32_t));
+}
+
+extern "C" pkv_status pkv_paged_attn_prefill_fp8(void* out, const void* q, pkv_dtype q_dtype, const void* k_pool,
+                                                 const void* v_pool, float k_scale, float v_scale,
+                                                 const int32_t* block_tables, int max_blocks_per_seq,
+                                                 const int32_t* context_lens, const int32_t* query_start,
+                                                 int max_query_len, int num_seqs, int num_tokens, int num_heads,
+                                                 int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                                 float scale, void* workspace, size_t workspace_bytes,
+                                                 uint32_t* device_error, void* stream) {
+    using namespace pkv;
+    // the same checks as pkv_paged_attn_prefill, before anything is launched
+    if (num_seqs < 0 || num_tokens < 0 || max_query_len < 0 || num_heads <= 0 || num_kv_heads <= 0 ||
+        num_blocks <= 0 || max_blocks_per_seq <= 0 || !(scale > 0.f) || !std::isfinite(scale) ||
+        !(k_scale > 0.f) || !std::isfinite(k_scale) || !(v_scale > 0.f) || !std::isfinite(v_scale))
+        return PKV_ERR_INVALID_ARG;
+    if (num_heads % num_kv_heads != 0) return PKV_ERR_INVALID_ARG;
+    if (q_dtype != PKV_F16 && q_dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
+    const int G = num_heads / num_kv_heads;
+    if ((head_dim != 64 && head_dim != 128) || (block_size != 16 && block_size != 32) ||
+        (G != 1 && G != 2 && G != 4 && G != 8 && G != 16))
+        return PKV_ERR_UNSUPPORTED;
+    const float folded = scale * k_scale;
+    if (!(folded > 0.f) || !std::isfinite(folded)) return PKV_ERR_INVALID_ARG;
+    if (num_seqs == 0 || num_tokens == 0 || max_query_len == 0) return PKV_OK;
+    if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens || !query_start) return PKV_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) ||
+        (reinterpret_cast<uintptr_t>(block_tables) & 3) || (reinterpret_cast<uintptr_t>(context_lens) & 3) ||
+        (reinterpret_cast<uintptr_t>(query_start) & 3) || (reinterpret_cast<uintptr_t>(device_error) & 3))
+        return PKV_ERR_ALIGNMENT;
+    if (num_seqs > 65535 || static_cast<long long>(num_seqs) * max_blocks_per_seq > 0x7fffffffLL)
+        return PKV_ERR_INVALID_ARG;
+    const size_t need = pkv_prefill_fp8_workspace_bytes(num_seqs, max_blocks_per_seq, num_kv_heads, head_dim,
+                                                        block_size);
+    if (!workspace || workspace_bytes < need) return PKV_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255) return PKV_ERR_ALIGNMENT;
+
+    const size_t blocks = static_cast<size_t>(num_seqs) * max_blocks_per_seq;
+    const size_t pool = align256(blocks * num_kv_heads * block_size * head_dim * 2);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    void* wk = ws;
+    void* wv = ws + pool;
+    int32_t* wtab = reinterpret_cast<int32_t*>(ws + 2 * pool);
+    const long long vec_per_block = static_cast<long long>(num_kv_heads) * block_size * head_dim / 16;
+    const long long total = static_cast<long long>(blocks) * vec_per_block;
+    long long grid = (total + kWidenThreads - 1) / kWidenThreads;
+    const long long cap = static_cast<long long>(num_sms()) * 8;
+    if (grid > cap) grid = cap;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    auto launch = [&](auto kern) {
+        return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(kWidenThreads), 0, st,
+                          static_cast<const uint4*>(k_pool), static_cast<const uint4*>(v_pool),
+                          static_cast<uint4*>(wk), static_cast<uint4*>(wv), wtab, block_tables, context_lens, num_seqs,
+                          max_blocks_per_seq, vec_per_block, block_size, num_blocks, v_scale, device_error);
+    };
+    const cudaError_t e = q_dtype == PKV_BF16 ? launch(widen_blocks_kernel<true>) : launch(widen_blocks_kernel<false>);
+    if (e != cudaSuccess) return PKV_ERR_CUDA;
+    return pkv_paged_attn_prefill(out, q, q_dtype, wk, wv, wtab, max_blocks_per_seq, context_lens, query_start,
+                                  max_query_len, num_seqs, num_tokens, num_heads, num_kv_heads, head_dim, block_size,
+                                  static_cast<int>(blocks), folded, device_error, stream);
+}

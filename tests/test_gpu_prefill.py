@@ -148,3 +148,40 @@ def test_full_size_sampled_rows():
             refs.append(ref[0])
     ok, rep = prefill_close(o[rows], np.stack(refs), w.dtype, vmax)
     assert ok, rep
+
+
+@pytest.mark.parametrize("dtype,Hq,Hkv,Bs,prior,chunks", [
+    ("f16", 8, 2, 16, [100, 0, 300], [60, 129, 1]),
+    ("bf16", 16, 2, 32, [700, 37], [150, 90]),
+])
+def test_fp8_cache_prefill_matches_oracle(dtype, Hq, Hkv, Bs, prior, chunks):
+    """E4M3 pools written by the library's scatter (per-tensor amax scales), prefilled through the
+    widening gather and the tensor-core kernel, against the oracle on the dequantised values (the
+    FP8 comparison rule: max-abs 3e-2, relative L2 1e-2)."""
+    dev = torch.device("cuda:0")
+    w = wl.chunked_prefill("fp8", 120 + Hq, Hq, Hkv, 128, Bs, 256, dtype, prior, chunks)
+    ops = [op for op in list(w.setup) + [w.step_scatter] if op.slots.size]
+    ks = max(wl.amax_scale(op.k, dtype) for op in ops)
+    vs = max(wl.amax_scale(op.v, dtype) for op in ops)
+    rng = np.random.default_rng(7)
+    shape = (w.num_blocks, Hkv, Bs, 128)
+    kp_h = wl.garbage_bytes(rng, int(np.prod(shape))).reshape(shape)
+    vp_h = wl.garbage_bytes(rng, int(np.prod(shape))).reshape(shape)
+    kp, vp = torch.from_numpy(kp_h.copy()).to(dev), torch.from_numpy(vp_h.copy()).to(dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    for op in ops:
+        B.reshape_and_cache(H.to_dev_bits(op.k, dtype, dev), H.to_dev_bits(op.v, dtype, dev), kp, vp,
+                            torch.from_numpy(op.slots).to(dev), float(ks), float(vs), device_error=err)
+        oracle.reshape_and_cache(op.k, op.v, dtype, kp_h, vp_h, "e4m3", op.slots, ks, vs)
+    q = H.to_dev_bits(w.q, dtype, dev)
+    out = torch.full_like(q, float("nan"))
+    B.paged_attn_prefill_fp8(out, q, kp, vp, torch.from_numpy(w.block_tables).to(dev),
+                             torch.from_numpy(w.context_lens).to(dev), torch.from_numpy(w.query_start).to(dev),
+                             float(w.scale), float(ks), float(vs), max_query_len=w.max_query_len, device_error=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert np.array_equal(kp.cpu().numpy(), kp_h) and np.array_equal(vp.cpu().numpy(), vp_h)
+    ref = oracle.paged_attn_prefill(w.q, dtype, kp_h, vp_h, "e4m3", w.block_tables, w.context_lens, w.query_start,
+                                    w.scale, k_scale=ks, v_scale=vs)
+    ok, rep = attention_close(H.out_f64(out), ref, "e4m3", dtype)
+    assert ok, rep
