@@ -23,7 +23,8 @@ over ranks.
 Other configurations: the other decode workloads by name (``--prefix-aware``
 decodes shared prompts with the shared-prefix call); ``--config prefill``
 (a chunk's scatter + the tensor-core prefill, in TFLOP/s against the measured
-bf16 throughput); ``--config swap`` (blocks out to pinned host memory and back,
+bf16 throughput); ``--config prefill_fp8`` (the same over an E4M3 cache: the
+quantising scatter, the widening gather and the prefill); ``--config swap`` (blocks out to pinned host memory and back,
 in GB/s against the copy engines' rate measured in the same run).
 """
 from __future__ import annotations
@@ -245,22 +246,36 @@ class DeviceStep:
 class PrefillStep:
     """The chunked-prefill workload on one GPU: the cache built, the chunk's inputs resident."""
 
-    def __init__(self, w: wl.PrefillWorkload, dev):
+    def __init__(self, w: wl.PrefillWorkload, dev, kv_fp8: bool = False):
         import torch
         from paged_kv_cache_324_b200 import binding as B
-        self.w, self.dev, self.B = w, dev, B
+        self.w, self.dev, self.B, self.kv_fp8 = w, dev, B, kv_fp8
         self.stream = torch.cuda.current_stream(dev)
         t16 = {"f16": torch.float16, "bf16": torch.bfloat16}
 
         def up(bits):
             return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(t16[w.dtype])
 
-        self.k_pool, self.v_pool = up(w.initial_pool("k")), up(w.initial_pool("v"))
+        self.k_scale = self.v_scale = 1.0
+        if kv_fp8:
+            # E4M3 pools with per-tensor amax / 448 scales over everything the step's cache holds
+            ops = [op for op in list(w.setup) + [w.step_scatter] if op.slots.size]
+            self.k_scale = float(max(wl.amax_scale(op.k, w.dtype) for op in ops))
+            self.v_scale = float(max(wl.amax_scale(op.v, w.dtype) for op in ops))
+            rng = np.random.default_rng(w.seed + 1)
+            n = int(np.prod(w.pool_shape))
+            self.k_pool = torch.from_numpy(wl.garbage_bytes(rng, n).reshape(w.pool_shape)).to(dev)
+            self.v_pool = torch.from_numpy(wl.garbage_bytes(rng, n).reshape(w.pool_shape)).to(dev)
+            self.ws = torch.empty(max(B.prefill_fp8_workspace_bytes(w.num_seqs, w.max_blocks, w.num_kv_heads,
+                                                                    w.head_dim, w.block_size), 256),
+                                  dtype=torch.uint8, device=dev)
+        else:
+            self.k_pool, self.v_pool = up(w.initial_pool("k")), up(w.initial_pool("v"))
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
         for op in w.setup:
             if op.slots.size:
                 B.reshape_and_cache(up(op.k), up(op.v), self.k_pool, self.v_pool, torch.from_numpy(op.slots).to(dev),
-                                    device_error=self.err)
+                                    self.k_scale, self.v_scale, device_error=self.err)
         sc = w.step_scatter
         self.host = {"q": w.q, "k_new": sc.k, "v_new": sc.v, "slots": sc.slots, "tables": w.block_tables,
                      "lens": w.context_lens, "qstart": w.query_start}
@@ -273,10 +288,16 @@ class PrefillStep:
 
     def scatter_op(self):
         self.B.reshape_and_cache(self.d["k_new"], self.d["v_new"], self.k_pool, self.v_pool, self.d["slots"],
-                                 device_error=self.err, stream=self.stream)
+                                 self.k_scale, self.v_scale, device_error=self.err, stream=self.stream)
 
     def prefill_op(self):
         w = self.w
+        if self.kv_fp8:
+            self.B.paged_attn_prefill_fp8(self.out, self.d["q"], self.k_pool, self.v_pool, self.d["tables"],
+                                          self.d["lens"], self.d["qstart"], float(w.scale), self.k_scale,
+                                          self.v_scale, max_query_len=w.max_query_len, workspace=self.ws,
+                                          device_error=self.err, stream=self.stream)
+            return
         self.B.paged_attn_prefill(self.out, self.d["q"], self.k_pool, self.v_pool, self.d["tables"], self.d["lens"],
                                   self.d["qstart"], float(w.scale), max_query_len=w.max_query_len,
                                   device_error=self.err, stream=self.stream)
@@ -303,8 +324,9 @@ def run_prefill(args, rank, world, local_rank):
     dist_on = world > 1
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
+    kv_fp8 = args.config == "prefill_fp8"
     w = wl.make_prefill()
-    ps = PrefillStep(w, dev)
+    ps = PrefillStep(w, dev, kv_fp8)
     flops = wl.prefill_flops(w)
     for _ in range(args.warmup):
         ps.step()
@@ -364,24 +386,33 @@ def run_prefill(args, rank, world, local_rank):
     line = {
         "metric": PREFILL_METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": w.dtype + " operands, f32 accumulate",
+        "vs_baseline": None,
+        "dtype": (w.dtype + " operands (E4M3 cache widened to " + w.dtype + "), f32 accumulate") if kv_fp8
+        else (w.dtype + " operands, f32 accumulate"),
         "data": "synthetic (seeded N(0,1) q/K/V; random-byte pool content in unwritten slots)",
-        "config": {"workload": w.description, "name": w.name, "num_seqs": w.num_seqs, "num_tokens": w.num_tokens,
+        "config": {"workload": w.description + (", E4M3 cache (per-tensor amax/448 scales)" if kv_fp8 else ""),
+                   "name": "prefill_fp8" if kv_fp8 else w.name, "num_seqs": w.num_seqs, "num_tokens": w.num_tokens,
                    "num_heads": w.num_heads, "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
                    "block_size": w.block_size, "num_blocks": w.num_blocks,
                    "total_context_tokens": int(w.context_lens.sum()), "flops_per_step": flops,
-                   "step": "reshape_and_cache (the chunk's K/V) + paged_attn_prefill",
+                   "step": ("reshape_and_cache (the chunk's K/V, quantised to E4M3) + paged_attn_prefill_fp8 "
+                            "(widen_blocks_kernel, then paged_prefill_kernel)") if kv_fp8
+                   else "reshape_and_cache (the chunk's K/V) + paged_attn_prefill",
                    "l2": "no flush: the step reads %.0f MB of K/V and q, %.0f MB of output are written; the "
                          "kernel is bound by the tensor cores, not HBM" % (wl.prefill_bytes(w) / 1e6,
                                                                            w.num_tokens * w.num_heads * w.head_dim * 2 / 1e6),
                    "parallelism": f"dp{world}" if world > 1 else "single GPU"},
         "tokens_per_s": round(sum_over_ranks(torch, float(w.num_tokens), dist_on) / (ms_step * 1e-3), 1),
-        "kernel_ms": {"paged_attn_prefill": round(pf_ms, 5), "reshape_and_cache": round(sc_ms, 5)},
-        "roofline": {"bound": "tensor", "kernel": "paged_prefill_kernel", "achieved": round(achieved, 2),
+        "kernel_ms": {("paged_attn_prefill_fp8" if kv_fp8 else "paged_attn_prefill"): round(pf_ms, 5),
+                      "reshape_and_cache": round(sc_ms, 5)},
+        "roofline": {"bound": "tensor",
+                     "kernel": ("the paged_attn_prefill_fp8 call (widen_blocks_kernel + paged_prefill_kernel)"
+                                if kv_fp8 else "paged_prefill_kernel"),
+                     "achieved": round(achieved, 2),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "frac_of_sustained": round(achieved / peak_sus, 4),
                      "traffic": (PREFILL_TRAFFIC["bytes_per_launch"]
-                                 if PREFILL_TRAFFIC["kernel_sha"] == prefill_source_sha() else None),
+                                 if PREFILL_TRAFFIC["kernel_sha"] == prefill_source_sha() and not kv_fp8 else None),
                      "flops_per_launch": flops,
                      "flops_counted": "4 * head_dim * num_heads * causal (query, key) pairs",
                      "peak_kind": f"{kind} (cuBLAS bf16, burst; sustained {peak_sus})"},
@@ -390,7 +421,7 @@ def run_prefill(args, rank, world, local_rank):
                 "overlap": PIPELINE_NOTE,
                 "serial_value": round(total_flops / (e2e_serial_ms * 1e-3) / 1e12, 2),
                 "serial_ms_per_step": round(e2e_serial_ms, 5)},
-        "gpu_launches": 2 * K,
+        "gpu_launches": (3 if kv_fp8 else 2) * K,
         "timing": ("value: CUDA events around K back-to-back steps; kernel_ms and roofline: CUDA events "
                    "around each call in a second run of K steps"),
         "clocks": clk.report(),
@@ -401,13 +432,23 @@ def run_prefill(args, rank, world, local_rank):
 class PrefillOracleRunner:
     """The float64 oracle's prefill on the host's cores, holding the workload's pools (built once)."""
 
-    def __init__(self, w: wl.PrefillWorkload):
+    def __init__(self, w: wl.PrefillWorkload, kv_fp8: bool = False):
         import oracle
         self.o, self.w = oracle, w
-        self.kp, self.vp = w.initial_pool("k"), w.initial_pool("v")
-        for op in list(w.setup) + [w.step_scatter]:
-            if op.slots.size:
-                oracle.reshape_and_cache(op.k, op.v, w.dtype, self.kp, self.vp, w.dtype, op.slots)
+        ops = [op for op in list(w.setup) + [w.step_scatter] if op.slots.size]
+        if kv_fp8:
+            self.kv_dtype = "e4m3"
+            self.ks = float(max(wl.amax_scale(op.k, w.dtype) for op in ops))
+            self.vs = float(max(wl.amax_scale(op.v, w.dtype) for op in ops))
+            rng = np.random.default_rng(w.seed + 1)
+            n = int(np.prod(w.pool_shape))
+            self.kp = wl.garbage_bytes(rng, n).reshape(w.pool_shape)
+            self.vp = wl.garbage_bytes(rng, n).reshape(w.pool_shape)
+        else:
+            self.kv_dtype, self.ks, self.vs = w.dtype, 1.0, 1.0
+            self.kp, self.vp = w.initial_pool("k"), w.initial_pool("v")
+        for op in ops:
+            oracle.reshape_and_cache(op.k, op.v, w.dtype, self.kp, self.vp, self.kv_dtype, op.slots, self.ks, self.vs)
         self.rng = np.random.default_rng(12)
         self.cores = os.cpu_count() or 1
 
@@ -422,8 +463,9 @@ class PrefillOracleRunner:
             n = min(slice_rows, q1 - q0)
             r0 = int(self.rng.integers(q0, q1 - n + 1))
             L = int(w.context_lens[s]) - (q1 - q0) + (r0 - q0) + n
-            o.paged_attn_prefill(w.q[r0:r0 + n], w.dtype, self.kp, self.vp, w.dtype, w.block_tables[s:s + 1],
-                                 np.array([L], np.int32), np.array([0, n], np.int32), w.scale, threads=self.cores)
+            o.paged_attn_prefill(w.q[r0:r0 + n], w.dtype, self.kp, self.vp, self.kv_dtype, w.block_tables[s:s + 1],
+                                 np.array([L], np.int32), np.array([0, n], np.int32), w.scale, self.ks, self.vs,
+                                 threads=self.cores)
             rows += n
             flops += 4 * w.head_dim * w.num_heads * (n * (L - n) + n * (n + 1) // 2)
             el = time.perf_counter() - t0
@@ -829,8 +871,10 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--config", default="opt13b",
-                    choices=list(wl.NAMES) + list(wl.EXTRA_NAMES) + list(wl.COMPACT_NAMES) + ["prefill", "swap"],
-                    help="a decode workload, 'prefill' (chunked prefill, TFLOP/s) or 'swap' (block swap, GB/s)")
+                    choices=list(wl.NAMES) + list(wl.EXTRA_NAMES) + list(wl.COMPACT_NAMES)
+                    + ["prefill", "prefill_fp8", "swap"],
+                    help="a decode workload, 'prefill' / 'prefill_fp8' (chunked prefill over a 16-bit or an "
+                         "E4M3 cache, TFLOP/s) or 'swap' (block swap, GB/s)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--prefix-aware", action="store_true",
                     help="decode with pkv_paged_attn_decode_shared_prefix (shared prompts read once per unit)")
@@ -876,11 +920,12 @@ def main():
         print(json.dumps(line), flush=True)
         return
 
-    if args.impl == "reference" and args.config == "prefill":
+    if args.impl == "reference" and args.config in ("prefill", "prefill_fp8"):
         if rank != 0:
             return
         w = wl.make_prefill()
-        r = PrefillOracleRunner(w)
+        kv_fp8 = args.config == "prefill_fp8"
+        r = PrefillOracleRunner(w, kv_fp8)
         cores = r.cores
         per_step = min(30.0, 150.0 / (args.steps + args.warmup))
         slice_rows = 64 if per_step >= 5.0 else 1      # one row over ~2k keys takes tens of ms
@@ -892,11 +937,13 @@ def main():
                 times.append(el)
         value = sum(rates) / len(rates) / 1e12
         sample = (f"{slice_rows}-row slices of random chunks (float64 prefill, each row over its full causal "
-                  f"prefix), ~{per_step:.2f} s per step, {len(times)} timed steps")
+                  f"prefix{', E4M3 cache' if kv_fp8 else ''}), ~{per_step:.2f} s per step, {len(times)} timed steps")
         line = {"metric": PREFILL_METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": args.gpus,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * sum(times) / len(times), 3),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "impl": "reference",
-                "dtype": "f64", "data": "synthetic", "config": {"workload": w.description, "name": w.name},
+                "dtype": "f64", "data": "synthetic",
+                "config": {"workload": w.description + (", E4M3 cache (per-tensor amax/448 scales)" if kv_fp8 else ""),
+                           "name": args.config},
                 "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                                  "sample": sample},
                 "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -967,10 +1014,10 @@ def main():
             if rank == 0:
                 print(json.dumps(line), flush=True)
             return
-        if args.config == "prefill":
+        if args.config in ("prefill", "prefill_fp8"):
             line, w = run_prefill(args, rank, world, local_rank)
             if rank == 0 and world == 1:
-                r = PrefillOracleRunner(w)
+                r = PrefillOracleRunner(w, args.config == "prefill_fp8")
                 rows, flops, el = r.sample(args.cpu_budget)
                 line["cpu_baseline"] = {"value": round(flops / el / 1e12, 6), "unit": "TFLOP/s", "cores": r.cores,
                                         "kind": "oracle",

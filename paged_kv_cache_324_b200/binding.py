@@ -188,6 +188,11 @@ def paged_attn_prefill(out: torch.Tensor, q: torch.Tensor, k_pool: torch.Tensor,
     return out
 
 
+def prefill_fp8_workspace_bytes(num_seqs, max_blocks_per_seq, num_kv_heads, head_dim, block_size) -> int:
+    """Bytes of device workspace paged_attn_prefill_fp8 needs (the widened pools and their table)."""
+    return lib().pkv_prefill_fp8_workspace_bytes(num_seqs, max_blocks_per_seq, num_kv_heads, head_dim, block_size)
+
+
 def paged_attn_prefill_fp8(out: torch.Tensor, q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
                            block_tables: torch.Tensor, context_lens: torch.Tensor, query_start: torch.Tensor,
                            scale: float, k_scale: float, v_scale: float, *, max_query_len: int,
@@ -204,7 +209,7 @@ def paged_attn_prefill_fp8(out: torch.Tensor, q: torch.Tensor, k_pool: torch.Ten
         raise TypeError("the pools hold E4M3 bytes (uint8)")
     if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32 or query_start.dtype != torch.int32:
         raise TypeError("block_tables, context_lens and query_start must be int32")
-    need = lib().pkv_prefill_fp8_workspace_bytes(S, block_tables.shape[1], Hkv, D, B)
+    need = prefill_fp8_workspace_bytes(S, block_tables.shape[1], Hkv, D, B)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
     status = lib().pkv_paged_attn_prefill_fp8(
