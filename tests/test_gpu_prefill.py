@@ -10,7 +10,9 @@ sampled rows (each an oracle call of its own) and on properties that hold at
 any size.  Data-dependent errors (a bad block id, a chunk longer than its
 context) must give NaN rows and the documented error bits while the other
 sequences stay correct.  A prefill of one-token chunks must agree with the
-decode kernel.
+decode kernel.  E4M3 caches go through the widening gather and the same
+kernel, compared with the oracle on the dequantised cache, a bad block id
+included.
 """
 import numpy as np
 import pytest
@@ -150,6 +152,40 @@ def test_full_size_sampled_rows():
     assert ok, rep
 
 
+def fp8_pools(w, dev):
+    """E4M3 pools (random bytes outside the written slots) filled by the library's scatter and by
+    the oracle's, with per-tensor amax / 448 scales over everything written."""
+    ops = [op for op in list(w.setup) + [w.step_scatter] if op.slots.size]
+    ks = max(wl.amax_scale(op.k, w.dtype) for op in ops)
+    vs = max(wl.amax_scale(op.v, w.dtype) for op in ops)
+    rng = np.random.default_rng(7)
+    n = int(np.prod(w.pool_shape))
+    kp_h = wl.garbage_bytes(rng, n).reshape(w.pool_shape)
+    vp_h = wl.garbage_bytes(rng, n).reshape(w.pool_shape)
+    kp, vp = torch.from_numpy(kp_h.copy()).to(dev), torch.from_numpy(vp_h.copy()).to(dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    for op in ops:
+        B.reshape_and_cache(H.to_dev_bits(op.k, w.dtype, dev), H.to_dev_bits(op.v, w.dtype, dev), kp, vp,
+                            torch.from_numpy(op.slots).to(dev), float(ks), float(vs), device_error=err)
+        oracle.reshape_and_cache(op.k, op.v, w.dtype, kp_h, vp_h, "e4m3", op.slots, ks, vs)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert np.array_equal(kp.cpu().numpy(), kp_h) and np.array_equal(vp.cpu().numpy(), vp_h)
+    return kp, vp, kp_h, vp_h, float(ks), float(vs)
+
+
+def gpu_prefill_fp8(w, kp, vp, ks, vs, dev, block_tables=None):
+    q = H.to_dev_bits(w.q, w.dtype, dev)
+    out = torch.full_like(q, float("nan"))
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    tab = w.block_tables if block_tables is None else block_tables
+    B.paged_attn_prefill_fp8(out, q, kp, vp, torch.from_numpy(tab).to(dev),
+                             torch.from_numpy(w.context_lens).to(dev), torch.from_numpy(w.query_start).to(dev),
+                             float(w.scale), ks, vs, max_query_len=w.max_query_len, device_error=err)
+    torch.cuda.synchronize()
+    return H.out_f64(out), int(err.item())
+
+
 @pytest.mark.parametrize("dtype,Hq,Hkv,Bs,prior,chunks", [
     ("f16", 8, 2, 16, [100, 0, 300], [60, 129, 1]),
     ("bf16", 16, 2, 32, [700, 37], [150, 90]),
@@ -160,28 +196,28 @@ def test_fp8_cache_prefill_matches_oracle(dtype, Hq, Hkv, Bs, prior, chunks):
     FP8 comparison rule: max-abs 3e-2, relative L2 1e-2)."""
     dev = torch.device("cuda:0")
     w = wl.chunked_prefill("fp8", 120 + Hq, Hq, Hkv, 128, Bs, 256, dtype, prior, chunks)
-    ops = [op for op in list(w.setup) + [w.step_scatter] if op.slots.size]
-    ks = max(wl.amax_scale(op.k, dtype) for op in ops)
-    vs = max(wl.amax_scale(op.v, dtype) for op in ops)
-    rng = np.random.default_rng(7)
-    shape = (w.num_blocks, Hkv, Bs, 128)
-    kp_h = wl.garbage_bytes(rng, int(np.prod(shape))).reshape(shape)
-    vp_h = wl.garbage_bytes(rng, int(np.prod(shape))).reshape(shape)
-    kp, vp = torch.from_numpy(kp_h.copy()).to(dev), torch.from_numpy(vp_h.copy()).to(dev)
-    err = torch.zeros(1, dtype=torch.int32, device=dev)
-    for op in ops:
-        B.reshape_and_cache(H.to_dev_bits(op.k, dtype, dev), H.to_dev_bits(op.v, dtype, dev), kp, vp,
-                            torch.from_numpy(op.slots).to(dev), float(ks), float(vs), device_error=err)
-        oracle.reshape_and_cache(op.k, op.v, dtype, kp_h, vp_h, "e4m3", op.slots, ks, vs)
-    q = H.to_dev_bits(w.q, dtype, dev)
-    out = torch.full_like(q, float("nan"))
-    B.paged_attn_prefill_fp8(out, q, kp, vp, torch.from_numpy(w.block_tables).to(dev),
-                             torch.from_numpy(w.context_lens).to(dev), torch.from_numpy(w.query_start).to(dev),
-                             float(w.scale), float(ks), float(vs), max_query_len=w.max_query_len, device_error=err)
-    torch.cuda.synchronize()
-    assert int(err.item()) == 0
-    assert np.array_equal(kp.cpu().numpy(), kp_h) and np.array_equal(vp.cpu().numpy(), vp_h)
+    kp, vp, kp_h, vp_h, ks, vs = fp8_pools(w, dev)
+    o, err = gpu_prefill_fp8(w, kp, vp, ks, vs, dev)
+    assert err == 0
     ref = oracle.paged_attn_prefill(w.q, dtype, kp_h, vp_h, "e4m3", w.block_tables, w.context_lens, w.query_start,
                                     w.scale, k_scale=ks, v_scale=vs)
-    ok, rep = attention_close(H.out_f64(out), ref, "e4m3", dtype)
+    ok, rep = attention_close(o, ref, "e4m3", dtype)
+    assert ok, rep
+
+
+def test_fp8_bad_block_id_gives_nan_rows_and_flag():
+    """A table entry outside the E4M3 pool: the widening gather marks the workspace entry invalid,
+    the prefill reports PKV_DEVERR_BLOCK_ID with NaN rows, and the other sequence is unaffected."""
+    dev = torch.device("cuda:0")
+    w = wl.chunked_prefill("fp8bad", 8, 8, 2, 128, 16, 128, "f16", [40, 100], [30, 60])
+    kp, vp, kp_h, vp_h, ks, vs = fp8_pools(w, dev)
+    tab = w.block_tables.copy()
+    tab[1, 2] = w.num_blocks + 5
+    o, err = gpu_prefill_fp8(w, kp, vp, ks, vs, dev, block_tables=tab)
+    assert err & 0x1
+    r0, r1 = int(w.query_start[1]), int(w.query_start[2])
+    assert np.isnan(o[r0:r1]).any()
+    ref = oracle.paged_attn_prefill(w.q, "f16", kp_h, vp_h, "e4m3", w.block_tables, w.context_lens, w.query_start,
+                                    w.scale, k_scale=ks, v_scale=vs)
+    ok, rep = attention_close(o[:r0], ref[:r0], "e4m3", "f16")
     assert ok, rep
