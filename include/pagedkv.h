@@ -323,8 +323,9 @@ pkv_status pkv_reshape_and_cache(const void* k, const void* v, pkv_dtype in_dtyp
  *   k_pool[pairs[i][1]] := k_pool[pairs[i][0]] and the same for v_pool,
  * block_bytes = num_kv_heads * block_size * head_dim * element size, a
  * multiple of 16.  pairs is int64 [num_pairs][2] (src, dst) in device memory.
- * Precondition (not checked): destinations are distinct and no destination
- * is also a source, so the copies are independent.
+ * Precondition (not checked on the device; pkv_check_block_pairs checks a
+ * host copy): destinations are distinct and no destination is also a source,
+ * so the copies are independent.
  */
 pkv_status pkv_copy_blocks(void* k_pool, void* v_pool, size_t block_bytes,
                            const int64_t* pairs, int num_pairs, int num_blocks,
@@ -347,6 +348,21 @@ pkv_status pkv_copy_blocks(void* k_pool, void* v_pool, size_t block_bytes,
 pkv_status pkv_swap_blocks(const void* src_k_pool, const void* src_v_pool, int src_num_blocks,
                            void* dst_k_pool, void* dst_v_pool, int dst_num_blocks, size_t block_bytes,
                            const int64_t* pairs, int num_pairs, uint32_t* device_error, void* stream);
+
+/*
+ * Host-side check of the preconditions of pkv_copy_blocks and pkv_swap_blocks
+ * (glossary "PagedAttention", section "Sharing blocks across sequences": a
+ * copy-on-write gives the writer a block of its own), which the kernels cannot
+ * check without a synchronisation: pairs is int64 [num_pairs][2] (src, dst) in
+ * HOST memory; every src in [0, src_num_blocks), every dst in
+ * [0, dst_num_blocks), the destinations distinct and, when same_pool is
+ * non-zero (a copy within one pool), no destination also a source.  Returns
+ * PKV_OK or PKV_ERR_INVALID_ARG; reads pairs only, launches nothing, keeps no
+ * state.  The Python binding runs it before those calls when asked to (or
+ * when the environment variable PKV_DEBUG is set).
+ */
+pkv_status pkv_check_block_pairs(const int64_t* pairs, int num_pairs, int src_num_blocks,
+                                 int dst_num_blocks, int same_pool);
 
 /*
  * Host-side block manager (no GPU involved): the bookkeeping that produces block

@@ -238,11 +238,34 @@ def reshape_and_cache(k: torch.Tensor, v: torch.Tensor, k_pool: torch.Tensor, v_
     _check(status, "reshape_and_cache")
 
 
+def check_block_pairs(pairs, src_num_blocks: int, dst_num_blocks: int, same_pool: bool) -> None:
+    """Raise ValueError unless the (src, dst) rows of pairs (int64 [n, 2], any device; copied to the
+    host, which synchronises) are in range, the destinations distinct and, within one pool, no
+    destination also a source (pkv_check_block_pairs)."""
+    import numpy as np
+    h = pairs.detach().cpu().numpy() if isinstance(pairs, torch.Tensor) else np.asarray(pairs)
+    h = np.ascontiguousarray(h, dtype=np.int64).reshape(-1, 2)
+    f = lib().pkv_check_block_pairs
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    f.restype = ctypes.c_int
+    if f(h.ctypes.data if h.size else None, h.shape[0], int(src_num_blocks), int(dst_num_blocks),
+         1 if same_pool else 0) != 0:
+        raise ValueError("block pairs: an id out of range, a repeated destination, or (one pool) a "
+                         "destination that is also a source")
+
+
+def _debug_checks() -> bool:
+    return os.environ.get("PKV_DEBUG", "") not in ("", "0")
+
+
 def copy_blocks(k_pool: torch.Tensor, v_pool: torch.Tensor, pairs: torch.Tensor, *,
-                device_error: Optional[torch.Tensor] = None, stream=None) -> None:
-    """k_pool[dst] := k_pool[src] (and v) for each row (src, dst) of pairs (int64 [n, 2])."""
+                device_error: Optional[torch.Tensor] = None, stream=None, check: Optional[bool] = None) -> None:
+    """k_pool[dst] := k_pool[src] (and v) for each row (src, dst) of pairs (int64 [n, 2]).  With
+    ``check`` (default: the PKV_DEBUG environment variable) the pairs are first checked on the host."""
     if pairs.dtype != torch.int64 or (pairs.numel() and pairs.shape[-1] != 2):
         raise TypeError("pairs must be int64 [n, 2]")
+    if check or (check is None and _debug_checks()):
+        check_block_pairs(pairs, k_pool.shape[0], k_pool.shape[0], True)
     block_bytes = k_pool[0].numel() * k_pool.element_size()
     status = lib().pkv_copy_blocks(
         _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"), block_bytes, _dev(pairs, "pairs"),
@@ -251,11 +274,15 @@ def copy_blocks(k_pool: torch.Tensor, v_pool: torch.Tensor, pairs: torch.Tensor,
 
 
 def swap_blocks(src_k: torch.Tensor, src_v: torch.Tensor, dst_k: torch.Tensor, dst_v: torch.Tensor,
-                pairs: torch.Tensor, *, device_error: Optional[torch.Tensor] = None, stream=None) -> None:
+                pairs: torch.Tensor, *, device_error: Optional[torch.Tensor] = None, stream=None,
+                check: Optional[bool] = None) -> None:
     """dst[d] := src[s] (K and V pools [NB, Hkv, B, D], whole blocks) for each row (s, d) of pairs
-    (int64 [n, 2], on the GPU).  Either side may be pinned host memory (``pin_memory()``)."""
+    (int64 [n, 2], on the GPU).  Either side may be pinned host memory (``pin_memory()``).  With
+    ``check`` (default: PKV_DEBUG) the pairs are first checked on the host."""
     if pairs.dtype != torch.int64 or (pairs.numel() and pairs.shape[-1] != 2):
         raise TypeError("pairs must be int64 [n, 2]")
+    if check or (check is None and _debug_checks()):
+        check_block_pairs(pairs, src_k.shape[0], dst_k.shape[0], src_k.data_ptr() == dst_k.data_ptr())
     if src_k.shape[1:] != dst_k.shape[1:] or src_k.dtype != dst_k.dtype or src_v.shape != src_k.shape \
             or dst_v.shape != dst_k.shape:
         raise ValueError("pools of one layout and dtype")

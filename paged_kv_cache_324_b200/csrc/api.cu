@@ -2,7 +2,9 @@
 // the launchers share.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <mutex>
+#include <vector>
 
 #include "pkv_device.cuh"
 #include "pkv_host.h"
@@ -45,6 +47,29 @@ extern "C" const char* pkv_status_string(pkv_status s) {
     case PKV_ERR_OUT_OF_BLOCKS: return "out of free blocks";
     }
     return "unknown status";
+}
+
+// ---- host check of a block-pair list (copy-on-write, swap) ----------------------------
+
+extern "C" pkv_status pkv_check_block_pairs(const int64_t* pairs, int num_pairs, int src_num_blocks,
+                                            int dst_num_blocks, int same_pool) {
+    if (num_pairs < 0 || src_num_blocks <= 0 || dst_num_blocks <= 0) return PKV_ERR_INVALID_ARG;
+    if (num_pairs == 0) return PKV_OK;
+    if (!pairs) return PKV_ERR_INVALID_ARG;
+    std::vector<int64_t> dst(static_cast<size_t>(num_pairs));
+    for (int i = 0; i < num_pairs; ++i) {
+        const int64_t s = pairs[2 * static_cast<size_t>(i)], d = pairs[2 * static_cast<size_t>(i) + 1];
+        if (s < 0 || s >= src_num_blocks || d < 0 || d >= dst_num_blocks) return PKV_ERR_INVALID_ARG;
+        dst[static_cast<size_t>(i)] = d;
+    }
+    std::sort(dst.begin(), dst.end());
+    if (std::adjacent_find(dst.begin(), dst.end()) != dst.end()) return PKV_ERR_INVALID_ARG;
+    if (same_pool) {
+        for (int i = 0; i < num_pairs; ++i)
+            if (std::binary_search(dst.begin(), dst.end(), pairs[2 * static_cast<size_t>(i)]))
+                return PKV_ERR_INVALID_ARG;
+    }
+    return PKV_OK;
 }
 
 // ---- diagnostic: one bounded wait that nothing completes ---------------------------
