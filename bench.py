@@ -853,8 +853,11 @@ class OracleRunner:
         return b
 
 
-def cpu_oracle_sample(w: wl.DecodeWorkload, budget_s: float):
-    """Whole steps of the workload on the oracle until the budget is spent (at least one)."""
+def cpu_oracle_sample(w: wl.DecodeWorkload, budget_s: float, one_core_s: float = 3.0):
+    """Whole steps of the workload on the oracle (all host cores) until the budget is spent (at
+    least one); then, on one core, a step over the first sequences, as many as fit in about
+    ``one_core_s`` after a one-sequence calibration.  Returns (steps, bytes, seconds, cores,
+    (one-core sequences, bytes, seconds))."""
     r = OracleRunner(w)
     n, nbytes, t0 = 0, 0, time.perf_counter()
     while True:
@@ -862,7 +865,17 @@ def cpu_oracle_sample(w: wl.DecodeWorkload, budget_s: float):
         n += 1
         el = time.perf_counter() - t0
         if el >= budget_s:
-            return n, nbytes, el, r.cores
+            break
+    cores, r.cores = r.cores, 1
+    t1 = time.perf_counter()
+    r.step(1)
+    t1 = time.perf_counter() - t1
+    n1 = max(1, min(w.num_seqs, int(one_core_s / max(t1, 1e-6))))
+    t2 = time.perf_counter()
+    b1 = r.step(n1)
+    el1 = time.perf_counter() - t2
+    r.cores = cores
+    return n, nbytes, el, cores, (n1, b1, el1)
 
 
 def main():
@@ -1028,11 +1041,14 @@ def main():
             return
         line, w = run_ours(args, rank, world, local_rank)
         if rank == 0 and world == 1:
-            n, nbytes, el, cores = cpu_oracle_sample(w, args.cpu_budget)
+            n, nbytes, el, cores, (n1, b1, el1) = cpu_oracle_sample(w, args.cpu_budget)
             v = nbytes / el / 1e9
             line["cpu_baseline"] = {"value": round(v, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
                                     "sample": f"{n} whole step(s) of the same workload (scatter + float64 decode "
-                                              f"of all {w.num_seqs} sequences), {el:.1f} s"}
+                                              f"of all {w.num_seqs} sequences), {el:.1f} s",
+                                    "one_core": {"value": round(b1 / el1 / 1e9, 4), "unit": UNIT, "cores": 1,
+                                                 "sample": f"one step over the first {n1} of {w.num_seqs} "
+                                                           f"sequences on one thread, {el1:.1f} s"}}
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

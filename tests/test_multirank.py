@@ -67,3 +67,14 @@ def test_reference_arm_byte_accounting_on_cpu():
     r = bench.OracleRunner(w)
     assert r.step() == wl.step_algorithmic_bytes(w)
     assert 0 < r.step(1) < wl.step_algorithmic_bytes(w)
+
+
+def test_cpu_baseline_sample_reports_a_one_core_figure():
+    """The bench's oracle sample: whole steps on all cores, then a one-thread step over a prefix
+    of the sequences, both with positive byte counts and times."""
+    import bench
+    from paged_kv_cache_324_b200 import workload as wl
+    w = wl.make("tiny")
+    n, nbytes, el, cores, (n1, b1, el1) = bench.cpu_oracle_sample(w, 0.05, one_core_s=0.05)
+    assert n >= 1 and nbytes == n * wl.step_algorithmic_bytes(w) and el > 0 and cores >= 1
+    assert 1 <= n1 <= w.num_seqs and b1 > 0 and el1 > 0
