@@ -395,6 +395,30 @@ def test_scatter_fp8_quantises_each_element():
         np.testing.assert_array_less(np.abs(deq - kf[t]), np.abs(kf[t]) * 2.0 ** -4 + 2.0 ** -10 * float(ks) + 1e-12)
 
 
+@pytest.mark.parametrize("name", ["fp8", "fp8_b32"])
+def test_fp8_cache_error_against_the_unquantised_cache(name):
+    """The E4M3 cache against the same f16 values kept in 16 bits (decode, float64 oracle on
+    both): the quantisation moves the output by well under the FP8 max-abs budget of 3e-2, and by
+    a relative L2 in the range that 3-bit-mantissa rounding of K and V gives (a few per cent:
+    an encoder that kept f16 precision would give ~0, a broken one far more).  Printed as
+    information; the parity tests compare against the oracle on the dequantised cache."""
+    w = wl.make(name, small=True)
+    kq, vq = w.initial_pool("k"), w.initial_pool("v")
+    k16 = np.zeros(kq.shape, np.uint16)
+    v16 = np.zeros(kq.shape, np.uint16)
+    for op in list(w.setup) + [w.step_scatter]:
+        oracle.reshape_and_cache(op.k, op.v, w.src_dtype, kq, vq, "e4m3", op.slots, w.k_scale, w.v_scale)
+        oracle.reshape_and_cache(op.k, op.v, w.src_dtype, k16, v16, "f16", op.slots)
+    a = oracle.paged_attn_decode(w.q, w.q_dtype, kq, vq, "e4m3", w.block_tables, w.context_lens, w.scale,
+                                 w.k_scale, w.v_scale)
+    b = oracle.paged_attn_decode(w.q, w.q_dtype, k16, v16, "f16", w.block_tables, w.context_lens, w.scale)
+    max_abs = float(np.abs(a - b).max())
+    rel_l2 = float(np.linalg.norm(a - b) / np.linalg.norm(b))
+    print(f"{name}: E4M3 vs f16 cache, max-abs {max_abs:.4f}, relative L2 {rel_l2:.4f}")
+    assert max_abs < 3e-2
+    assert 0.01 < rel_l2 < 0.1
+
+
 def test_copy_blocks_copies_only_destinations():
     rng = np.random.default_rng(52)
     kp = wl.garbage_bytes(rng, 10 * 2 * 4 * 8 * 2).view(np.uint16).reshape(10, 2, 4, 8)
