@@ -3,8 +3,10 @@
  * block manager through the glossary "PagedAttention" worked example (section
  * "How paging works": 40 tokens, blocks of 16, free list 41, 7, 19, 2, 33 ->
  * block table 41, 7, 19) and the copy-on-write rule of its section "Sharing
- * blocks across sequences", and checks status strings.  Prints "ok" and exits
- * 0 when every check holds.
+ * blocks across sequences", checks the copy pairs with the host pair check,
+ * caches a prompt's full blocks and shares them with a second request, swaps
+ * both sequences to a second manager, and checks status strings.  Prints "ok"
+ * and exits 0 when every check holds.
  */
 #include <stdio.h>
 #include <stdlib.h>
@@ -54,6 +56,16 @@ int main(void) {
     int64_t child = 1;
     CHECK(pkv_bm_append_slots(m, &child, 1, &slot, pairs, 1, &np) == PKV_OK);
     CHECK(np == 1 && pairs[0] == 19 && pairs[1] == 2);  /* the next free block in FIFO order */
+    CHECK(pkv_check_block_pairs(pairs, np, 64, 64, 1) == PKV_OK);
+    {
+        const int64_t onto_source[4] = {19, 2, 2, 5};      /* block 2 written, then read */
+        const int64_t repeated[4] = {19, 2, 7, 2};
+        const int64_t outside[2] = {19, 64};
+        CHECK(pkv_check_block_pairs(onto_source, 2, 64, 64, 1) == PKV_ERR_INVALID_ARG);
+        CHECK(pkv_check_block_pairs(onto_source, 2, 64, 64, 0) == PKV_OK);
+        CHECK(pkv_check_block_pairs(repeated, 2, 64, 64, 0) == PKV_ERR_INVALID_ARG);
+        CHECK(pkv_check_block_pairs(outside, 1, 64, 64, 0) == PKV_ERR_INVALID_ARG);
+    }
     CHECK(pkv_bm_ref_count(m, 19) == 1 && pkv_bm_ref_count(m, 41) == 2);
     /* the parent is now the only holder of block 19: it writes in place */
     CHECK(pkv_bm_append_slots(m, &id, 1, &slot, pairs, 1, &np) == PKV_OK);
@@ -64,6 +76,39 @@ int main(void) {
     CHECK(pkv_bm_num_free(m) == 64);
     CHECK(pkv_bm_add_sequence(m, 1) == PKV_OK);
     CHECK(pkv_bm_add_sequence(m, 1) == PKV_ERR_INVALID_ARG);
+    CHECK(pkv_bm_free_sequence(m, 1) == PKV_OK);
+
+    /* prefix caching: a 40-token prompt cached, then a second request with the same first 35
+     * tokens shares the two full blocks they cover (32 tokens) */
+    int32_t prompt[40];
+    for (int t = 0; t < 40; ++t) prompt[t] = 1000 + 3 * t;
+    int64_t a = 10, b = 11;
+    CHECK(pkv_bm_add_sequence(m, a) == PKV_OK);
+    for (int t = 0; t < 40; ++t) CHECK(pkv_bm_append_slots(m, &a, 1, &slot, pairs, 1, &np) == PKV_OK);
+    CHECK(pkv_bm_cache_sequence(m, a, prompt, 40) == PKV_OK);
+    CHECK(pkv_bm_num_cached(m) == 2);                /* two full blocks; the partial one is not */
+    int hit = -1;
+    CHECK(pkv_bm_add_sequence_cached(m, b, prompt, 35, &hit) == PKV_OK);
+    CHECK(hit == 32 && pkv_bm_sequence_length(m, b) == 32);
+    int32_t ta[3], tb[3];
+    CHECK(pkv_bm_block_tables(m, &a, 1, ta, 3, -1, NULL) == PKV_OK);
+    CHECK(pkv_bm_block_tables(m, &b, 1, tb, 3, -1, NULL) == PKV_OK);
+    CHECK(ta[0] == tb[0] && ta[1] == tb[1] && tb[2] == -1 && pkv_bm_ref_count(m, ta[0]) == 2);
+
+    /* swap both sequences to a second manager: one destination block per distinct source block */
+    pkv_block_manager* h = pkv_bm_create(16, 16, NULL);
+    CHECK(h != NULL);
+    const int64_t both[2] = {10, 11};
+    int64_t sp[2 * 6];
+    int nsp = 0;
+    CHECK(pkv_bm_swap(m, h, both, 2, sp, 6, &nsp) == PKV_OK);
+    CHECK(nsp == 3);                                 /* a's three blocks; b's two are among them */
+    CHECK(pkv_check_block_pairs(sp, nsp, 64, 16, 0) == PKV_OK);
+    CHECK(pkv_bm_sequence_length(m, a) == -1 && pkv_bm_sequence_length(h, a) == 40);
+    CHECK(pkv_bm_sequence_length(h, b) == 32 && pkv_bm_num_free(h) == 13);
+    CHECK(pkv_bm_block_tables(h, &b, 1, tb, 3, -1, NULL) == PKV_OK);
+    CHECK(pkv_bm_ref_count(h, tb[0]) == 2 && pkv_bm_ref_count(h, tb[1]) == 2);
+    pkv_bm_destroy(h);
     pkv_bm_destroy(m);
     printf("ok\n");
     return 0;
