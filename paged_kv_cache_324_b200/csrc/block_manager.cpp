@@ -137,6 +137,12 @@ struct pkv_block_manager {
         x ^= x >> 33;
         return x;
     }
+    // A cached block b holds exactly these tokens and follows block prev (-1: the first block)
+    // of the same generation.
+    bool confirms(int32_t b, int32_t prev, const int32_t* toks) const {
+        return parent_of[b] == prev && (prev < 0 || parent_gen_of[b] == gen[prev]) &&
+               std::memcmp(tokens_of[b].data(), toks, sizeof(int32_t) * block_size) == 0;
+    }
     uint64_t block_hash(uint64_t parent, const int32_t* toks) const {
         uint64_t h = mix(parent ^ 0x9e3779b97f4a7c15ull);
         for (int i = 0; i < block_size; ++i) h = mix(h ^ (static_cast<uint64_t>(static_cast<uint32_t>(toks[i])) +
@@ -315,9 +321,7 @@ extern "C" pkv_status pkv_bm_add_sequence_cached(pkv_block_manager* m, int64_t s
         auto it = m->cache.find(h);
         if (it == m->cache.end()) break;
         const int32_t b = it->second;
-        if (m->parent_of[b] != prev || (prev >= 0 && m->parent_gen_of[b] != m->gen[prev]) ||
-            std::memcmp(m->tokens_of[b].data(), toks, sizeof(int32_t) * B) != 0)
-            break;                                             // hash collision or stale entry: stop
+        if (!m->confirms(b, prev, toks)) break;                // hash collision or stale entry: stop
         s.blocks.push_back(b);
         prev = b;
     }
@@ -343,8 +347,13 @@ extern "C" pkv_status pkv_bm_cache_sequence(pkv_block_manager* m, int64_t seq_id
         const int32_t b = s.blocks[j];
         h = m->block_hash(h, toks);
         if (!m->cached[b]) {
-            if (m->cache.count(h)) {   // the same content already cached in another block: keep that one
-                prev = b;
+            auto hit = m->cache.find(h);
+            if (hit != m->cache.end()) {
+                // The same prefix already cached in another block: keep that one and chain the
+                // following blocks on it, so that a lookup walking the cached chain reaches them.
+                // A colliding hash whose block holds another prefix ends the registration.
+                if (!m->confirms(hit->second, prev, toks)) break;
+                prev = hit->second;
                 continue;
             }
             m->cache.emplace(h, b);

@@ -228,6 +228,24 @@ def test_idle_cached_blocks_are_reused_then_evicted_oldest_first(BM):
     assert m.add_sequence_cached(4, [1, 2, 3, 4, 0]) == 0     # its first block was evicted: no hit
 
 
+def test_blocks_after_a_duplicate_prefix_block_stay_reachable(BM):
+    """Two sequences prefilled with the same first block in different physical blocks: the second
+    one's later blocks are chained on the block already cached for that content, so a request
+    with the second sequence's prompt hits all of its full blocks."""
+    m = BM(16, 2)
+    x, y = [1, 2, 3, 4], [1, 2, 7, 8]
+    m.add_sequence(0)
+    _fill(m, 0, 4)
+    m.cache_sequence(0, x)
+    m.add_sequence(1)
+    _fill(m, 1, 4)                                            # its own copy of tokens 1, 2
+    m.cache_sequence(1, y)
+    assert m.num_cached == 3                                  # [1,2] once, [3,4] and [7,8]
+    assert m.add_sequence_cached(2, y + [9]) == 4
+    t, _ = m.block_tables([0, 1, 2], 3)
+    assert t[2, 0] == t[0, 0] and t[2, 1] == t[1, 1]
+
+
 def test_stale_child_of_a_recycled_block_does_not_match(BM):
     m = BM(4, 2, np.arange(4))
     m.add_sequence(0)
@@ -377,7 +395,9 @@ class _ModelManager:
         for j in range(len(toks) // self.bs):
             b = blocks[j]
             key = (tuple(toks[j * self.bs:(j + 1) * self.bs]), prev, prev_gen)
-            if b not in self.key_of and key not in self.cache:
+            if b not in self.key_of and key in self.cache:
+                b = self.cache[key]               # the same prefix is cached in another block
+            elif b not in self.key_of:
                 self.key_of[b] = key
                 self.cache[key] = b
             prev, prev_gen = b, self.gen[b]
