@@ -309,6 +309,7 @@ pkv_status pkv_paged_attn_prefill_fp8(void* out, const void* q, pkv_dtype q_dtyp
  *   k, v           [num_tokens][num_kv_heads][head_dim], in_dtype in {F16, BF16}, 16-byte aligned
  *   slot_mapping   int64 [num_tokens]
  *   head_dim       a multiple of 8
+ *   k_scale, v_scale   E4M3 pools only: positive and finite (else PKV_ERR_INVALID_ARG)
  */
 pkv_status pkv_reshape_and_cache(const void* k, const void* v, pkv_dtype in_dtype,
                                  void* k_pool, void* v_pool, pkv_dtype kv_dtype,

@@ -13,6 +13,8 @@
 // vectors of a token's row so loads and stores coalesce, and the grid is a
 // multiple of the SM count with a grid-stride loop.
 
+#include <cmath>
+
 #include <cuda_runtime.h>
 
 #include "pkv_device.cuh"
@@ -130,7 +132,9 @@ extern "C" pkv_status pkv_reshape_and_cache(const void* k, const void* v, pkv_dt
     if (head_dim % 8 != 0) return PKV_ERR_UNSUPPORTED;
     if (num_tokens == 0) return PKV_OK;
     if (!k || !v || !k_pool || !v_pool || !slot_mapping) return PKV_ERR_INVALID_ARG;
-    if (kv_dtype == PKV_FP8_E4M3 && !(k_scale > 0.f && v_scale > 0.f)) return PKV_ERR_INVALID_ARG;
+    if (kv_dtype == PKV_FP8_E4M3 &&
+        !(k_scale > 0.f && v_scale > 0.f && std::isfinite(k_scale) && std::isfinite(v_scale)))
+        return PKV_ERR_INVALID_ARG;
     if (!aligned16(k) || !aligned16(v) || !aligned16(k_pool) || !aligned16(v_pool) ||
         (reinterpret_cast<uintptr_t>(slot_mapping) & 7))
         return PKV_ERR_ALIGNMENT;

@@ -110,6 +110,9 @@ def test_reshape_and_copy_reject_bad_arguments(lib):
                                      None, None) == 2   # head_dim not a multiple of 8
     assert lib.pkv_reshape_and_cache(P(16), P(16), 0, P(16), P(16), 0, 1.0, 1.0, P(16), 0, 2, 128, 16, 10,
                                      None, None) == 0   # nothing to do
+    for ks, vs in ((0.0, 1.0), (1.0, -1.0), (float("inf"), 1.0), (1.0, float("nan"))):
+        assert lib.pkv_reshape_and_cache(P(16), P(16), 0, P(16), P(16), 2, ks, vs, P(16), 4, 2, 128, 16, 10,
+                                         None, None) == 1   # E4M3 scales must be positive and finite
     assert lib.pkv_copy_blocks(P(16), P(16), 24, P(16), 3, 10, None, None) == 2
     assert lib.pkv_copy_blocks(P(16), P(16), 32, P(16), -1, 10, None, None) == 1
     assert lib.pkv_copy_blocks(P(16), P(16), 32, P(16), 0, 10, None, None) == 0
