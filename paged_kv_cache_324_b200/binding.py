@@ -95,6 +95,26 @@ def _dev(t: Optional[torch.Tensor], name: str):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _err(t: Optional[torch.Tensor]):
+    """The device error word: a 4-byte integer tensor on the GPU (element 0 is used), or None."""
+    if t is None:
+        return None
+    if t.element_size() != 4 or t.dtype.is_floating_point or t.numel() < 1:
+        raise TypeError("device_error must be an int32 tensor with at least one element")
+    return _dev(t, "device_error")
+
+
+def _tables(block_tables: torch.Tensor, context_lens: torch.Tensor, num_seqs: int):
+    """Block tables int32 [>= num_seqs, max_blocks] and context lengths int32 [>= num_seqs]: the
+    kernels read num_seqs rows of each."""
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    if block_tables.dim() != 2 or block_tables.shape[0] < num_seqs or block_tables.shape[1] < 1:
+        raise ValueError("block_tables must be [num_seqs, max_blocks]")
+    if context_lens.numel() < num_seqs:
+        raise ValueError("context_lens must hold num_seqs lengths")
+
+
 def _stream(stream) -> ctypes.c_void_p:
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -142,8 +162,7 @@ def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_pool: torch.Tensor, 
     NB, Hkv, B, D2 = k_pool.shape
     if out.shape != q.shape or out.dtype != q.dtype or D2 != D or v_pool.shape != k_pool.shape:
         raise ValueError("inconsistent shapes or dtypes")
-    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
-        raise TypeError("block_tables and context_lens must be int32")
+    _tables(block_tables, context_lens, S)
     need = decode_workspace_bytes(S, H, Hkv, D, k_pool.dtype, B, max_context_len, partition_size)
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
@@ -153,7 +172,7 @@ def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_pool: torch.Tensor, 
         _code(k_pool), float(k_scale), float(v_scale), _dev(block_tables, "block_tables"),
         block_tables.shape[1], _dev(context_lens, "context_lens"), int(max_context_len), S, H, Hkv, D, B,
         NB, float(scale), int(partition_size), _dev(workspace, "workspace"), ws_bytes,
-        _dev(device_error, "device_error"), _stream(stream))
+        _err(device_error), _stream(stream))
     _check(status, "paged_attn_decode")
     return out
 
@@ -175,15 +194,16 @@ def paged_attn_prefill(out: torch.Tensor, q: torch.Tensor, k_pool: torch.Tensor,
         raise ValueError("inconsistent shapes or dtypes")
     if k_pool.dtype != q.dtype or v_pool.dtype != q.dtype:
         raise TypeError("prefill needs q and the pools in one 16-bit dtype")
-    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32 or query_start.dtype != torch.int32:
-        raise TypeError("block_tables, context_lens and query_start must be int32")
+    _tables(block_tables, context_lens, S)
+    if query_start.dtype != torch.int32:
+        raise TypeError("query_start must be int32")
     if query_start.numel() != S + 1:
         raise ValueError("query_start must hold num_seqs + 1 offsets")
     status = lib().pkv_paged_attn_prefill(
         _dev(out, "out"), _dev(q, "q"), _code(q), _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"),
         _dev(block_tables, "block_tables"), block_tables.shape[1], _dev(context_lens, "context_lens"),
         _dev(query_start, "query_start"), int(max_query_len), S, T, H, Hkv, D, B, NB, float(scale),
-        _dev(device_error, "device_error"), _stream(stream))
+        _err(device_error), _stream(stream))
     _check(status, "paged_attn_prefill")
     return out
 
@@ -207,8 +227,13 @@ def paged_attn_prefill_fp8(out: torch.Tensor, q: torch.Tensor, k_pool: torch.Ten
         raise ValueError("inconsistent shapes or dtypes")
     if k_pool.dtype != torch.uint8 or v_pool.dtype != torch.uint8:
         raise TypeError("the pools hold E4M3 bytes (uint8)")
-    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32 or query_start.dtype != torch.int32:
-        raise TypeError("block_tables, context_lens and query_start must be int32")
+    _tables(block_tables, context_lens, S)
+    if query_start.dtype != torch.int32:
+        raise TypeError("query_start must be int32")
+    if query_start.numel() != S + 1:
+        raise ValueError("query_start must hold num_seqs + 1 offsets")
+    if q.dtype not in (torch.float16, torch.bfloat16):
+        raise TypeError("q and out must be float16 or bfloat16")
     need = prefill_fp8_workspace_bytes(S, block_tables.shape[1], Hkv, D, B)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
@@ -216,7 +241,7 @@ def paged_attn_prefill_fp8(out: torch.Tensor, q: torch.Tensor, k_pool: torch.Ten
         _dev(out, "out"), _dev(q, "q"), _code(q), _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"), float(k_scale),
         float(v_scale), _dev(block_tables, "block_tables"), block_tables.shape[1], _dev(context_lens, "context_lens"),
         _dev(query_start, "query_start"), int(max_query_len), S, T, H, Hkv, D, B, NB, float(scale),
-        _dev(workspace, "workspace"), workspace.numel(), _dev(device_error, "device_error"), _stream(stream))
+        _dev(workspace, "workspace"), workspace.numel(), _err(device_error), _stream(stream))
     _check(status, "paged_attn_prefill_fp8")
     return out
 
@@ -234,7 +259,7 @@ def reshape_and_cache(k: torch.Tensor, v: torch.Tensor, k_pool: torch.Tensor, v_
     status = lib().pkv_reshape_and_cache(
         _dev(k, "k"), _dev(v, "v"), _code(k), _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"),
         _code(k_pool), float(k_scale), float(v_scale), _dev(slot_mapping, "slot_mapping"), T, Hkv, D, B, NB,
-        _dev(device_error, "device_error"), _stream(stream))
+        _err(device_error), _stream(stream))
     _check(status, "reshape_and_cache")
 
 
@@ -269,7 +294,7 @@ def copy_blocks(k_pool: torch.Tensor, v_pool: torch.Tensor, pairs: torch.Tensor,
     block_bytes = k_pool[0].numel() * k_pool.element_size()
     status = lib().pkv_copy_blocks(
         _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"), block_bytes, _dev(pairs, "pairs"),
-        pairs.numel() // 2, k_pool.shape[0], _dev(device_error, "device_error"), _stream(stream))
+        pairs.numel() // 2, k_pool.shape[0], _err(device_error), _stream(stream))
     _check(status, "copy_blocks")
 
 
@@ -295,13 +320,13 @@ def swap_blocks(src_k: torch.Tensor, src_v: torch.Tensor, dst_k: torch.Tensor, d
     status = lib().pkv_swap_blocks(
         ctypes.c_void_p(src_k.data_ptr()), ctypes.c_void_p(src_v.data_ptr()), src_k.shape[0],
         ctypes.c_void_p(dst_k.data_ptr()), ctypes.c_void_p(dst_v.data_ptr()), dst_k.shape[0], block_bytes,
-        _dev(pairs, "pairs"), pairs.numel() // 2, _dev(device_error, "device_error"), _stream(stream))
+        _dev(pairs, "pairs"), pairs.numel() // 2, _err(device_error), _stream(stream))
     _check(status, "swap_blocks")
 
 
 def selftest_bounded_wait(device_error: torch.Tensor, timeout_us: int, stream=None) -> None:
     """Run one bounded wait that nothing completes; it sets DEVERR_TIMEOUT in device_error."""
-    _check(lib().pkv_selftest_bounded_wait(_dev(device_error, "device_error"), int(timeout_us), _stream(stream)),
+    _check(lib().pkv_selftest_bounded_wait(_err(device_error), int(timeout_us), _stream(stream)),
            "selftest_bounded_wait")
 
 
@@ -466,7 +491,15 @@ def paged_attn_decode_shared_prefix(out, q, k_pool, v_pool, block_tables, contex
     L.pkv_paged_attn_decode_shared_prefix.argtypes = [P, P, I, P, P, I, F, F, P, I, P, I, I, I, I, I, I, I, F, I,
                                                       P, P, P, I, I, I, P, Z, P, P]
     S, H, D = q.shape
-    NB, Hkv, B, _ = k_pool.shape
+    NB, Hkv, B, D2 = k_pool.shape
+    if out.shape != q.shape or out.dtype != q.dtype or D2 != D or v_pool.shape != k_pool.shape:
+        raise ValueError("inconsistent shapes or dtypes")
+    _tables(block_tables, context_lens, S)
+    for t, name in ((seq_prefix_len, "seq_prefix_len"), (unit_seqs, "unit_seqs"), (unit_len, "unit_len")):
+        if t.dtype != torch.int32:
+            raise TypeError(f"{name} must be int32")
+    if seq_prefix_len.numel() < S:
+        raise ValueError("seq_prefix_len must hold num_seqs entries")
     need = shared_prefix_workspace_bytes(S, H, Hkv, D, k_pool.dtype, B, max_context_len, unit_len.numel(),
                                          max_prefix_len, partition_size)
     if workspace is None:
@@ -479,7 +512,7 @@ def paged_attn_decode_shared_prefix(out, q, k_pool, v_pool, block_tables, contex
         _dev(context_lens, "context_lens"), int(max_context_len), S, H, Hkv, D, B, NB, float(scale),
         int(partition_size), _dev(seq_prefix_len, "seq_prefix_len"),
         _dev(unit_seqs, "unit_seqs") if U else None, _dev(unit_len, "unit_len") if U else None, U, W,
-        int(max_prefix_len), _dev(workspace, "workspace"), workspace.numel(), _dev(device_error, "device_error"),
+        int(max_prefix_len), _dev(workspace, "workspace"), workspace.numel(), _err(device_error),
         _stream(stream))
     _check(status, "paged_attn_decode_shared_prefix")
     return out
