@@ -1,0 +1,51 @@
+"""bench.py's command line and JSON contract, on CPU.
+
+The reference arm (the float64 oracle on the host's cores) runs here on the small
+decode workload and must print one JSON line with the contract's keys; fewer
+than three warm-up steps are refused; and the product arm, which has no CPU
+fallback, must fail without printing a result when no GPU is present.
+"""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def run_bench(*args, timeout=240):
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], capture_output=True, text=True,
+                          cwd=ROOT, timeout=timeout)
+
+
+def test_reference_arm_prints_one_contract_line():
+    r = run_bench("--impl", "reference", "--config", "tiny", "--steps", "2", "--warmup", "3")
+    assert r.returncode == 0, r.stderr
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["steps"] == 2 and d["warmup"] == 3 and d["n_gpus"] == 1
+    assert d["value"] > 0 and d["higher_is_better"] is True and d["scaling"] == "weak"
+    assert d["vs_baseline"] is None and d["config"]["name"] == "tiny" and "workload" in d["config"]
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_fewer_than_three_warmup_steps_are_refused():
+    r = run_bench("--impl", "reference", "--config", "tiny", "--steps", "1", "--warmup", "2")
+    assert r.returncode != 0 and not r.stdout.strip()
+    assert "warmup" in r.stderr
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the behaviour without a GPU")
+def test_product_arm_fails_loudly_without_a_gpu():
+    r = run_bench("--steps", "1", "--warmup", "3")
+    assert r.returncode != 0
+    assert not r.stdout.strip()                      # no result line from any fallback
