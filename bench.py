@@ -1041,7 +1041,8 @@ def main():
             return
         line, w = run_ours(args, rank, world, local_rank)
         if rank == 0 and world == 1:
-            n, nbytes, el, cores, (n1, b1, el1) = cpu_oracle_sample(w, args.cpu_budget)
+            n, nbytes, el, cores, (n1, b1, el1) = cpu_oracle_sample(w, args.cpu_budget,
+                                                                     one_core_s=min(3.0, args.cpu_budget))
             v = nbytes / el / 1e9
             line["cpu_baseline"] = {"value": round(v, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
                                     "sample": f"{n} whole step(s) of the same workload (scatter + float64 decode "
