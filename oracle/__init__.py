@@ -77,6 +77,12 @@ def _load():
     return _lib
 
 
+def _threads(n) -> int:
+    """OpenMP threads for one call: n, or every host core when n is 0 (so that an earlier call's
+    count does not carry over)."""
+    return int(n) if n else (os.cpu_count() or 1)
+
+
 def _ptr(a: np.ndarray):
     assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
     return a.ctypes.data_as(ctypes.c_void_p)
@@ -128,7 +134,7 @@ def paged_attn_decode(q_bits, q_dtype, k_pool, v_pool, kv_dtype, block_tables, c
     _check(_load().orc_paged_attn_decode(
         _ptr(out), _ptr(q_bits), _code(q_dtype), _ptr(k_pool), _ptr(v_pool), _code(kv_dtype),
         float(k_scale), float(v_scale), _ptr(block_tables), block_tables.shape[1],
-        _ptr(context_lens), S, H, Hkv, D, B, NB, float(scale), int(threads)))
+        _ptr(context_lens), S, H, Hkv, D, B, NB, float(scale), _threads(threads)))
     return out
 
 
@@ -157,7 +163,7 @@ def paged_attn_prefill(q_bits, q_dtype, k_pool, v_pool, kv_dtype, block_tables, 
     _check(_load().orc_paged_attn_prefill(
         _ptr(out), _ptr(q_bits), _code(q_dtype), _ptr(k_pool), _ptr(v_pool), _code(kv_dtype),
         float(k_scale), float(v_scale), _ptr(block_tables), block_tables.shape[1],
-        _ptr(context_lens), _ptr(query_start), S, H, Hkv, D, B, NB, float(scale), int(threads)))
+        _ptr(context_lens), _ptr(query_start), S, H, Hkv, D, B, NB, float(scale), _threads(threads)))
     return out
 
 

@@ -49,3 +49,27 @@ def test_product_arm_fails_loudly_without_a_gpu():
     r = run_bench("--steps", "1", "--warmup", "3")
     assert r.returncode != 0
     assert not r.stdout.strip()                      # no result line from any fallback
+
+
+@pytest.mark.parametrize("config", ["tiny", "prefill", "prefill_fp8"])
+def test_product_arm_adds_the_cpu_baseline(config, monkeypatch, capsys):
+    """main()'s product arm after the GPU timing, with the timing replaced by a stub returning a
+    fixed line on the small workload: the cpu_baseline the oracle adds is complete."""
+    import bench
+    from paged_kv_cache_324_b200 import workload as wl
+    stub = {"metric": "m", "value": 1.0, "unit": "u"}
+    if config == "tiny":
+        monkeypatch.setattr(bench, "run_ours", lambda *a: (dict(stub), wl.make("tiny")))
+    else:
+        monkeypatch.setattr(bench, "run_prefill", lambda *a: (dict(stub), wl.make_prefill(small=True)))
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--config", config, "--steps", "1", "--warmup", "3",
+                                      "--cpu-budget", "0.05"])
+    for var in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        monkeypatch.delenv(var, raising=False)
+    bench.main()
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    cb = json.loads(lines[0])["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["cores"] >= 1 and cb["sample"]
+    if config == "tiny":
+        assert cb["one_core"]["cores"] == 1 and cb["one_core"]["value"] > 0
