@@ -127,3 +127,24 @@ def oracle_prefill_pools(w):
             oracle.reshape_and_cache(op.k, op.v, w.dtype, kp, vp, w.dtype, op.slots)
             vmax = max(vmax, float(np.abs(oracle.decode_values(op.v, w.dtype)).max()))
     return kp, vp, vmax
+
+
+class Guarded:
+    """A buffer with guard bytes on both sides, to catch writes just outside it: the tensor
+    ``t`` (shape, dtype) sits between two GUARD-byte runs of PATTERN inside one allocation.
+    GUARD is a multiple of 256, so ``t`` keeps the allocation's alignment."""
+    GUARD = 4096
+    PATTERN = 0xA5
+
+    def __init__(self, shape, dtype, dev, init=None):
+        shape = tuple(int(x) for x in shape)
+        n = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
+        self.n = n
+        self.raw = torch.full((self.GUARD + n + self.GUARD,), self.PATTERN, dtype=torch.uint8, device=dev)
+        self.t = self.raw[self.GUARD:self.GUARD + n].view(dtype).view(shape)
+        if init is not None:
+            self.t.copy_(init)
+
+    def intact(self) -> bool:
+        g = self.GUARD
+        return bool((self.raw[:g] == self.PATTERN).all()) and bool((self.raw[g + self.n:] == self.PATTERN).all())
