@@ -397,6 +397,14 @@ pkv_status pkv_bm_fork(pkv_block_manager* m, int64_t parent, int64_t child);
  * list is too short (nothing changes: the caller may free or preempt and retry). */
 pkv_status pkv_bm_append_slots(pkv_block_manager* m, const int64_t* seq_ids, int n, int64_t* slots,
                                int64_t* pairs, int max_pairs, int* num_pairs);
+/* Append n tokens to one sequence (a prefill chunk): slots[0..n) receive the
+ * tokens' slots in order; a shared partially filled last block is copied once
+ * before the first write (one (src, dst) pair, *num_pairs = 1, else 0), and the
+ * tokens beyond it take new blocks.  The same result as n calls of
+ * pkv_bm_append_slots for this sequence alone.  PKV_ERR_OUT_OF_BLOCKS if the
+ * free list is too short (nothing changes). */
+pkv_status pkv_bm_append_tokens(pkv_block_manager* m, int64_t seq_id, int n, int64_t* slots,
+                                int64_t* pairs, int max_pairs, int* num_pairs);
 /* Drop a sequence; its blocks' reference counts fall, unreferenced blocks return. */
 pkv_status pkv_bm_free_sequence(pkv_block_manager* m, int64_t seq_id);
 /* Rows of int32 [n][max_blocks] block tables (entries past a sequence's last block

@@ -395,6 +395,20 @@ class BlockManager:
                  "append_slots")
         return slots, pairs[:k.value].copy()
 
+    def append_tokens(self, seq_id: int, n: int):
+        """n new tokens for one sequence (a prefill chunk): (slots int64 [n], copy pairs int64 [k, 2])."""
+        np = self._np
+        slots = np.empty(max(int(n), 1), np.int64)
+        pairs = np.empty((1, 2), np.int64)
+        k = ctypes.c_int(0)
+        P = ctypes.c_void_p
+        f = self._L.pkv_bm_append_tokens
+        f.argtypes = [P, ctypes.c_int64, ctypes.c_int, P, P, ctypes.c_int, P]
+        f.restype = ctypes.c_int
+        self._ok(f(self._h, seq_id, int(n), slots.ctypes.data_as(P), pairs.ctypes.data_as(P), 1, ctypes.byref(k)),
+                 "append_tokens")
+        return slots[:int(n)].copy(), pairs[:k.value].copy()
+
     def free_sequence(self, seq_id: int):
         self._ok(self._L.pkv_bm_free_sequence(self._h, seq_id), "free_sequence")
 

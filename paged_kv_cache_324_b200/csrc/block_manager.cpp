@@ -260,6 +260,44 @@ extern "C" pkv_status pkv_bm_append_slots(pkv_block_manager* m, const int64_t* s
     return PKV_OK;
 }
 
+extern "C" pkv_status pkv_bm_append_tokens(pkv_block_manager* m, int64_t seq_id, int n, int64_t* slots,
+                                           int64_t* pairs, int max_pairs, int* num_pairs) {
+    if (!m || n < 0 || (n > 0 && !slots) || !num_pairs || max_pairs < 0 || (max_pairs > 0 && !pairs))
+        return PKV_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> g(m->mu);
+    auto it = m->seqs.find(seq_id);
+    if (it == m->seqs.end()) return PKV_ERR_INVALID_ARG;
+    auto& s = it->second;
+    const int64_t B = m->block_size;
+    const int64_t off = s.len % B;
+    // a shared partial last block is copied once, before the first write; the tokens that do
+    // not fit in the last block take ceil(rest / B) new blocks
+    const bool copy = n > 0 && off != 0 && m->ref[s.blocks.back()] > 1;
+    const int64_t room = off == 0 ? 0 : B - off;
+    const int64_t rest = n > room ? n - room : 0;
+    const size_t need = static_cast<size_t>((rest + B - 1) / B) + (copy ? 1 : 0);
+    if (need > m->available()) return PKV_ERR_OUT_OF_BLOCKS;
+    if (copy && max_pairs < 1) return PKV_ERR_INVALID_ARG;
+    int np = 0;
+    if (copy) {
+        const int32_t last = s.blocks.back();
+        const int32_t fresh = m->take();
+        pairs[0] = last;
+        pairs[1] = fresh;
+        np = 1;
+        --m->ref[last];
+        s.blocks.back() = fresh;
+    }
+    for (int i = 0; i < n; ++i) {
+        const int64_t o = s.len % B;
+        if (o == 0) s.blocks.push_back(m->take());
+        slots[i] = static_cast<int64_t>(s.blocks.back()) * B + o;
+        ++s.len;
+    }
+    *num_pairs = np;
+    return PKV_OK;
+}
+
 extern "C" pkv_status pkv_bm_free_sequence(pkv_block_manager* m, int64_t seq_id) {
     if (!m) return PKV_ERR_INVALID_ARG;
     std::lock_guard<std::mutex> g(m->mu);

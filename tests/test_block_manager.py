@@ -470,3 +470,58 @@ def test_randomized_against_a_python_model(BM):
     for i, s in enumerate(live):
         blocks, L = py.seqs[s]
         assert tabs[i, :len(blocks)].tolist() == blocks and lens[i] == L
+
+
+def test_append_tokens_equals_repeated_single_appends(BM):
+    """A chunk append gives the same slots, copy pairs, tables and free counts as one
+    single-token append per token, on twin managers driven through random forks and chunks."""
+    rng = np.random.default_rng(23)
+    for B in (1, 4, 16):
+        NB = 400
+        order = rng.permutation(NB).tolist()
+        a, b = BM(NB, B, order), BM(NB, B, order)
+        live = []
+        for step in range(150):
+            r = rng.random()
+            if r < 0.15 or not live:
+                sid = 1000 * B + step
+                a.add_sequence(sid)
+                b.add_sequence(sid)
+                live.append(sid)
+            elif r < 0.35:
+                sid, child = int(rng.choice(live)), 1000 * B + step
+                a.fork(sid, child)
+                b.fork(sid, child)
+                live.append(child)
+            else:
+                sid, n = int(rng.choice(live)), int(rng.integers(0, 3 * B + 2))
+                try:
+                    got_slots, got_pairs = a.append_tokens(sid, n)
+                except Exception:
+                    assert a.num_free < n // B + 2      # only for want of blocks
+                    continue
+                want_slots, want_pairs = [], []
+                for _ in range(n):
+                    s1, p1 = b.append_slots([sid])
+                    want_slots.append(int(s1[0]))
+                    want_pairs += [tuple(x) for x in p1.tolist()]
+                assert got_slots.tolist() == want_slots
+                assert [tuple(x) for x in got_pairs.tolist()] == want_pairs and len(want_pairs) <= 1
+            assert a.num_free == b.num_free
+        ta, la = a.block_tables(live, 64)
+        tb, lb = b.block_tables(live, 64)
+        assert np.array_equal(ta, tb) and np.array_equal(la, lb)
+
+
+def test_append_tokens_is_all_or_nothing(BM):
+    from paged_kv_cache_324_b200.binding import PagedKVError
+    m = BM(4, 4)
+    m.add_sequence(0)
+    m.append_tokens(0, 6)                              # blocks 0, 1 (two slots left)
+    m.fork(0, 1)
+    with pytest.raises(PagedKVError):
+        m.append_tokens(1, 11)                         # a copy + 2 new blocks > 2 free
+    assert m.num_free == 2 and m.sequence_length(1) == 6
+    slots, pairs = m.append_tokens(1, 2)               # the copy of the shared partial block
+    assert len(pairs) == 1 and m.num_free == 1 and m.sequence_length(1) == 8
+    assert m.append_tokens(0, 0)[0].size == 0 and m.sequence_length(0) == 6
