@@ -207,9 +207,11 @@ class DeviceStep:
         assert int(self.err.item()) == 0, "setup raised a device error"
 
     def launches_per_step(self) -> int:
-        if self.prefix_aware:   # prefix pass (if any unit), own-token pass, merge
+        """Library kernels one step launches: [copy_blocks] + reshape_and_cache + the decode call
+        (shared-prefix: [prefix pass] + tail pass + merge; plain: pass 1 + [merge when split])."""
+        if self.prefix_aware:
             return ("pairs" in self.d) + 1 + (self.sp["units"] > 0) + 2
-        return ("pairs" in self.d) + 1 + 1 + int(self.w.max_context_len > self.partition) + int(self.split)
+        return ("pairs" in self.d) + 1 + 1 + int(self.split)
 
     def copy_op(self):
         if "pairs" in self.d:
