@@ -21,18 +21,22 @@
  * and the prefill of a chunk of new tokens over the same cache
  * (pkv_paged_attn_prefill: every query of the chunk attends causally, the
  * dense phase of the "vLLM and PagedAttention" transcript's opening
- * paragraph), on the 5th-generation tensor cores.  Around them: a decode
- * that reads shared prompt blocks once per group of sequences
+ * paragraph), on the 5th-generation tensor cores, also over an E4M3 cache
+ * (pkv_paged_attn_prefill_fp8).  Around them: a decode that reads shared
+ * prompt blocks once per group of sequences
  * (pkv_paged_attn_decode_shared_prefix), block swapping between the device
- * pool and pinned host memory (pkv_swap_blocks), and a host-side block
- * manager with copy-on-write, prefix caching by block content and swap
- * bookkeeping (pkv_bm_*).
+ * pool and pinned host memory (pkv_swap_blocks), a host-side block manager
+ * with copy-on-write, chunk appends, prefix caching by block content and
+ * swap bookkeeping (pkv_bm_*), and a host check of copy and swap pair lists
+ * (pkv_check_block_pairs).
  *
  * Conventions shared by every entry point
  *   - All pointers except scalars are DEVICE pointers, owned by the caller
  *     (exceptions, stated where they apply: the block manager's arrays are
  *     host memory; pkv_swap_blocks also takes pinned, mapped host pools).
- *     The library allocates nothing and keeps no per-call state; calls are
+ *     The GPU calls allocate nothing (the one exception,
+ *     pkv_paged_attn_decode_static_ws, uses a file-scope device array of
+ *     the library) and keep no state between calls; calls are
  *     asynchronous on `stream` (a cudaStream_t passed as void*, NULL = the
  *     legacy default stream) and nothing synchronises.
  *   - Pools have layout [num_blocks][num_kv_heads][block_size][head_dim],
