@@ -73,3 +73,17 @@ def test_product_arm_adds_the_cpu_baseline(config, monkeypatch, capsys):
     assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["cores"] >= 1 and cb["sample"]
     if config == "tiny":
         assert cb["one_core"]["cores"] == 1 and cb["one_core"]["value"] > 0
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    """Under two ranks the reference arm prints one line from rank 0; rank 1 exits at once."""
+    outs = []
+    for rank in (0, 1):
+        env = dict(os.environ, RANK=str(rank), WORLD_SIZE="2", LOCAL_RANK=str(rank))
+        r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "tiny",
+                            "--gpus", "2", "--steps", "1", "--warmup", "3"], capture_output=True, text=True,
+                           cwd=ROOT, env=env, timeout=240)
+        assert r.returncode == 0, r.stderr
+        outs.append([ln for ln in r.stdout.splitlines() if ln.strip()])
+    assert len(outs[0]) == 1 and json.loads(outs[0][0])["n_gpus"] == 2
+    assert outs[1] == []
