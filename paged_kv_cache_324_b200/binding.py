@@ -353,10 +353,14 @@ class BlockManager:
         L.pkv_bm_add_sequence_cached.argtypes = [P, I64, P, I, P]
         L.pkv_bm_cache_sequence.argtypes = [P, I64, P, I]
         L.pkv_bm_swap.argtypes = [P, P, P, I, P, I, P]
+        L.pkv_bm_append_tokens.argtypes = [P, I64, I, P, P, I, P]
+        L.pkv_bm_append_tokens.restype = I
         self._L, self._np = L, np
         order = None
         if free_order is not None:
-            order = np.ascontiguousarray(free_order, dtype=np.int32)
+            order = np.ascontiguousarray(free_order, dtype=np.int32).reshape(-1)
+            if order.size != num_blocks:            # the library reads num_blocks entries
+                raise ValueError("free_order must hold num_blocks entries")
         self.block_size = block_size
         self._h = L.pkv_bm_create(num_blocks, block_size,
                                   order.ctypes.data_as(P) if order is not None else None)
@@ -402,11 +406,8 @@ class BlockManager:
         pairs = np.empty((1, 2), np.int64)
         k = ctypes.c_int(0)
         P = ctypes.c_void_p
-        f = self._L.pkv_bm_append_tokens
-        f.argtypes = [P, ctypes.c_int64, ctypes.c_int, P, P, ctypes.c_int, P]
-        f.restype = ctypes.c_int
-        self._ok(f(self._h, seq_id, int(n), slots.ctypes.data_as(P), pairs.ctypes.data_as(P), 1, ctypes.byref(k)),
-                 "append_tokens")
+        self._ok(self._L.pkv_bm_append_tokens(self._h, seq_id, int(n), slots.ctypes.data_as(P),
+                                              pairs.ctypes.data_as(P), 1, ctypes.byref(k)), "append_tokens")
         return slots[:int(n)].copy(), pairs[:k.value].copy()
 
     def free_sequence(self, seq_id: int):

@@ -150,6 +150,14 @@ def test_matches_the_harness_allocator(BM):
         assert tabs[i, :len(py_tables[s])].tolist() == py_tables[s] and L[i] == lens[s]
 
 
+def test_free_order_must_cover_the_pool(BM):
+    with pytest.raises(ValueError):
+        BM(8, 4, [0, 1, 2])                              # shorter than the pool: refused before the library
+    with pytest.raises(ValueError):
+        BM(4, 4, [0, 1, 1, 2])                           # not a permutation: refused by the library
+    assert BM(4, 4, [3, 1, 0, 2]).num_free == 4
+
+
 def test_bad_arguments(BM):
     with pytest.raises(ValueError):
         BM(4, 16, [0, 1, 1, 2])                         # not a permutation
