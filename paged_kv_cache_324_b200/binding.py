@@ -289,6 +289,8 @@ def copy_blocks(k_pool: torch.Tensor, v_pool: torch.Tensor, pairs: torch.Tensor,
     ``check`` (default: the PKV_DEBUG environment variable) the pairs are first checked on the host."""
     if pairs.dtype != torch.int64 or (pairs.numel() and pairs.shape[-1] != 2):
         raise TypeError("pairs must be int64 [n, 2]")
+    if v_pool.shape != k_pool.shape or v_pool.dtype != k_pool.dtype:
+        raise ValueError("k_pool and v_pool must have one shape and dtype")
     if check or (check is None and _debug_checks()):
         check_block_pairs(pairs, k_pool.shape[0], k_pool.shape[0], True)
     block_bytes = k_pool[0].numel() * k_pool.element_size()

@@ -92,3 +92,12 @@ def test_device_error_word_must_be_a_4_byte_integer():
             B._err(bad)
     with pytest.raises(ValueError, match="CUDA tensor"):       # right type, but on the host
         B._err(torch.zeros(1, dtype=torch.int32))
+
+
+def test_copy_blocks_needs_matching_pools():
+    k = torch.zeros((8, 2, 16, 64), dtype=torch.float16)
+    pairs = torch.tensor([[0, 1]], dtype=torch.int64)
+    with pytest.raises(ValueError, match="one shape and dtype"):
+        B.copy_blocks(k, torch.zeros((4, 2, 16, 64), dtype=torch.float16), pairs)
+    with pytest.raises(ValueError, match="one shape and dtype"):
+        B.copy_blocks(k, torch.zeros((8, 2, 16, 64), dtype=torch.bfloat16), pairs)
