@@ -160,7 +160,8 @@ def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_pool: torch.Tensor, 
     """
     S, H, D = q.shape
     NB, Hkv, B, D2 = k_pool.shape
-    if out.shape != q.shape or out.dtype != q.dtype or D2 != D or v_pool.shape != k_pool.shape:
+    if (out.shape != q.shape or out.dtype != q.dtype or D2 != D or v_pool.shape != k_pool.shape
+            or v_pool.dtype != k_pool.dtype):
         raise ValueError("inconsistent shapes or dtypes")
     _tables(block_tables, context_lens, S)
     need = decode_workspace_bytes(S, H, Hkv, D, k_pool.dtype, B, max_context_len, partition_size)
@@ -190,7 +191,8 @@ def paged_attn_prefill(out: torch.Tensor, q: torch.Tensor, k_pool: torch.Tensor,
     T, H, D = q.shape
     NB, Hkv, B, D2 = k_pool.shape
     S = context_lens.numel()
-    if out.shape != q.shape or out.dtype != q.dtype or D2 != D or v_pool.shape != k_pool.shape:
+    if (out.shape != q.shape or out.dtype != q.dtype or D2 != D or v_pool.shape != k_pool.shape
+            or v_pool.dtype != k_pool.dtype):
         raise ValueError("inconsistent shapes or dtypes")
     if k_pool.dtype != q.dtype or v_pool.dtype != q.dtype:
         raise TypeError("prefill needs q and the pools in one 16-bit dtype")
@@ -223,7 +225,8 @@ def paged_attn_prefill_fp8(out: torch.Tensor, q: torch.Tensor, k_pool: torch.Ten
     T, H, D = q.shape
     NB, Hkv, B, D2 = k_pool.shape
     S = context_lens.numel()
-    if out.shape != q.shape or out.dtype != q.dtype or D2 != D or v_pool.shape != k_pool.shape:
+    if (out.shape != q.shape or out.dtype != q.dtype or D2 != D or v_pool.shape != k_pool.shape
+            or v_pool.dtype != k_pool.dtype):
         raise ValueError("inconsistent shapes or dtypes")
     if k_pool.dtype != torch.uint8 or v_pool.dtype != torch.uint8:
         raise TypeError("the pools hold E4M3 bytes (uint8)")
@@ -509,7 +512,8 @@ def paged_attn_decode_shared_prefix(out, q, k_pool, v_pool, block_tables, contex
                                                       P, P, P, I, I, I, P, Z, P, P]
     S, H, D = q.shape
     NB, Hkv, B, D2 = k_pool.shape
-    if out.shape != q.shape or out.dtype != q.dtype or D2 != D or v_pool.shape != k_pool.shape:
+    if (out.shape != q.shape or out.dtype != q.dtype or D2 != D or v_pool.shape != k_pool.shape
+            or v_pool.dtype != k_pool.dtype):
         raise ValueError("inconsistent shapes or dtypes")
     _tables(block_tables, context_lens, S)
     for t, name in ((seq_prefix_len, "seq_prefix_len"), (unit_seqs, "unit_seqs"), (unit_len, "unit_len")):

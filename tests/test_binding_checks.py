@@ -101,3 +101,14 @@ def test_copy_blocks_needs_matching_pools():
         B.copy_blocks(k, torch.zeros((4, 2, 16, 64), dtype=torch.float16), pairs)
     with pytest.raises(ValueError, match="one shape and dtype"):
         B.copy_blocks(k, torch.zeros((8, 2, 16, 64), dtype=torch.bfloat16), pairs)
+
+
+def test_decode_needs_one_pool_dtype():
+    out, q, kp, vp, tables, lens, scale = decode_args()
+    with pytest.raises(ValueError, match="inconsistent"):
+        B.paged_attn_decode(out, q, kp, vp.to(torch.bfloat16), tables, lens, scale, max_context_len=16)
+    with pytest.raises(ValueError, match="inconsistent"):
+        B.paged_attn_decode_shared_prefix(out, q, kp, vp.to(torch.bfloat16), tables, lens, scale, max_context_len=16,
+                                          seq_prefix_len=torch.zeros(S, dtype=torch.int32),
+                                          unit_seqs=torch.zeros((1, 2), dtype=torch.int32),
+                                          unit_len=torch.zeros(1, dtype=torch.int32), max_prefix_len=16)
