@@ -257,6 +257,8 @@ def reshape_and_cache(k: torch.Tensor, v: torch.Tensor, k_pool: torch.Tensor, v_
     NB, Hkv2, B, D2 = k_pool.shape
     if (Hkv2, D2) != (Hkv, D) or v.shape != k.shape or v_pool.shape != k_pool.shape:
         raise ValueError("inconsistent shapes")
+    if v.dtype != k.dtype or v_pool.dtype != k_pool.dtype:
+        raise ValueError("k and v (and the two pools) must share a dtype")
     if slot_mapping.dtype != torch.int64 or slot_mapping.numel() != T:
         raise TypeError("slot_mapping must be int64 [T]")
     status = lib().pkv_reshape_and_cache(
@@ -314,7 +316,7 @@ def swap_blocks(src_k: torch.Tensor, src_v: torch.Tensor, dst_k: torch.Tensor, d
     if check or (check is None and _debug_checks()):
         check_block_pairs(pairs, src_k.shape[0], dst_k.shape[0], src_k.data_ptr() == dst_k.data_ptr())
     if src_k.shape[1:] != dst_k.shape[1:] or src_k.dtype != dst_k.dtype or src_v.shape != src_k.shape \
-            or dst_v.shape != dst_k.shape:
+            or dst_v.shape != dst_k.shape or src_v.dtype != src_k.dtype or dst_v.dtype != dst_k.dtype:
         raise ValueError("pools of one layout and dtype")
     for t, name in ((src_k, "src_k"), (src_v, "src_v"), (dst_k, "dst_k"), (dst_v, "dst_v")):
         if not t.is_cuda and not t.is_pinned():

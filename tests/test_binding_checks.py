@@ -112,3 +112,16 @@ def test_decode_needs_one_pool_dtype():
                                           seq_prefix_len=torch.zeros(S, dtype=torch.int32),
                                           unit_seqs=torch.zeros((1, 2), dtype=torch.int32),
                                           unit_len=torch.zeros(1, dtype=torch.int32), max_prefix_len=16)
+
+
+def test_scatter_and_swap_need_one_dtype_per_pair():
+    k = torch.zeros((3, Hkv, D), dtype=torch.float16)
+    pool = torch.zeros((NB, Hkv, Bs, D), dtype=torch.float16)
+    slots = torch.zeros(3, dtype=torch.int64)
+    with pytest.raises(ValueError, match="share a dtype"):
+        B.reshape_and_cache(k, k.to(torch.bfloat16), pool, pool, slots)
+    with pytest.raises(ValueError, match="share a dtype"):
+        B.reshape_and_cache(k, k, pool, pool.to(torch.bfloat16), slots)
+    pairs = torch.zeros((1, 2), dtype=torch.int64)
+    with pytest.raises(ValueError, match="one layout and dtype"):
+        B.swap_blocks(pool, pool.to(torch.bfloat16), pool, pool, pairs)
