@@ -48,6 +48,20 @@ MUTANTS = {
         "const double vs = kv_dtype == ORC_E4M3 ? v_scale : 1.0;\n\n    /* validate",
         "const double vs = 1.0;\n\n    /* validate",
         lambda: pins.test_fp8_cache_error_against_the_unquantised_cache("fp8")),
+    "decode ignores the K scale of an E4M3 cache": (
+        "const double ks = kv_dtype == ORC_E4M3 ? k_scale : 1.0;\n    const double vs = kv_dtype == ORC_E4M3 ? "
+        "v_scale : 1.0;\n\n    /* validate",
+        "const double ks = 1.0;\n    const double vs = kv_dtype == ORC_E4M3 ? v_scale : 1.0;\n\n    /* validate",
+        lambda: pins.test_fp8_cache_error_against_the_unquantised_cache("fp8")),
+    "prefill ignores the K scale of an E4M3 cache": (
+        "const double ks = kv_dtype == ORC_E4M3 ? k_scale : 1.0;\n    const double vs = kv_dtype == ORC_E4M3 ? "
+        "v_scale : 1.0;\n    for (int s = 0;",
+        "const double ks = 1.0;\n    const double vs = kv_dtype == ORC_E4M3 ? v_scale : 1.0;\n    for (int s = 0;",
+        ppins.test_fp8_cache_uses_the_dequantised_values),
+    "prefill ignores the V scale of an E4M3 cache": (
+        "const double vs = kv_dtype == ORC_E4M3 ? v_scale : 1.0;\n    for (int s = 0;",
+        "const double vs = 1.0;\n    for (int s = 0;",
+        ppins.test_fp8_cache_uses_the_dequantised_values),
     "E4M3 subnormals decoded one binade low": (
         "v = ldexp((double)m, -9);",
         "v = ldexp((double)m, -10);",
