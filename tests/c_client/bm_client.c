@@ -5,7 +5,8 @@
  * block table 41, 7, 19) and the copy-on-write rule of its section "Sharing
  * blocks across sequences", checks the copy pairs with the host pair check,
  * caches a prompt's full blocks and shares them with a second request, swaps
- * both sequences to a second manager, and checks status strings.  Prints "ok"
+ * both sequences to a second manager, packs shared-prefix units from host
+ * tables, checks workspace sizes and status strings.  Prints "ok"
  * and exits 0 when every check holds.
  */
 #include <stdio.h>
@@ -110,6 +111,32 @@ int main(void) {
     CHECK(pkv_bm_ref_count(h, tb[0]) == 2 && pkv_bm_ref_count(h, tb[1]) == 2);
     pkv_bm_destroy(h);
     pkv_bm_destroy(m);
+
+    /* shared-prefix units from host tables: three sequences share their first two full blocks,
+     * a fourth shares nothing; units of at most two members */
+    {
+        const int32_t tables[4 * 3] = {5, 6, 7, 5, 6, 9, 5, 6, 10, 1, 2, -1};
+        const int32_t lens[4] = {40, 40, 35, 20};
+        int32_t spl[4], us[4 * 2], ul[4];
+        int nu = -1, mp = -1;
+        CHECK(pkv_find_shared_prefixes(tables, lens, 4, 3, 16, 2, spl, us, ul, 4, &nu, &mp) == PKV_OK);
+        CHECK(nu == 2 && mp == 32 && ul[0] == 32 && ul[1] == 32);
+        CHECK(spl[0] == 32 && spl[1] == 32 && spl[2] == 32 && spl[3] == 0);
+        CHECK(us[0] == 0 && us[1] == 1 && us[2] == 2 && us[3] == -1);
+        CHECK(pkv_find_shared_prefixes(tables, lens, 4, 3, 16, 2, spl, us, ul, 1, &nu, &mp) ==
+              PKV_ERR_INVALID_ARG);                     /* two units needed, room for one */
+    }
+
+    /* workspace sizes: none when every sequence fits one partition (an explicit 128-token
+     * partition, or the automatic rule, which splits a small batch down to 4 blocks but not
+     * below); the FP8 prefill's widened pools (2 x 6 blocks x 2 heads x 16 x 64 x 2 bytes) plus
+     * a 256-byte-aligned table */
+    CHECK(pkv_decode_workspace_bytes(1, 8, 8, 128, PKV_F16, 16, 100, 128) == 0);
+    CHECK(pkv_decode_workspace_bytes(1, 8, 8, 128, PKV_F16, 16, 60, 0) == 0);
+    CHECK(pkv_decode_workspace_bytes(1, 8, 8, 128, PKV_F16, 16, 100, 0) > 0);
+    CHECK(pkv_decode_workspace_bytes(1, 8, 8, 128, PKV_F16, 16, 100, 16) > 0);
+    CHECK(pkv_prefill_fp8_workspace_bytes(2, 3, 2, 64, 16) == 2 * 24576 + 256);
+    CHECK(pkv_prefill_fp8_workspace_bytes(0, 3, 2, 64, 16) == 0);
     printf("ok\n");
     return 0;
 }
