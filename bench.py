@@ -687,6 +687,9 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = wl.make(args.config)        # weak scaling: every rank runs a batch of the same shape
+    heads = args.shard == "heads" and world > 1
+    if heads:                       # strong scaling: one batch, each rank its share of the KV heads
+        w = wl.shard_heads(w, rank, world)
     ps = w.partition_size if args.partition == "config" else (0 if args.partition == "auto" else int(args.partition))
     ds = DeviceStep(w, dev, ps, prefix_aware=args.prefix_aware)
     step_bytes = wl.step_algorithmic_bytes(w)
@@ -772,12 +775,12 @@ def run_ours(args, rank, world, local_rank):
     tr = NCU_TRAFFIC.get(args.config)
     # the capture ran the plain decode at the workload's own partition size
     if (tr and tr.get("kernel_sha") == decode_source_sha() and args.partition == "config"
-            and not args.prefix_aware):
+            and not args.prefix_aware and not heads):
         traffic = tr["bytes_per_launch"]
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None,
+        "scaling": "strong" if heads else "weak", "vs_baseline": None,
         "dtype": w.kv_dtype if w.kv_dtype != "e4m3" else "e4m3 (KV), f16 (q/out), f32 accumulate",
         "data": "synthetic (seeded N(0,1) K/V/q; random-byte pool content in unwritten slots)",
         "config": {
@@ -793,9 +796,10 @@ def run_ours(args, rank, world, local_rank):
                    if roof_bytes > L2_BYTES else
                    ("no flush: the %.0f MB of distinct KV fit in the 126 MB L2, so repeated reads of shared "
                     "blocks may hit L2" % (roof_bytes / 1e6))),
-            "parallelism": f"dp{world}" if world > 1 else "single GPU",
+            "parallelism": (f"tp{world} (KV heads split, identical block tables)" if heads
+                            else f"dp{world}" if world > 1 else "single GPU"),
         },
-        "sequences_per_s": round(seqs / (ms_step * 1e-3), 1),
+        "sequences_per_s": round((w.num_seqs if heads else seqs) / (ms_step * 1e-3), 1),
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
         "pct_of_nominal_8tbs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
         "kernel_ms": {"paged_attn_decode": round(dec_avg, 5), "reshape_and_cache": round(sum(sc_ms) / K, 5),
@@ -896,6 +900,9 @@ def main():
     ap.add_argument("--partition", default="config",
                     help="'config' (the workload's stated partition size, else automatic), 'auto', or tokens")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--shard", default="sequences", choices=["sequences", "heads"],
+                    help="decode under torchrun: each rank its own batch (weak scaling) or one batch with the "
+                         "KV heads split over the ranks (strong scaling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -159,6 +159,8 @@ class DecodeWorkload:
     step_scatter: Scatter        # the step's appended tokens (one per sequence)
     partition_size: int = 0      # split-context partition (tokens) the workload states; 0 = automatic
     description: str = ""
+    kv_head_range: Optional[Tuple[int, int]] = None   # a head shard: its KV heads in the full pools
+    pool_heads: int = 0          # KV heads of the full pools a shard is cut from (0 = num_kv_heads)
 
     @property
     def max_blocks(self) -> int:
@@ -181,10 +183,42 @@ class DecodeWorkload:
         chunk repeated, so that large pools are cheap to make).  Unwritten slots therefore
         hold arbitrary bit patterns, NaN and Inf included."""
         rng = np.random.default_rng([self.seed, 1 if which == "k" else 2])
-        chunk = garbage_bytes(rng, min(self.pool_bytes, 32 << 20))
-        raw = np.resize(chunk, self.pool_bytes)
+        full = (self.num_blocks, self.pool_heads or self.num_kv_heads, self.block_size, self.head_dim)
+        nbytes = int(np.prod(full)) * ELEM_BYTES[self.kv_dtype]
+        chunk = garbage_bytes(rng, min(nbytes, 32 << 20))
+        raw = np.resize(chunk, nbytes)
         dt = np.uint8 if self.kv_dtype == "e4m3" else np.uint16
-        return raw.view(dt).reshape(self.pool_shape)
+        pool = raw.view(dt).reshape(full)
+        if self.kv_head_range is None:
+            return pool
+        k0, k1 = self.kv_head_range
+        return np.ascontiguousarray(pool[:, k0:k1])
+
+
+def shard_heads(w: DecodeWorkload, rank: int, world: int) -> DecodeWorkload:
+    """Rank ``rank`` of ``world``'s share of a decode workload split by KV head: KV heads
+    [rank * Hkv / world, (rank + 1) * Hkv / world) with the query heads that use them (query head
+    h uses KV head h / G), the same sequences, lengths and block tables, and the same slice of
+    every pool, new token and query.  Attention of each (sequence, KV head) is independent, so
+    the shards' outputs side by side along the head axis are the whole workload's."""
+    if w.kv_head_range is not None:
+        raise ValueError("already a shard")
+    if world <= 0 or not 0 <= rank < world or w.num_kv_heads % world:
+        raise ValueError(f"{w.num_kv_heads} KV heads do not split over {world} ranks")
+    n = w.num_kv_heads // world
+    G = w.num_heads // w.num_kv_heads
+    k0, k1 = rank * n, (rank + 1) * n
+
+    def cut(op):
+        if not isinstance(op, Scatter):
+            return op                                  # block copies move whole blocks: every head
+        return Scatter(np.ascontiguousarray(op.k[:, k0:k1]), np.ascontiguousarray(op.v[:, k0:k1]), op.slots)
+
+    return dataclasses.replace(
+        w, name=f"{w.name}_kv{k0}-{k1}", num_heads=n * G, num_kv_heads=n,
+        q=np.ascontiguousarray(w.q[:, k0 * G:k1 * G]), setup=[cut(op) for op in w.setup],
+        step_scatter=cut(w.step_scatter), kv_head_range=(k0, k1), pool_heads=w.num_kv_heads,
+        description=f"{w.description}; KV heads {k0}..{k1 - 1} of {w.num_kv_heads}")
 
 
 def _new_values(rng, tokens, hkv, d, dtype):
