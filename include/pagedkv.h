@@ -140,6 +140,7 @@ int pkv_decode_partition_size(int num_seqs, int num_kv_heads, int head_dim, pkv_
  *                  parallel and are merged exactly by log-sum-exp
  *   workspace      device buffer of at least pkv_decode_workspace_bytes()
  *                  bytes (may be NULL when that is 0), 256-byte aligned
+ *   scale          finite; k_scale, v_scale (FP8 pools only) positive and finite
  */
 pkv_status pkv_paged_attn_decode(void* out, const void* q, pkv_dtype q_dtype,
                                  const void* k_pool, const void* v_pool, pkv_dtype kv_dtype,
@@ -168,11 +169,29 @@ pkv_status pkv_paged_attn_decode(void* out, const void* q, pkv_dtype q_dtype,
  *                   unit (-1 pads the last slots); members must share their first
  *                   unit_len[u] / block_size table entries and have that prefix length
  *   unit_len        device int32 [num_units]
- *   max_prefix_len  bound of the prefix lengths
+ *   max_prefix_len  bound of every seq_prefix_len and unit_len
+ *   plan            PKV_PREFIX_PLAN_AUTO: the passes above only when the units'
+ *                   shared prefixes, counted once per unit, exceed the device's
+ *                   L2 (otherwise the plain call's repeated reads of them hit L2
+ *                   and its single pass is faster, so it runs instead);
+ *                   PKV_PREFIX_PLAN_SHARED: always the passes above;
+ *                   PKV_PREFIX_PLAN_PLAIN: always the plain call
  *   workspace       >= pkv_shared_prefix_workspace_bytes() bytes (always needed)
+ * Preconditions, checked on the device: every sequence with seq_prefix_len > 0
+ * is a member of exactly one unit, and every member's seq_prefix_len equals its
+ * unit's unit_len; members are packed before the -1 pads; no length exceeds
+ * max_prefix_len.  A sequence whose prefix no unit covers, every member of a
+ * unit that breaks these rules, and a length beyond max_prefix_len get NaN
+ * outputs and PKV_DEVERR_CONTEXT_LEN (nothing is read outside the workspace).
  * Other arguments, errors and results as for pkv_paged_attn_decode.
  * pkv_find_shared_prefixes() builds the three arrays from host copies of the tables.
  */
+typedef enum {
+    PKV_PREFIX_PLAN_AUTO = 0,
+    PKV_PREFIX_PLAN_SHARED = 1,
+    PKV_PREFIX_PLAN_PLAIN = 2
+} pkv_prefix_plan;
+
 size_t pkv_shared_prefix_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
                                          pkv_dtype kv_dtype, int block_size, int max_context_len,
                                          int num_units, int max_prefix_len, int partition_size);
@@ -186,7 +205,8 @@ pkv_status pkv_paged_attn_decode_shared_prefix(void* out, const void* q, pkv_dty
                                                int block_size, int num_blocks, float scale, int partition_size,
                                                const int32_t* seq_prefix_len, const int32_t* unit_seqs,
                                                const int32_t* unit_len, int num_units, int unit_width,
-                                               int max_prefix_len, void* workspace, size_t workspace_bytes,
+                                               int max_prefix_len, int plan, void* workspace,
+                                               size_t workspace_bytes,
                                                uint32_t* device_error, void* stream);
 
 /*
@@ -226,7 +246,10 @@ pkv_status pkv_find_shared_prefixes(const int32_t* block_tables, const int32_t* 
  * call shares the one array and leaves its contents behind (nothing in it
  * needs to start at zero: each call writes every entry it reads), so calls
  * that overlap on the GPU -- concurrent streams, or several host threads --
- * race on it; serialise them.
+ * race on it; serialise them.  Arguments are checked exactly as for
+ * pkv_paged_attn_decode before the size test.  The looked-up address is kept
+ * for the life of the process and does not survive cudaDeviceReset: do not
+ * use this call after one.
  */
 pkv_status pkv_paged_attn_decode_static_ws(void* out, const void* q, pkv_dtype q_dtype,
                                            const void* k_pool, const void* v_pool, pkv_dtype kv_dtype,

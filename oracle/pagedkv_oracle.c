@@ -45,6 +45,7 @@
  *     division done in IEEE float32.
  */
 #include <math.h>
+#include <pthread.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -144,11 +145,27 @@ uint8_t orc_f32_to_e4m3(float x)
     return sign | (uint8_t)(((unb + 7) << 3) | mant);
 }
 
+/*
+ * Every 16-bit pattern's value, filled once from the decoders above: the
+ * attention loops read each cached element many times, and a table lookup
+ * gives the same float64 value as calling the decoder again, only faster.
+ */
+static double f16_value[65536], bf16_value[65536];
+static pthread_once_t value_tables_once = PTHREAD_ONCE_INIT;
+
+static void fill_value_tables(void)
+{
+    for (uint32_t h = 0; h < 65536; ++h) {
+        f16_value[h] = orc_f16_to_f64((uint16_t)h);
+        bf16_value[h] = orc_bf16_to_f64((uint16_t)h);
+    }
+}
+
 static double load_elem(const void* base, size_t idx, int dtype, double scale)
 {
     switch (dtype) {
-    case ORC_F16:  return orc_f16_to_f64(((const uint16_t*)base)[idx]);
-    case ORC_BF16: return orc_bf16_to_f64(((const uint16_t*)base)[idx]);
+    case ORC_F16:  return f16_value[((const uint16_t*)base)[idx]];
+    case ORC_BF16: return bf16_value[((const uint16_t*)base)[idx]];
     default:       return orc_e4m3_to_f64(((const uint8_t*)base)[idx]) * scale;
     }
 }
@@ -173,6 +190,7 @@ int orc_paged_attn_decode(double* out, const void* q, int q_dtype,
                           int num_kv_heads, int head_dim, int block_size,
                           int num_blocks, double scale, int num_threads)
 {
+    pthread_once(&value_tables_once, fill_value_tables);
     if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
         block_size <= 0 || num_blocks <= 0 || num_heads % num_kv_heads != 0 ||
         (q_dtype != ORC_F16 && q_dtype != ORC_BF16) ||
@@ -273,6 +291,7 @@ int orc_paged_attn_prefill(double* out, const void* q, int q_dtype,
                            int num_seqs, int num_heads, int num_kv_heads, int head_dim,
                            int block_size, int num_blocks, double scale, int num_threads)
 {
+    pthread_once(&value_tables_once, fill_value_tables);
     if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
         block_size <= 0 || num_blocks <= 0 || num_heads % num_kv_heads != 0 ||
         (q_dtype != ORC_F16 && q_dtype != ORC_BF16) ||
@@ -367,6 +386,7 @@ int orc_reshape_and_cache(const void* k, const void* v, int in_dtype,
                           const int64_t* slot_mapping, int num_tokens,
                           int num_kv_heads, int head_dim, int block_size, int num_blocks)
 {
+    pthread_once(&value_tables_once, fill_value_tables);
     if ((in_dtype != ORC_F16 && in_dtype != ORC_BF16) ||
         (kv_dtype != in_dtype && kv_dtype != ORC_E4M3) || num_tokens < 0 ||
         num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
@@ -473,6 +493,7 @@ int orc_gather(void* out, const void* pool, int kv_dtype, const int32_t* table,
 /* Element-wise decoders over arrays, for the tests' exhaustive checks. */
 void orc_decode_array(double* out, const void* in, int dtype, size_t n)
 {
+    pthread_once(&value_tables_once, fill_value_tables);
     for (size_t i = 0; i < n; ++i)
         out[i] = load_elem(in, i, dtype, 1.0);
 }

@@ -503,15 +503,23 @@ def shared_prefix_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, k
                                                partition_size)
 
 
+#: pkv_prefix_plan codes
+PREFIX_PLANS = {"auto": 0, "shared": 1, "plain": 2}
+
+
 def paged_attn_decode_shared_prefix(out, q, k_pool, v_pool, block_tables, context_lens, scale, *,
                                     max_context_len: int, seq_prefix_len, unit_seqs, unit_len,
                                     max_prefix_len: int, k_scale: float = 1.0, v_scale: float = 1.0,
-                                    partition_size: int = 0, workspace=None, device_error=None, stream=None):
-    """Shared-prefix decode: device tensors; seq_prefix_len int32 [S], unit_seqs int32 [U, W], unit_len int32 [U]."""
+                                    partition_size: int = 0, plan: str = "auto", workspace=None, device_error=None,
+                                    stream=None):
+    """Shared-prefix decode: device tensors; seq_prefix_len int32 [S], unit_seqs int32 [U, W], unit_len int32 [U].
+    plan: "auto" (the library picks the shared-prefix passes or the plain call), "shared" or "plain"."""
     L = lib()
     P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     L.pkv_paged_attn_decode_shared_prefix.argtypes = [P, P, I, P, P, I, F, F, P, I, P, I, I, I, I, I, I, I, F, I,
-                                                      P, P, P, I, I, I, P, Z, P, P]
+                                                      P, P, P, I, I, I, I, P, Z, P, P]
+    if plan not in PREFIX_PLANS:
+        raise ValueError(f"plan must be one of {sorted(PREFIX_PLANS)}")
     S, H, D = q.shape
     NB, Hkv, B, D2 = k_pool.shape
     if (out.shape != q.shape or out.dtype != q.dtype or D2 != D or v_pool.shape != k_pool.shape
@@ -535,7 +543,7 @@ def paged_attn_decode_shared_prefix(out, q, k_pool, v_pool, block_tables, contex
         _dev(context_lens, "context_lens"), int(max_context_len), S, H, Hkv, D, B, NB, float(scale),
         int(partition_size), _dev(seq_prefix_len, "seq_prefix_len"),
         _dev(unit_seqs, "unit_seqs") if U else None, _dev(unit_len, "unit_len") if U else None, U, W,
-        int(max_prefix_len), _dev(workspace, "workspace"), workspace.numel(), _err(device_error),
-        _stream(stream))
+        int(max_prefix_len), PREFIX_PLANS[plan], _dev(workspace, "workspace"), workspace.numel(),
+        _err(device_error), _stream(stream))
     _check(status, "paged_attn_decode_shared_prefix")
     return out

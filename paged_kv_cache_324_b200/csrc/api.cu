@@ -18,6 +18,13 @@ int num_sms() {
     return n;
 }
 
+long long l2_bytes() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 126ll << 20;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrL2CacheSize, dev) != cudaSuccess || n <= 0) return 126ll << 20;
+    return n;
+}
+
 EncodeTiledFn encode_tiled_fn() {
     static EncodeTiledFn fn = nullptr;
     static std::once_flag once;

@@ -85,8 +85,13 @@ struct DecodeArgs {
     const int32_t* unit_len;    // prefix pass: [units] shared tokens of each unit
     int unit_width;
     int slot_base;              // first partition slot of the workspace this pass writes
-    int prefix_partition_size;  // merge: partition size of the prefix pass
+    int prefix_partition_size;  // tail pass and merge: partition size of the prefix pass
+    int max_prefix_len;         // bound of every unit_len and seq_start (0 in the plain call)
 };
+
+// Written by the tail pass into every prefix slot a sequence's merge will read, before the
+// prefix pass runs: a slot still holding it was not covered by a unit (max NaN, sum -1).
+constexpr uint32_t kUnwrittenSum = 0xbf800000u;   // -1.0f
 
 // ---- MMA and conversions ------------------------------------------------------
 
@@ -266,28 +271,53 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
     const bool prefix_pass = a.unit_seqs != nullptr;
     int rows = G, L, start = 0, tseq = z;
     bool bad_len;
+    // Every CTA passes pdl_wait() before it exits, so that a grid only completes after the
+    // kernel before it on the stream has: the merge relies on that ordering through both passes.
     if (prefix_pass) {
+        // members: valid sequence ids packed first, -1 pads after them; each member's own prefix
+        // length must be the unit's (seq_start holds seq_prefix_len here)
         const int32_t* mem = a.unit_seqs + static_cast<size_t>(z) * a.unit_width;
         tseq = __ldg(mem);
-        int members = 0;
-        for (int m = 0; m < a.unit_width; ++m) members += __ldg(mem + m) >= 0;
-        rows = members * G;
         L = __ldg(a.unit_len + z);
-        bad_len = tseq < 0 || tseq >= a.num_seqs || L < 0 || L % BS != 0 || L > a.max_blocks_per_seq * BS;
+        int members = 0;
+        bool bad_member = false, padded = false;
+        for (int m = 0; m < a.unit_width; ++m) {
+            const int id = __ldg(mem + m);
+            if (id < 0) {
+                padded = true;
+                continue;
+            }
+            ++members;
+            bad_member |= padded || id >= a.num_seqs || (a.seq_start && __ldg(a.seq_start + id) != L);
+        }
+        rows = members * G;
+        bad_len = members == 0 || bad_member || L < 0 || L % BS != 0 || L > a.max_blocks_per_seq * BS ||
+                  L > a.max_prefix_len;
         if (bad_len || L == 0 || grid_timed_out(a.err)) {
             if (bad_len && part == 0 && threadIdx.x == 0) raise_error(a.err, PKV_DEVERR_CONTEXT_LEN);
-            return;   // members' merges see a bad or empty prefix and answer for it
+            pdl_wait();
+            return;   // the members' prefix slots keep the tail pass's marker: their merges give NaN
         }
     } else {
         const int Lt = __ldg(a.context_lens + z);
         start = a.seq_start ? __ldg(a.seq_start + z) : 0;
         bad_len = Lt < 0 || Lt > a.max_blocks_per_seq * BS || Lt > a.max_context_len || start < 0 || start > Lt ||
-                  start % BS != 0;
+                  start % BS != 0 || start > a.max_prefix_len;
         L = Lt - start;
+        if (!bad_len && start > 0 && part == 0) {
+            // mark the prefix slots this sequence's merge reads; the prefix pass (next on the
+            // stream) overwrites those of the units that cover it
+            pdl_wait();
+            const int np_pre = (start + a.prefix_partition_size - 1) / a.prefix_partition_size;
+            const size_t row0 = static_cast<size_t>(z) * H + static_cast<size_t>(kvh) * G;
+            for (int e = threadIdx.x; e < G * np_pre; e += kThreads)
+                a.ws_ml[(row0 + e / np_pre) * a.max_partitions + e % np_pre] =
+                    make_float2(__int_as_float(0x7fc00000), __uint_as_float(kUnwrittenSum));
+        }
         const bool give_up = grid_timed_out(a.err);
         if (bad_len || L == 0 || give_up) {
+            pdl_wait();
             if (part == 0 && (start == 0 || bad_len)) {
-                pdl_wait();
                 if (bad_len && threadIdx.x == 0) raise_error(a.err, PKV_DEVERR_CONTEXT_LEN);
                 const float v = (bad_len || give_up) ? __int_as_float(0x7fc00000) : 0.f;
                 const size_t row0 = static_cast<size_t>(z) * H + static_cast<size_t>(kvh) * G;
@@ -305,7 +335,10 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
     };
     const int PS = a.partition_size;
     const int nparts = (L + PS - 1) / PS;
-    if (part >= nparts) return;
+    if (part >= nparts) {
+        pdl_wait();
+        return;
+    }
     const int tok_begin = part * PS;
     const int tok_end = min(L, tok_begin + PS);
     const int nblk = (tok_end - tok_begin + BS - 1) / BS;
@@ -696,7 +729,7 @@ __global__ void __launch_bounds__(D) decode_reduce_kernel(const DecodeArgs a) {
     const int start = a.seq_start ? __ldg(a.seq_start + s) : 0;
     const size_t row = static_cast<size_t>(s) * a.num_heads + qh;
     if (L < 0 || L > a.max_blocks_per_seq * a.block_size || L > a.max_context_len || start < 0 || start > L ||
-        start % a.block_size != 0) {
+        start % a.block_size != 0 || start > a.max_prefix_len) {
         if (start > 0) store_out<kQBf16>(a.out, row * D + d, __int_as_float(0x7fc00000));
         return;   // (a sequence without a prefix got its NaN from pass 1)
     }
@@ -723,7 +756,11 @@ __global__ void __launch_bounds__(D) decode_reduce_kernel(const DecodeArgs a) {
         float M = -INFINITY;
 #pragma unroll
         for (int p = 0; p < 8; ++p)
-            if (p < np) M = fmaxf(M, v[p].x);
+            if (p < np) {
+                M = fmaxf(M, v[p].x);
+                if (d == 0 && p < np_pre && __float_as_uint(v[p].y) == kUnwrittenSum)
+                    raise_error(a.err, PKV_DEVERR_CONTEXT_LEN);   // no unit covered this prefix slot: NaN
+            }
         float num = 0.f, den = 0.f;
 #pragma unroll
         for (int p = 0; p < 8; ++p)
@@ -750,6 +787,7 @@ __global__ void __launch_bounds__(D) decode_reduce_kernel(const DecodeArgs a) {
     float den = 0.f;
     for (int p = d; p < np; p += D) {
         const float2 v = ml[slot(p)];
+        if (p < np_pre && __float_as_uint(v.y) == kUnwrittenSum) raise_error(a.err, PKV_DEVERR_CONTEXT_LEN);
         const float w = exp2f(v.x - M) * v.y;
         sw[p] = w;
         den += w;
@@ -893,7 +931,7 @@ pkv_status validate(const void* out, const void* q, pkv_dtype q_dtype, const voi
         num_blocks <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0 || partition_size < 0)
         return PKV_ERR_INVALID_ARG;
     if (num_heads % num_kv_heads != 0) return PKV_ERR_INVALID_ARG;
-    if (!(scale == scale)) return PKV_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return PKV_ERR_INVALID_ARG;
     if (num_heads / num_kv_heads > 16) return PKV_ERR_UNSUPPORTED;
     if (block_size != 16 && block_size != 32) return PKV_ERR_UNSUPPORTED;
     if (partition_size % block_size != 0) return PKV_ERR_INVALID_ARG;
@@ -901,7 +939,8 @@ pkv_status validate(const void* out, const void* q, pkv_dtype q_dtype, const voi
     if (kv_dtype != q_dtype && kv_dtype != PKV_FP8_E4M3) return PKV_ERR_UNSUPPORTED;
     if (kv_dtype == PKV_FP8_E4M3) {
         if (head_dim != 128) return PKV_ERR_UNSUPPORTED;
-        if (!(k_scale > 0.f && v_scale > 0.f)) return PKV_ERR_INVALID_ARG;
+        if (!(k_scale > 0.f && v_scale > 0.f) || !std::isfinite(k_scale) || !std::isfinite(v_scale))
+            return PKV_ERR_INVALID_ARG;
     } else if (head_dim != 64 && head_dim != 128) {
         return PKV_ERR_UNSUPPORTED;
     }
@@ -1056,7 +1095,7 @@ extern "C" pkv_status pkv_paged_attn_decode_shared_prefix(
     float k_scale, float v_scale, const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
     int max_context_len, int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
     int num_blocks, float scale, int partition_size, const int32_t* seq_prefix_len, const int32_t* unit_seqs,
-    const int32_t* unit_len, int num_units, int unit_width, int max_prefix_len, void* workspace,
+    const int32_t* unit_len, int num_units, int unit_width, int max_prefix_len, int plan, void* workspace,
     size_t workspace_bytes, uint32_t* device_error, void* stream) {
     using namespace pkv;
     const pkv_status v = validate(out, q, q_dtype, k_pool, v_pool, kv_dtype, k_scale, v_scale, block_tables,
@@ -1065,7 +1104,8 @@ extern "C" pkv_status pkv_paged_attn_decode_shared_prefix(
     if (v != PKV_OK || num_seqs == 0) return v;
     const int G = num_heads / num_kv_heads;
     if (num_units < 0 || num_units > 65535 || unit_width <= 0 || max_prefix_len < 0 ||
-        max_prefix_len > max_context_len || max_prefix_len % block_size != 0)
+        max_prefix_len > max_context_len || max_prefix_len % block_size != 0 ||
+        (plan != PKV_PREFIX_PLAN_AUTO && plan != PKV_PREFIX_PLAN_SHARED && plan != PKV_PREFIX_PLAN_PLAIN))
         return PKV_ERR_INVALID_ARG;
     if (unit_width * G > 16) return PKV_ERR_UNSUPPORTED;
     if (!seq_prefix_len || (num_units > 0 && (!unit_seqs || !unit_len))) return PKV_ERR_INVALID_ARG;
@@ -1084,10 +1124,26 @@ extern "C" pkv_status pkv_paged_attn_decode_shared_prefix(
     if (!workspace || workspace_bytes < need) return PKV_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) & 255) return PKV_ERR_ALIGNMENT;
 
+    // Automatic plan: when the shared prefixes, counted once per unit, fit in L2, the plain call's
+    // repeated reads of them are L2 hits and its single pass beats the prefix pass + tail pass +
+    // merge; the plain call then runs (its workspace is never larger than this one's).
+    bool shared = num_units > 0 && p_pre > 0 && plan != PKV_PREFIX_PLAN_PLAIN;
+    if (shared && plan == PKV_PREFIX_PLAN_AUTO) {
+        const double per_token = 2.0 * num_kv_heads * head_dim * (kv_dtype == PKV_FP8_E4M3 ? 1 : 2);
+        shared = static_cast<double>(num_units) * max_prefix_len * per_token > static_cast<double>(l2_bytes());
+    }
+    if (!shared)
+        return pkv_paged_attn_decode(out, q, q_dtype, k_pool, v_pool, kv_dtype, k_scale, v_scale, block_tables,
+                                     max_blocks_per_seq, context_lens, max_context_len, num_seqs, num_heads,
+                                     num_kv_heads, head_dim, block_size, num_blocks, scale, partition_size,
+                                     workspace, workspace_bytes, device_error, stream);
+
     DecodeArgs a = base_args(out, q, block_tables, max_blocks_per_seq, context_lens, max_context_len, num_seqs,
                              num_heads, num_kv_heads, num_blocks, block_size, kv_dtype, k_scale, v_scale, scale, ps,
                              device_error);
     a.max_partitions = p_pre + p_tail;
+    a.max_prefix_len = max_prefix_len;
+    a.prefix_partition_size = ps_pre;
     set_partials(a, workspace, static_cast<size_t>(num_seqs) * num_heads * a.max_partitions, head_dim);
 
     alignas(64) CUtensorMap km;
@@ -1096,10 +1152,17 @@ extern "C" pkv_status pkv_paged_attn_decode_shared_prefix(
         !encode_pool_map(&vm, v_pool, kv_dtype, head_dim, block_size, num_kv_heads, num_blocks))
         return PKV_ERR_CUDA;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    pkv_status r = PKV_OK;
-    if (num_units > 0 && p_pre > 0) {   // shared tokens: every unit's rows against its prefix, once
+    // The tail pass runs first: it also marks every prefix slot a merge will read, so that the
+    // prefix pass (next) leaves the marker only where no unit covers a sequence's prefix.
+    DecodeArgs at = a;   // each sequence's own tokens, from the end of its prefix
+    at.seq_start = seq_prefix_len;
+    at.slot_base = p_pre;
+    pkv_status r = with_instance(kv_dtype, q_dtype, head_dim, block_size, G > 8,
+                                 Pass1{at, km, vm, static_cast<unsigned>(p_tail), static_cast<unsigned>(num_seqs), st});
+    if (r == PKV_OK) {   // shared tokens: every unit's rows against its prefix, once
         DecodeArgs ap = a;
         ap.partition_size = ps_pre;
+        ap.seq_start = seq_prefix_len;   // read only to check the members' prefix lengths
         ap.unit_seqs = unit_seqs;
         ap.unit_len = unit_len;
         ap.unit_width = unit_width;
@@ -1107,13 +1170,6 @@ extern "C" pkv_status pkv_paged_attn_decode_shared_prefix(
         r = with_instance(kv_dtype, q_dtype, head_dim, block_size, unit_width * G > 8,
                           Pass1{ap, km, vm, static_cast<unsigned>(p_pre), static_cast<unsigned>(num_units), st});
     }
-    DecodeArgs at = a;   // each sequence's own tokens, from the end of its prefix
-    at.seq_start = seq_prefix_len;
-    at.slot_base = p_pre;
-    at.prefix_partition_size = ps_pre;
-    if (r == PKV_OK)
-        r = with_instance(kv_dtype, q_dtype, head_dim, block_size, G > 8,
-                          Pass1{at, km, vm, static_cast<unsigned>(p_tail), static_cast<unsigned>(num_seqs), st});
     if (r == PKV_OK) r = with_instance(kv_dtype, q_dtype, head_dim, block_size, G > 8, Merge{at, st});
     return r;
 }
@@ -1129,7 +1185,9 @@ extern "C" pkv_status pkv_paged_attn_decode_shared_prefix(
 // Host code cannot use the array's name as a device address (it names a
 // host-side stand-in), so each device's address is looked up once with
 // cudaGetSymbolAddress, with that device current, on the first call made on
-// that device; make that first call before any stream capture.
+// that device; make that first call before any stream capture.  The address
+// is kept for the life of the process: it does not survive cudaDeviceReset
+// (which unloads the module), so do not use this call after one.
 
 namespace pkv {
 namespace {
@@ -1169,6 +1227,10 @@ extern "C" pkv_status pkv_paged_attn_decode_static_ws(
     const int32_t* context_lens, int max_context_len, int num_seqs, int num_heads, int num_kv_heads,
     int head_dim, int block_size, int num_blocks, float scale, int partition_size, uint32_t* device_error,
     void* stream) {
+    const pkv_status v = pkv::validate(out, q, q_dtype, k_pool, v_pool, kv_dtype, k_scale, v_scale, block_tables,
+                                       max_blocks_per_seq, context_lens, max_context_len, num_seqs, num_heads,
+                                       num_kv_heads, head_dim, block_size, num_blocks, scale, partition_size);
+    if (v != PKV_OK || num_seqs == 0) return v;
     const size_t need = pkv_decode_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, kv_dtype,
                                                    block_size, max_context_len, partition_size);
     if (need > pkv::kStaticWsBytes) return PKV_ERR_WORKSPACE;

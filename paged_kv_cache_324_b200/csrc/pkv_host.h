@@ -11,8 +11,9 @@ namespace pkv {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// SM count of the current device.
+// SM count and L2 size in bytes of the current device.
 int num_sms();
+long long l2_bytes();
 
 // cuTensorMapEncodeTiled from the driver, looked up once through the runtime
 // (no link-time dependency on libcuda).  nullptr if unavailable.

@@ -22,7 +22,8 @@
 //              (tile B half a period behind tile A)
 //              S = Q K^T (M=128, N=128, both operands K-major in shared
 //              memory) and O += P V (M=128, N=head_dim; P read from tensor
-//              memory, V an MN-major shared-memory operand).  The MMAs of a CTA
+//              memory, V an MN-major shared-memory operand; for bf16 a second
+//              product O += P_lo V over the same V tile).  The MMAs of a CTA
 //              execute in issue order, which is what lets P overwrite the S it
 //              came from and S_X(j+1) overwrite P_X(j) once PV_X(j) has read it;
 //   warps 2-9  softmax of tile A, warps 10-17 of tile B, two warps per TMEM
@@ -33,8 +34,10 @@
 //              one exceeds it by more than 2^8 (the result does not depend on
 //              the reference maximum; the lag only bounds the weights), write P
 //              as packed 16-bit pairs into the upper half of the same S columns
-//              with tcgen05.st, and rescale O in TMEM when the maximum moves;
-//              finally O / l.
+//              with tcgen05.st (bf16: also the residual P - bf16(P) into the
+//              lower half, so that P.V sees ~16 significant bits of every
+//              weight, as a 16-bit f16 P's 11 bits nearly do), and rescale O in
+//              TMEM when the maximum moves; finally O / l.
 // While tile A's softmax works on S_A(j+1), the tensor core computes PV_B(j)
 // and S_B(j+1), and the other way round.
 //
@@ -67,7 +70,9 @@ constexpr int kTileWarps = 4 * kHalves;
 constexpr int kVWarp = 2 + kTiles * kTileWarps;
 constexpr int kPThreads = 32 * (kVWarp + 1);   // warp 0 TMA (Q, K), warp 1 MMA, softmax, last warp TMA (V)
 constexpr uint32_t kTmemCols = 512;   // S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512)
-constexpr uint32_t kTmemS = 0, kTmemO = 256, kTmemP = 64;   // P_X: the upper half of S_X, packed pairs
+// P_X: the upper half of S_X, packed pairs; for bf16 the residual P_X - bf16(P_X) (P_lo) goes over the
+// lower half, so that the P.V product sees ~16 significant bits of each weight (two MMAs per key step)
+constexpr uint32_t kTmemS = 0, kTmemO = 256, kTmemP = 64, kTmemPlo = 0;
 constexpr float kMaxLag = 8.0f;       // log2 of the largest weight the lagging maximum allows
 constexpr uint32_t kChunkBytes = kRows * 128;   // 128 rows x 128 bytes: one 64-column chunk
 
@@ -223,6 +228,15 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
         : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
     return d;
 }
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+    float2 d;
+    asm("{.reg .b64 pa, pb, pd;\n\t"
+        "mov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %5};\n\t"
+        "sub.rn.f32x2 pd, pa, pb;\n\tmov.b64 {%0, %1}, pd;}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
 __device__ __forceinline__ float max3f(float a, float b, float c) {
     float d;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -250,6 +264,12 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
     asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
                  "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t (&r)[4]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(r[0]), "r"(r[1]),
+                 "r"(r[2]), "r"(r[3])
                  : "memory");
 }
 
@@ -499,9 +519,12 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
                 const int vs = j % kVStages;
 #pragma unroll
                 for (int kk = 0; kk < kKeys / 16; ++kk) {
-                    mma_f16_ts(tmem + kTmemO + t * 128, tmem + kTmemS + t * kKeys + kTmemP + kk * 8,
-                               smem_desc(sV + vs * Gm::kTile + kk * 16 * 128, kChunkBytes, 1024), idesc_o,
+                    const uint64_t vdesc = smem_desc(sV + vs * Gm::kTile + kk * 16 * 128, kChunkBytes, 1024);
+                    mma_f16_ts(tmem + kTmemO + t * 128, tmem + kTmemS + t * kKeys + kTmemP + kk * 8, vdesc, idesc_o,
                                j > 0 || kk > 0);
+                    if constexpr (kBf16)   // the weights' bf16 residual against the same V rows
+                        mma_f16_ts(tmem + kTmemO + t * 128, tmem + kTmemS + t * kKeys + kTmemPlo + kk * 8, vdesc,
+                                   idesc_o, true);
                 }
                 if (j == (t == 0 ? ntk_a : ntk_b) - 1) mma_commit(o_done(t));
                 return true;
@@ -590,16 +613,23 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
             const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nm2 = make_float2(-m_used, -m_used);
             float2 sp[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-            for (int h = 0; h < 4; ++h) {                    // 16 keys (8 packed words) at a time
-                uint32_t pk[8];
+            for (int h = 0; h < 8; ++h) {                    // 8 keys (4 packed words) at a time
+                uint32_t pk[4], pl[4];
 #pragma unroll
-                for (int c = 0; c < 16; c += 2) {
-                    const float2 e = fma2(make_float2(x[16 * h + c], x[16 * h + c + 1]), sc2, nm2);
+                for (int c = 0; c < 8; c += 2) {
+                    const float2 e = fma2(make_float2(x[8 * h + c], x[8 * h + c + 1]), sc2, nm2);
                     const float2 p = make_float2(ex2(e.x), ex2(e.y));
                     sp[(c >> 1) & 1] = add2(sp[(c >> 1) & 1], p);
                     pk[c / 2] = pack2<kBf16>(p.x, p.y);
+                    if constexpr (kBf16) {
+                        // p - bf16(p) is exact in fp32; widening bf16 is a 16-bit shift
+                        const float2 r = sub2(p, make_float2(__uint_as_float(pk[c / 2] << 16),
+                                                             __uint_as_float(pk[c / 2] & 0xffff0000u)));
+                        pl[c / 2] = pack2<true>(r.x, r.y);
+                    }
                 }
-                tmem_st8(tS + kTmemP + half * 32 + h * 8, pk);
+                tmem_st4(tS + kTmemP + half * 32 + h * 4, pk);
+                if constexpr (kBf16) tmem_st4(tS + kTmemPlo + half * 32 + h * 4, pl);
             }
             const float2 s01 = add2(sp[0], sp[1]);
             l = l * alpha + (s01.x + s01.y);

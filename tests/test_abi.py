@@ -69,9 +69,47 @@ def _decode(lib, **over):
     (dict(H=0), 1), (dict(H=6, Hkv=4), 1), (dict(S=-1), 1), (dict(ps=24), 1),
     (dict(B=8), 2), (dict(D=96), 2), (dict(H=34, Hkv=2), 2), (dict(q_dtype=0, kv_dtype=1), 2),
     (dict(kv_dtype=2, D=64), 2), (dict(kv_dtype=2, k_scale=0.0), 1), (dict(q_dtype=2), 2),
+    (dict(scale=float("inf")), 1), (dict(scale=float("-inf")), 1), (dict(scale=float("nan")), 1),
+    (dict(kv_dtype=2, k_scale=float("inf")), 1), (dict(kv_dtype=2, v_scale=float("inf")), 1),
+    (dict(kv_dtype=2, v_scale=float("nan")), 1),
 ])
 def test_decode_rejects_bad_arguments(lib, over, status):
+    """Host-side checks of pkv_paged_attn_decode, non-finite scales included: nothing is launched."""
     assert _decode(lib, **over) == status
+
+
+def test_static_workspace_call_checks_arguments_before_its_size(lib):
+    """The allocation-free decode call answers a bad argument with the same status as the ordinary
+    call, even when the (meaningless) request would also be too large for its array."""
+    f = lib.pkv_paged_attn_decode_static_ws
+    P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    f.argtypes = [P, P, I, P, P, I, F, F, P, I, P, I, I, I, I, I, I, I, F, I, P, P]
+    f.restype = I
+    big = 1 << 24                      # 16M tokens in 16-token partitions: far beyond the 64 MiB array
+    base = [P(16), P(16), 0, P(16), P(16), 0, 1.0, 1.0, P(16), big // 16, P(16), big, 64, 8, 2, 128, 16, 10, 0.1,
+            16, None, None]
+    assert f(*base) == 3               # well-formed: refused for its size
+    bad_q = list(base)
+    bad_q[1] = None
+    assert f(*bad_q) == 1
+    bad_scale = list(base)
+    bad_scale[18] = float("inf")
+    assert f(*bad_scale) == 1
+    bad_group = list(base)
+    bad_group[13], bad_group[14] = 34, 2
+    assert f(*bad_group) == 2
+
+
+def test_shared_prefix_rejects_an_unknown_plan(lib):
+    f = lib.pkv_paged_attn_decode_shared_prefix
+    P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    f.argtypes = [P, P, I, P, P, I, F, F, P, I, P, I, I, I, I, I, I, I, F, I, P, P, P, I, I, I, I, P, Z, P, P]
+    f.restype = I
+    args = [P(16), P(16), 0, P(16), P(16), 0, 1.0, 1.0, P(16), 4, P(16), 64, 2, 8, 2, 128, 16, 10, 0.1, 0,
+            P(16), P(16), P(16), 1, 2, 32, 0, P(256), 1 << 20, None, None]
+    for plan in (3, -1):
+        args[26] = plan
+        assert f(*args) == 1
 
 
 def test_decode_rejects_null_and_misaligned(lib):

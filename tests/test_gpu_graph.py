@@ -121,9 +121,7 @@ def test_prefill_graph_replays_with_new_inputs():
         torch.cuda.synchronize()
         assert int(err.item()) == 0
         oracle.reshape_and_cache(kb, vb, "bf16", kp_h, vp_h, "bf16", w.step_scatter.slots)
-        vmax = max([float(np.abs(oracle.decode_values(op.v, "bf16")).max()) for op in w.setup if op.slots.size] +
-                   [float(np.abs(oracle.decode_values(vb, "bf16")).max())])
         ref = oracle.paged_attn_prefill(qb, "bf16", kp_h, vp_h, "bf16", w.block_tables, w.context_lens,
                                         w.query_start, w.scale)
-        ok, rep = prefill_close(H.out_f64(out), ref, "bf16", vmax)
+        ok, rep = prefill_close(H.out_f64(out), ref, "bf16")
         assert ok, rep

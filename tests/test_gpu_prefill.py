@@ -6,8 +6,7 @@ f16 and bf16, whole prompts, chunks after earlier context that start inside a
 partially filled block, single-token chunks, empty chunks, chunk lengths that
 leave ragged query and key tiles, a long context, and logits wide enough that
 the running maximum moves many times.  The full-size workload is checked on
-sampled rows (each an oracle call of its own) and on properties that hold at
-any size.  Data-dependent errors (a bad block id, a chunk longer than its
+every row.  Data-dependent errors (a bad block id, a chunk longer than its
 context) must give NaN rows and the documented error bits while the other
 sequences stay correct.  A prefill of one-token chunks must agree with the
 decode kernel.  E4M3 caches go through the widening gather and the same
@@ -60,9 +59,9 @@ def test_prefill_matches_oracle(name):
     w = make_case(name)
     out, err, _, _ = H.gpu_prefill(w)
     assert err == 0
-    kp, vp, vmax = H.oracle_prefill_pools(w)
+    kp, vp = H.oracle_prefill_pools(w)
     ref = oracle_out(w, kp, vp)
-    ok, rep = prefill_close(H.out_f64(out), ref, w.dtype, vmax)
+    ok, rep = prefill_close(H.out_f64(out), ref, w.dtype)
     assert ok, (name, rep)
 
 
@@ -73,9 +72,9 @@ def test_wide_logits_move_the_running_maximum():
     q6 = torch.from_numpy(qf).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     out, err, _, _ = H.gpu_prefill(w, q_bits=q6)
     assert err == 0
-    kp, vp, vmax = H.oracle_prefill_pools(w)
+    kp, vp = H.oracle_prefill_pools(w)
     ref = oracle_out(w, kp, vp, q_bits=q6)
-    ok, rep = prefill_close(H.out_f64(out), ref, "bf16", vmax)
+    ok, rep = prefill_close(H.out_f64(out), ref, "bf16")
     assert ok, rep
 
 
@@ -88,9 +87,9 @@ def test_bad_block_id_gives_nan_rows_and_flag():
     o = H.out_f64(out)
     r0, r1 = int(w.query_start[1]), int(w.query_start[2])
     assert np.isnan(o[r0:r1]).any()              # the tiles that needed the block
-    kp, vp, vmax = H.oracle_prefill_pools(w)
+    kp, vp = H.oracle_prefill_pools(w)
     ref = oracle_out(w, kp, vp)
-    ok, rep = prefill_close(o[:r0], ref[:r0], "f16", vmax)   # sequence 0 untouched
+    ok, rep = prefill_close(o[:r0], ref[:r0], "f16")   # sequence 0 untouched
     assert ok, rep
 
 
@@ -103,9 +102,9 @@ def test_chunk_longer_than_context_is_flagged():
     o = H.out_f64(out)
     r0 = int(w.query_start[1])
     assert np.isnan(o[r0:]).all()
-    kp, vp, vmax = H.oracle_prefill_pools(w)
+    kp, vp = H.oracle_prefill_pools(w)
     ref = oracle_out(w, kp, vp)
-    ok, rep = prefill_close(o[:r0], ref[:r0], "bf16", vmax)
+    ok, rep = prefill_close(o[:r0], ref[:r0], "bf16")
     assert ok, rep
 
 
@@ -123,32 +122,21 @@ def test_single_token_chunks_agree_with_the_decode_kernel():
                         torch.from_numpy(w.context_lens).to(dev), float(w.scale),
                         max_context_len=int(w.context_lens.max()))
     torch.cuda.synchronize()
-    _, _, vmax = H.oracle_prefill_pools(w)
-    ok, rep = prefill_close(H.out_f64(out), H.out_f64(dec), "bf16", vmax)
+    ok, rep = prefill_close(H.out_f64(out), H.out_f64(dec), "bf16")
     assert ok, rep
 
 
-def test_full_size_sampled_rows():
-    """The full chunked-prefill workload: every output finite; sampled rows against the oracle
-    (first, last and random rows of every sequence, each an oracle call of its own)."""
+def test_full_size_every_row():
+    """The full chunked-prefill workload (16 sequences, 23,714 query rows x 32 heads): every output
+    row against the oracle, under the same rule as decode."""
     w = wl.make_prefill()
     out, err, _, _ = H.gpu_prefill(w)
     assert err == 0
     o = H.out_f64(out)
     assert np.isfinite(o).all()
-    kp, vp, vmax = H.oracle_prefill_pools(w)
-    rng = np.random.default_rng(11)
-    rows, refs = [], []
-    for s in range(w.num_seqs):
-        q0, q1 = int(w.query_start[s]), int(w.query_start[s + 1])
-        pick = {q0, q1 - 1, *rng.integers(q0, q1, size=2).tolist()}
-        for r in sorted(pick):
-            p = int(w.context_lens[s]) - (q1 - q0) + (r - q0)
-            ref = oracle.paged_attn_prefill(w.q[r:r + 1], w.dtype, kp, vp, w.dtype, w.block_tables[s:s + 1],
-                                            np.array([p + 1], np.int32), np.array([0, 1], np.int32), w.scale)
-            rows.append(r)
-            refs.append(ref[0])
-    ok, rep = prefill_close(o[rows], np.stack(refs), w.dtype, vmax)
+    kp, vp = H.oracle_prefill_pools(w)
+    ref = oracle_out(w, kp, vp)
+    ok, rep = prefill_close(o, ref, w.dtype)
     assert ok, rep
 
 

@@ -173,6 +173,5 @@ def test_prefix_cache_hit_then_partial_prefill_equals_full_prefill():
                              "bf16", pos.astype(np.int64))
     ref = oracle.paged_attn_prefill(q, "bf16", fk, fv, "bf16", np.arange(nblk, dtype=np.int32)[None],
                                     np.array([len(b)], np.int32), np.array([0, C], np.int32), np.float32(1 / np.sqrt(D)))
-    vmax = float(np.abs(oracle.decode_values(vtab, "bf16")).max())
-    ok, rep = prefill_close(H.out_f64(out), ref, "bf16", vmax)
+    ok, rep = prefill_close(H.out_f64(out), ref, "bf16")
     assert ok, rep

@@ -6,10 +6,10 @@ once it runs because cudaMalloc can synchronise the device.  For them the
 library keeps the split-context workspace in a device array of its own.
 This test calls that entry point through the C ABI, twice in a row on
 different workloads that both need the workspace, and checks each result
-against the ordinary entry point (given a caller-allocated workspace) with
-the comparison rule the other parity tests use.  It lives in a file that
-pytest collects last, so a run that stops at the first failure has already
-run every other test.
+against the float64 oracle and against the ordinary entry point (given a
+caller-allocated workspace) with the comparison rule the other parity tests
+use.  It lives in a file that pytest collects last, so a run that stops at
+the first failure has already run every other test.
 """
 import ctypes
 
@@ -77,8 +77,10 @@ def test_static_workspace_matches_caller_workspace_on_two_calls():
         assert call_static(f, w, t, out, err, ps) == 0
         torch.cuda.synchronize()
         assert int(err.item()) == 0
+        ok, rep = attention_close(H.out_f64(out), H.oracle_step(w)["out"], w.kv_dtype, w.q_dtype)
+        assert ok, (w.name, "against the oracle", rep)
         ok, rep = attention_close(H.out_f64(out), H.out_f64(ref), w.kv_dtype, w.q_dtype)
-        assert ok, (w.name, rep)
+        assert ok, (w.name, "against the ordinary entry point", rep)
 
 
 def test_static_workspace_rejects_oversized_requests():
