@@ -55,17 +55,17 @@ FALLBACK_HBM_GBS = 6650.0
 # for the decode kernel source it was measured on (sha256 prefix of decode.cu).
 NCU_TRAFFIC = {
     "opt13b": {"bytes_per_launch": 1_316_705_536, "kernel_sha": "05714f1368298826",
-               "capture": "profiles/paged_decode_kernel_opt13b.md (opt13b_compact: same sequences)"},
+               "capture": "ncu, opt13b_compact (the same sequences, pool cut to the blocks in use)"},
     "gqa": {"bytes_per_launch": 1_224_799_136, "kernel_sha": "05714f1368298826",
-            "capture": "profiles/paged_decode_kernel_gqa.md (gqa_compact: same sequences)"},
+            "capture": "ncu, gqa_compact (the same sequences, pool cut to the blocks in use)"},
     "fp8": {"bytes_per_launch": 1_118_479_160, "kernel_sha": "05714f1368298826",
-            "capture": "profiles/paged_decode_kernel_fp8.md (fp8_compact: same sequences, 512-token partitions)"},
+            "capture": "ncu, fp8_compact (the same sequences, 512-token partitions)"},
 }
 
 
 # the same for the prefill kernel (sha256 prefix of prefill.cu), on the prefill workload
 PREFILL_TRAFFIC = {"bytes_per_launch": 568_925_952, "kernel_sha": "538588bfa1f1bfab",
-                   "capture": "profiles/paged_prefill_kernel_prefill.md"}
+                   "capture": "ncu, prefill workload, paged_prefill_kernel"}
 
 
 def prefill_source_sha() -> str:
@@ -343,6 +343,14 @@ def run_prefill(args, rank, world, local_rank):
         end.record()
         barrier_sync(torch, dist_on)
     ms_step = max_over_ranks(torch, start.elapsed_time(end), dist_on) / K
+    # the prefill call's own rate: K calls back to back, events at both ends (the roofline's duration)
+    barrier_sync(torch, dist_on)
+    start.record()
+    for _ in range(K):
+        ps.prefill_op()
+    end.record()
+    barrier_sync(torch, dist_on)
+    pf_stream_ms = max_over_ranks(torch, start.elapsed_time(end), dist_on) / K
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     barrier_sync(torch, dist_on)
     for i in range(K):
@@ -384,7 +392,7 @@ def run_prefill(args, rank, world, local_rank):
     e2e_serial_ms = max_over_ranks(torch, s2.elapsed_time(e2), dist_on) / K
     e2e_ms = pipelined_e2e_ms(torch, dev, ps, pinned, args.warmup, K, dist_on)
     peak, peak_sus, kind = tensor_peak()
-    achieved = flops / (pf_ms * 1e-3) / 1e12
+    achieved = flops / (pf_stream_ms * 1e-3) / 1e12
     line = {
         "metric": PREFILL_METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
@@ -405,6 +413,7 @@ def run_prefill(args, rank, world, local_rank):
                                                                            w.num_tokens * w.num_heads * w.head_dim * 2 / 1e6),
                    "parallelism": f"dp{world}" if world > 1 else "single GPU"},
         "tokens_per_s": round(sum_over_ranks(torch, float(w.num_tokens), dist_on) / (ms_step * 1e-3), 1),
+        "prefill_ms_in_stream": round(pf_stream_ms, 5),
         "kernel_ms": {("paged_attn_prefill_fp8" if kv_fp8 else "paged_attn_prefill"): round(pf_ms, 5),
                       "reshape_and_cache": round(sc_ms, 5)},
         "roofline": {"bound": "tensor",
@@ -424,8 +433,8 @@ def run_prefill(args, rank, world, local_rank):
                 "serial_value": round(total_flops / (e2e_serial_ms * 1e-3) / 1e12, 2),
                 "serial_ms_per_step": round(e2e_serial_ms, 5)},
         "gpu_launches": (3 if kv_fp8 else 2) * K,
-        "timing": ("value: CUDA events around K back-to-back steps; kernel_ms and roofline: CUDA events "
-                   "around each call in a second run of K steps"),
+        "timing": ("value: CUDA events around K back-to-back steps; roofline: K prefill calls back to back in "
+                   "the same run (prefill_ms_in_stream); kernel_ms: CUDA events around each call in a third pass"),
         "clocks": clk.report(),
     }
     return line, w
@@ -681,30 +690,10 @@ def job_throughput(step_bytes_this_rank: float, ms_total_this_rank: float, steps
     return total / (ms_step * 1e-3) / 1e9, ms_step
 
 
-def run_ours(args, rank, world, local_rank):
-    import torch
-    dist_on = world > 1
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    w = wl.make(args.config)        # weak scaling: every rank runs a batch of the same shape
-    heads = args.shard == "heads" and world > 1
-    if heads:                       # strong scaling: one batch, each rank its share of the KV heads
-        w = wl.shard_heads(w, rank, world)
-    ps = w.partition_size if args.partition == "config" else (0 if args.partition == "auto" else int(args.partition))
-    ds = DeviceStep(w, dev, ps, prefix_aware=args.prefix_aware)
-    step_bytes = wl.step_algorithmic_bytes(w)
-    dec_bytes = wl.decode_algorithmic_bytes(w)
-    # the roofline counts each physical KV slot once: on shared prompts that is what must cross HBM
-    roof_bytes = wl.decode_distinct_bytes(w)
-
-    for _ in range(args.warmup):
-        ds.step()
-    barrier_sync(torch, dist_on)
-
-    K = args.steps
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    # timed region 1: K steps back to back (the kernels overlap their launches), for `value`
+def time_steps(torch, ds, K: int, dist_on: bool, local_rank: int):
+    """Device time of K back-to-back steps (no events between the kernels, so they overlap their
+    launches as a serving loop's do), with the clocks sampled meanwhile: (ms in total, clocks)."""
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank) as clk:
         barrier_sync(torch, dist_on)
         start.record()
@@ -712,8 +701,26 @@ def run_ours(args, rank, world, local_rank):
             ds.step()
         end.record()
         barrier_sync(torch, dist_on)
-    ms_total = start.elapsed_time(end)
-    # timed region 2: the same K steps with events around each call, for the per-kernel times
+    return start.elapsed_time(end), clk.report()
+
+
+def time_decode_stream(torch, ds, K: int, dist_on: bool) -> float:
+    """Milliseconds per decode call over K calls back to back (events only at both ends): the
+    dominant kernel's own rate, never more than the step that contains it, since each step
+    runs the same call plus the scatter (and copies)."""
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier_sync(torch, dist_on)
+    start.record()
+    for _ in range(K):
+        ds.decode_op()
+    end.record()
+    barrier_sync(torch, dist_on)
+    return max_over_ranks(torch, start.elapsed_time(end), dist_on) / K
+
+
+def time_each_call(torch, ds, K: int, dist_on: bool) -> dict:
+    """Mean milliseconds of each call with CUDA events around every call (these events keep
+    the kernels from overlapping, so the per-call times add up to more than a step)."""
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
     barrier_sync(torch, dist_on)
     for i in range(K):
@@ -726,13 +733,149 @@ def run_ours(args, rank, world, local_rank):
         ds.decode_op()
         e[3].record()
     barrier_sync(torch, dist_on)
-    dec_ms = [ev[i][2].elapsed_time(ev[i][3]) for i in range(K)]
-    sc_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
-    cp_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
+    mean = lambda a, b: sum(ev[i][a].elapsed_time(ev[i][b]) for i in range(K)) / K  # noqa: E731
+    return {"paged_attn_decode": round(mean(2, 3), 5), "reshape_and_cache": round(mean(1, 2), 5),
+            "copy_blocks": round(mean(0, 1), 5) if "pairs" in ds.d else None}
+
+
+def read_peak(torch, ds, reps: int = 5) -> float:
+    """Read-only HBM rate (GB/s) of a pass over this workload's K and V pools (pkv_stream_read),
+    timed with CUDA events on the launching stream: the denominator for a read-mostly kernel."""
+    from paged_kv_cache_324_b200 import binding as B
+    sink = torch.zeros(1, dtype=torch.int32, device=ds.k_pool.device)
+    pools = (ds.k_pool.view(torch.uint8).view(-1), ds.v_pool.view(torch.uint8).view(-1))
+    nbytes = sum(p.numel() for p in pools)
+    for _ in range(2):
+        for p in pools:
+            B.stream_read(p, sink)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s.record()
+    for _ in range(reps):
+        for p in pools:
+            B.stream_read(p, sink)
+    e.record()
+    torch.cuda.synchronize()
+    return nbytes * reps / (s.elapsed_time(e) * 1e-3) / 1e9, nbytes
+
+
+def traffic_for(name: str, partition_arg: str, prefix_aware: bool, heads: bool):
+    """ncu DRAM bytes of one decode call, if a capture of this exact kernel source exists."""
+    tr = NCU_TRAFFIC.get(name)
+    # the capture ran the plain decode at the workload's own partition size
+    if tr and tr.get("kernel_sha") == decode_source_sha() and partition_arg == "config" and not prefix_aware \
+            and not heads:
+        return tr["bytes_per_launch"]
+    return None
+
+
+def measure_decode(torch, w, dev, ps: int, prefix_aware: bool, K: int, warmup: int, dist_on: bool,
+                   local_rank: int, peak: float, peak_kind: str, rpeak: float, partition_arg: str = "config",
+                   heads: bool = False):
+    """One decode workload on this GPU: the step rate, the decode call's roofline, per-call times.
+    Returns (result dict, DeviceStep)."""
+    ds = DeviceStep(w, dev, ps, prefix_aware=prefix_aware)
+    step_bytes = wl.step_algorithmic_bytes(w)
+    # the roofline counts each physical KV slot once: on shared prompts that is what must cross HBM
+    roof_bytes = wl.decode_distinct_bytes(w)
+    for _ in range(warmup):
+        ds.step()
+    barrier_sync(torch, dist_on)
+    ms_total, clocks = time_steps(torch, ds, K, dist_on, local_rank)
+    dec_ms = time_decode_stream(torch, ds, K, dist_on)
+    kernel_ms = time_each_call(torch, ds, K, dist_on)
     assert int(ds.err.item()) == 0, "device error during the timed region"
     value, ms_step = job_throughput(step_bytes, ms_total, K, dist_on, torch)
+    achieved = roof_bytes / (dec_ms * 1e-3) / 1e9
+    res = {
+        "value": round(value, 2), "ms_per_step": round(ms_step, 5),
+        "sequences_per_s": round(sum_over_ranks(torch, float(w.num_seqs), dist_on) / (ms_step * 1e-3), 1),
+        "decode_ms_in_stream": round(dec_ms, 5), "kernel_ms": kernel_ms,
+        "roofline": {"bound": "hbm", "kernel": "paged_decode_kernel + decode_reduce_kernel",
+                     "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "peak_read": round(rpeak, 1), "frac_read": round(achieved / rpeak, 4),
+                     "traffic": traffic_for(w.name, partition_arg, prefix_aware, heads),
+                     "bytes_per_launch": roof_bytes,
+                     "bytes_counted": "distinct KV slots attended (each once) + q + out + table entries + lengths",
+                     "peak_kind": f"{peak_kind} (copy, burst)",
+                     "peak_read_kind": "measured in this run (pkv_stream_read over the K and V pools)",
+                     "duration": "decode_ms_in_stream: K decode calls back to back, CUDA events at both ends"},
+        "clocks": clocks,
+    }
+    return res, ds
+
+
+def config_summary(w, ds) -> dict:
+    plan = "plain"
+    if ds.prefix_aware:
+        plan = ds.B.shared_prefix_plan_used(ds.sp["units"], w.num_kv_heads, w.head_dim, w.kv_dtype,
+                                            ds.sp["max_prefix_len"])
+    return {"workload": w.description, "name": w.name, "num_seqs": w.num_seqs, "num_heads": w.num_heads,
+            "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "block_size": w.block_size,
+            "num_blocks": w.num_blocks, "max_context_len": w.max_context_len,
+            "total_context_tokens": int(w.context_lens.sum()), "partition_size": ds.partition,
+            "partition_rule": "automatic" if ds.partition_arg == 0 else "set by the workload or --partition",
+            "kv_dtype": w.kv_dtype,
+            "step": ("copy_blocks + " if "pairs" in ds.d else "") + "reshape_and_cache + " +
+                    ("paged_attn_decode_shared_prefix (plan: %s)" % plan if ds.prefix_aware else "paged_attn_decode"),
+            "step_bytes": wl.step_algorithmic_bytes(w), "decode_bytes": wl.decode_algorithmic_bytes(w),
+            "decode_distinct_bytes": wl.decode_distinct_bytes(w)}
+
+
+def l2_note(roof_bytes: int) -> str:
+    if roof_bytes > L2_BYTES:
+        return "no flush: each step reads %.2f GB of distinct KV, more than the 126 MB L2" % (roof_bytes / 1e9)
+    return ("no flush: the %.0f MB of distinct KV fit in the 126 MB L2, so repeated reads of shared blocks may "
+            "hit L2" % (roof_bytes / 1e6))
+
+
+#: the other decode workloads measured in the default run (name, shared-prefix call)
+CONFIG_ROWS = [("gqa", False), ("fp8", False), ("fp8_b32", False), ("prefix", False), ("prefix", True),
+               ("prefix_long", False), ("prefix_long", True)]
+
+
+def run_configs(args, torch, dev, dist_on, local_rank, peak, peak_kind, rpeak) -> dict:
+    """Every workload of CONFIG_ROWS, timed like the headline (K steps back to back, then the decode
+    call's stream), one after the other with the previous one's memory released."""
+    out = {}
+    for name, shared in CONFIG_ROWS:
+        w = wl.make(name)
+        ps = w.partition_size if args.partition == "config" else (0 if args.partition == "auto"
+                                                                  else int(args.partition))
+        res, ds = measure_decode(torch, w, dev, ps, shared, args.steps, args.warmup, dist_on, local_rank, peak,
+                                 peak_kind, rpeak, args.partition)
+        key = name + ("+shared_prefix_call" if shared else "")
+        res["config"] = config_summary(w, ds)
+        res["config"]["l2"] = l2_note(wl.decode_distinct_bytes(w))
+        res["gpu_launches"] = ds.launches_per_step() * args.steps
+        out[key] = res
+        del ds
+        torch.cuda.empty_cache()
+    return out
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    dist_on = world > 1
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = wl.make(args.config)        # weak scaling: every rank runs a batch of the same shape
+    heads = args.shard == "heads" and world > 1
+    if heads:                       # strong scaling: one batch, each rank its share of the KV heads
+        w = wl.shard_heads(w, rank, world)
+    ps = w.partition_size if args.partition == "config" else (0 if args.partition == "auto" else int(args.partition))
+    peak, peak_kind = hbm_peak()
+    K = args.steps
+    # the read-only denominator first, on this workload's pools (each rank its own)
+    probe = DeviceStep(w, dev, ps, prefix_aware=args.prefix_aware)
+    rpeak, rbytes = read_peak(torch, probe)
+    del probe
+    torch.cuda.empty_cache()
+    res, ds = measure_decode(torch, w, dev, ps, args.prefix_aware, K, args.warmup, dist_on, local_rank, peak,
+                             peak_kind, rpeak, args.partition, heads)
+    step_bytes = wl.step_algorithmic_bytes(w)
     total_bytes = sum_over_ranks(torch, float(step_bytes), dist_on)
-    seqs = sum_over_ranks(torch, float(w.num_seqs), dist_on)
+    ms_step = res["ms_per_step"]
 
     # end to end: the step's inputs from pinned host memory, the output back to the host
     def pin(a):
@@ -767,58 +910,40 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = pipelined_e2e_ms(torch, dev, ds, pinned, args.warmup, K, dist_on)
     e2e_value = total_bytes / (e2e_ms * 1e-3) / 1e9
     e2e_serial_value = total_bytes / (e2e_serial_ms * 1e-3) / 1e9
-
-    peak, peak_kind = hbm_peak()
-    dec_avg = sum(dec_ms) / K
-    achieved = roof_bytes / (dec_avg * 1e-3) / 1e9
-    traffic = None
-    tr = NCU_TRAFFIC.get(args.config)
-    # the capture ran the plain decode at the workload's own partition size
-    if (tr and tr.get("kernel_sha") == decode_source_sha() and args.partition == "config"
-            and not args.prefix_aware and not heads):
-        traffic = tr["bytes_per_launch"]
+    cfg = config_summary(w, ds)
+    cfg["l2"] = l2_note(wl.decode_distinct_bytes(w))
+    cfg["parallelism"] = (f"tp{world} (KV heads split, identical block tables)" if heads
+                          else f"dp{world}" if world > 1 else "single GPU")
+    roof = res["roofline"]
+    roof["peak_read_bytes"] = rbytes
     line = {
-        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
-        "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True,
+        "metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "strong" if heads else "weak", "vs_baseline": None,
         "dtype": w.kv_dtype if w.kv_dtype != "e4m3" else "e4m3 (KV), f16 (q/out), f32 accumulate",
         "data": "synthetic (seeded N(0,1) K/V/q; random-byte pool content in unwritten slots)",
-        "config": {
-            "workload": w.description, "name": w.name, "num_seqs": w.num_seqs, "num_heads": w.num_heads,
-            "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "block_size": w.block_size,
-            "num_blocks": w.num_blocks, "max_context_len": w.max_context_len,
-            "total_context_tokens": int(w.context_lens.sum()), "partition_size": ds.partition,
-            "partition_rule": "automatic" if ds.partition_arg == 0 else "set by the workload or --partition",
-            "step": ("copy_blocks + " if "pairs" in ds.d else "") + "reshape_and_cache + " +
-                    ("paged_attn_decode_shared_prefix" if ds.prefix_aware else "paged_attn_decode"),
-            "step_bytes": step_bytes, "decode_bytes": dec_bytes, "decode_distinct_bytes": roof_bytes,
-            "l2": (("no flush: each step reads %.2f GB of distinct KV, more than the 126 MB L2" % (roof_bytes / 1e9))
-                   if roof_bytes > L2_BYTES else
-                   ("no flush: the %.0f MB of distinct KV fit in the 126 MB L2, so repeated reads of shared "
-                    "blocks may hit L2" % (roof_bytes / 1e6))),
-            "parallelism": (f"tp{world} (KV heads split, identical block tables)" if heads
-                            else f"dp{world}" if world > 1 else "single GPU"),
-        },
-        "sequences_per_s": round((w.num_seqs if heads else seqs) / (ms_step * 1e-3), 1),
-        "pct_of_hbm_peak": round(100 * value / world / peak, 2),
-        "pct_of_nominal_8tbs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
-        "kernel_ms": {"paged_attn_decode": round(dec_avg, 5), "reshape_and_cache": round(sum(sc_ms) / K, 5),
-                      "copy_blocks": round(sum(cp_ms) / K, 5) if "pairs" in ds.d else None},
-        "roofline": {"bound": "hbm", "kernel": "paged_decode_kernel + decode_reduce_kernel",
-                     "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "bytes_per_launch": roof_bytes,
-                     "bytes_counted": "distinct KV slots attended (each once) + q + out + table entries + lengths",
-                     "peak_kind": f"{peak_kind} (copy, burst)"},
+        "config": cfg,
+        "sequences_per_s": round((w.num_seqs if heads else sum_over_ranks(torch, float(w.num_seqs), dist_on))
+                                 / (ms_step * 1e-3), 1),
+        "pct_of_hbm_peak": round(100 * res["value"] / world / peak, 2),
+        "pct_of_nominal_8tbs": round(100 * res["value"] / world / NOMINAL_HBM_GBS, 2),
+        "decode_ms_in_stream": res["decode_ms_in_stream"],
+        "kernel_ms": res["kernel_ms"],
+        "roofline": roof,
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "ms_per_step": round(e2e_ms, 5),
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "overlap": PIPELINE_NOTE,
                 "serial_value": round(e2e_serial_value, 2), "serial_ms_per_step": round(e2e_serial_ms, 5)},
         "gpu_launches": ds.launches_per_step() * K,
-        "timing": ("value: CUDA events around K back-to-back steps; kernel_ms and roofline: CUDA events "
-                   "around each call in a second run of K steps"),
-        "clocks": clk.report(),
+        "timing": ("value and ms_per_step: CUDA events around K back-to-back steps; roofline: K decode calls back "
+                   "to back in the same run (decode_ms_in_stream); kernel_ms: CUDA events around each call in a "
+                   "third pass (events between kernels stop their overlap, so those add up to more than a step)"),
+        "clocks": res["clocks"],
     }
+    del ds, pinned, dq
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_configs:
+        line["configs"] = run_configs(args, torch, dev, dist_on, local_rank, peak, peak_kind, rpeak)
     return line, w
 
 
@@ -900,6 +1025,9 @@ def main():
     ap.add_argument("--partition", default="config",
                     help="'config' (the workload's stated partition size, else automatic), 'auto', or tokens")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="decode workloads: time only --config (by default a single-GPU run also times the "
+                         "other decode workloads and reports them under 'configs')")
     ap.add_argument("--shard", default="sequences", choices=["sequences", "heads"],
                     help="decode under torchrun: each rank its own batch (weak scaling) or one batch with the "
                          "KV heads split over the ranks (strong scaling)")

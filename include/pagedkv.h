@@ -192,6 +192,13 @@ typedef enum {
     PKV_PREFIX_PLAN_PLAIN = 2
 } pkv_prefix_plan;
 
+/* The plan pkv_paged_attn_decode_shared_prefix carries out for these arguments:
+ * PKV_PREFIX_PLAN_SHARED (three launches: tail pass, prefix pass, merge) or
+ * PKV_PREFIX_PLAN_PLAIN (pkv_paged_attn_decode's one or two); -1 for an unknown
+ * plan.  Reads the current device's L2 size for PKV_PREFIX_PLAN_AUTO. */
+int pkv_shared_prefix_plan_used(int num_units, int num_kv_heads, int head_dim, pkv_dtype kv_dtype,
+                                int max_prefix_len, int plan);
+
 size_t pkv_shared_prefix_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
                                          pkv_dtype kv_dtype, int block_size, int max_context_len,
                                          int num_units, int max_prefix_len, int partition_size);
@@ -481,6 +488,18 @@ pkv_status pkv_bm_swap(pkv_block_manager* from, pkv_block_manager* to, const int
  * wait give up stops early), so clear the word after reading it.
  */
 pkv_status pkv_selftest_bounded_wait(uint32_t* device_error, unsigned timeout_us, void* stream);
+
+/*
+ * Measurement helper (no counterpart on the pages): reads every byte of a device
+ * buffer once and discards it, the read-only HBM rate that a read-mostly kernel
+ * such as pkv_paged_attn_decode can be held against (a copy's rate counts
+ * writes too).  buf: device pointer, 16-byte aligned; bytes: a multiple of 16;
+ * sink: device uint32 word, may be NULL (it is only written in the practically
+ * impossible case that the folded data equal a fixed constant, which keeps the
+ * loads from being optimised away).  Asynchronous on stream; PKV_ERR_ALIGNMENT
+ * for a misaligned buffer or size.
+ */
+pkv_status pkv_stream_read(const void* buf, size_t bytes, uint32_t* sink, void* stream);
 
 #ifdef __cplusplus
 }

@@ -337,6 +337,16 @@ def selftest_bounded_wait(device_error: torch.Tensor, timeout_us: int, stream=No
            "selftest_bounded_wait")
 
 
+def stream_read(buf: torch.Tensor, sink: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Read every byte of ``buf`` (a contiguous device tensor) once: the read-only HBM rate."""
+    if not buf.is_cuda or not buf.is_contiguous():
+        raise ValueError("buf must be a contiguous device tensor")
+    L = lib()
+    L.pkv_stream_read.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p]
+    _check(L.pkv_stream_read(ctypes.c_void_p(buf.data_ptr()), buf.numel() * buf.element_size(), _err(sink),
+                             _stream(stream)), "stream_read")
+
+
 class BlockManager:
     """Host-side block manager of the library (pkv_bm_* in include/pagedkv.h)."""
 
@@ -505,6 +515,18 @@ def shared_prefix_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, k
 
 #: pkv_prefix_plan codes
 PREFIX_PLANS = {"auto": 0, "shared": 1, "plain": 2}
+
+
+def shared_prefix_plan_used(num_units: int, num_kv_heads: int, head_dim: int, kv_dtype, max_prefix_len: int,
+                            plan: str = "auto") -> str:
+    """"shared" or "plain": what paged_attn_decode_shared_prefix does for these arguments."""
+    L = lib()
+    I = ctypes.c_int
+    L.pkv_shared_prefix_plan_used.argtypes = [I, I, I, I, I, I]
+    L.pkv_shared_prefix_plan_used.restype = I
+    r = L.pkv_shared_prefix_plan_used(num_units, num_kv_heads, head_dim, _kv_code(kv_dtype), max_prefix_len,
+                                      PREFIX_PLANS[plan])
+    return {1: "shared", 2: "plain"}[r]
 
 
 def paged_attn_decode_shared_prefix(out, q, k_pool, v_pool, block_tables, context_lens, scale, *,

@@ -453,11 +453,26 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
             const bool ok = hq < rows;
             const uint32_t* qrow = reinterpret_cast<const uint32_t*>(static_cast<const uint16_t*>(a.q) +
                                                                      row_of(ok ? hq : 0) * D);
+            if constexpr (Gm::E == 1) {
+                // permuted order: the lane's words of all k-steps are one 64-byte run of the row
+                // (words 16c .. 16c + 15), so four 16-byte loads fetch them
+                static_assert(Gm::kKsteps == 8, "E4M3 fragments assume head_dim 128");
+                const uint4* q4 = reinterpret_cast<const uint4*>(qrow) + 4 * c;
+                uint4 v[4];
 #pragma unroll
-            for (int ks = 0; ks < Gm::kKsteps; ++ks) {
-                const int d0 = Gm::qk_dim(c, ks);
-                qb[ks][nh][0] = ok ? __ldg(qrow + (d0 >> 1)) : 0u;
-                qb[ks][nh][1] = ok ? __ldg(qrow + ((d0 + Gm::kQkB1) >> 1)) : 0u;
+                for (int i = 0; i < 4; ++i) v[i] = ok ? __ldg(q4 + i) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                for (int ks = 0; ks < Gm::kKsteps; ++ks) {
+                    qb[ks][nh][0] = word(v[ks >> 1], 2 * (ks & 1));       // dims 32c + 4ks, +1
+                    qb[ks][nh][1] = word(v[ks >> 1], 2 * (ks & 1) + 1);   // dims 32c + 4ks + 2, +3
+                }
+            } else {
+#pragma unroll
+                for (int ks = 0; ks < Gm::kKsteps; ++ks) {
+                    const int d0 = Gm::qk_dim(c, ks);
+                    qb[ks][nh][0] = ok ? __ldg(qrow + (d0 >> 1)) : 0u;
+                    qb[ks][nh][1] = ok ? __ldg(qrow + ((d0 + Gm::kQkB1) >> 1)) : 0u;
+                }
             }
         }
         pdl_wait();   // outputs and partials are written only after the previous kernel
@@ -1090,6 +1105,20 @@ extern "C" size_t pkv_shared_prefix_workspace_bytes(int num_seqs, int num_heads,
     return pkv::partials_bytes(static_cast<size_t>(num_seqs) * num_heads * static_cast<size_t>(parts), head_dim);
 }
 
+// Automatic plan: when the shared prefixes, counted once per unit, fit in L2, the plain call's
+// repeated reads of them are L2 hits and its single pass beats the tail pass + prefix pass +
+// merge, so the plain call runs.
+extern "C" int pkv_shared_prefix_plan_used(int num_units, int num_kv_heads, int head_dim, pkv_dtype kv_dtype,
+                                           int max_prefix_len, int plan) {
+    if (plan != PKV_PREFIX_PLAN_AUTO && plan != PKV_PREFIX_PLAN_SHARED && plan != PKV_PREFIX_PLAN_PLAIN) return -1;
+    if (plan == PKV_PREFIX_PLAN_PLAIN || num_units <= 0 || max_prefix_len <= 0) return PKV_PREFIX_PLAN_PLAIN;
+    if (plan == PKV_PREFIX_PLAN_SHARED) return PKV_PREFIX_PLAN_SHARED;
+    const double per_token = 2.0 * num_kv_heads * head_dim * (kv_dtype == PKV_FP8_E4M3 ? 1 : 2);
+    return static_cast<double>(num_units) * max_prefix_len * per_token > static_cast<double>(pkv::l2_bytes())
+               ? PKV_PREFIX_PLAN_SHARED
+               : PKV_PREFIX_PLAN_PLAIN;
+}
+
 extern "C" pkv_status pkv_paged_attn_decode_shared_prefix(
     void* out, const void* q, pkv_dtype q_dtype, const void* k_pool, const void* v_pool, pkv_dtype kv_dtype,
     float k_scale, float v_scale, const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
@@ -1124,15 +1153,9 @@ extern "C" pkv_status pkv_paged_attn_decode_shared_prefix(
     if (!workspace || workspace_bytes < need) return PKV_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) & 255) return PKV_ERR_ALIGNMENT;
 
-    // Automatic plan: when the shared prefixes, counted once per unit, fit in L2, the plain call's
-    // repeated reads of them are L2 hits and its single pass beats the prefix pass + tail pass +
-    // merge; the plain call then runs (its workspace is never larger than this one's).
-    bool shared = num_units > 0 && p_pre > 0 && plan != PKV_PREFIX_PLAN_PLAIN;
-    if (shared && plan == PKV_PREFIX_PLAN_AUTO) {
-        const double per_token = 2.0 * num_kv_heads * head_dim * (kv_dtype == PKV_FP8_E4M3 ? 1 : 2);
-        shared = static_cast<double>(num_units) * max_prefix_len * per_token > static_cast<double>(l2_bytes());
-    }
-    if (!shared)
+    // the plain call's workspace is never larger than this one's
+    if (pkv_shared_prefix_plan_used(num_units, num_kv_heads, head_dim, kv_dtype, max_prefix_len, plan) !=
+        PKV_PREFIX_PLAN_SHARED)
         return pkv_paged_attn_decode(out, q, q_dtype, k_pool, v_pool, kv_dtype, k_scale, v_scale, block_tables,
                                      max_blocks_per_seq, context_lens, max_context_len, num_seqs, num_heads,
                                      num_kv_heads, head_dim, block_size, num_blocks, scale, partition_size,

@@ -37,7 +37,11 @@
 //              with tcgen05.st (bf16: also the residual P - bf16(P) into the
 //              lower half, so that P.V sees ~16 significant bits of every
 //              weight, as a 16-bit f16 P's 11 bits nearly do), and rescale O in
-//              TMEM when the maximum moves; finally O / l.
+//              TMEM when the maximum moves; finally O / l, written into the
+//              query tile's own shared memory (free by then) and sent out by
+//              warp 0 with one TMA store per 64-column chunk, so that whole
+//              128-byte rows reach HBM (a tile cut short by the chunk's end is
+//              stored row by row instead).
 // While tile A's softmax works on S_A(j+1), the tensor core computes PV_B(j)
 // and S_B(j+1), and the other way round.
 //
@@ -284,6 +288,14 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
         : "memory");
 }
 
+// Shared memory -> global through a tensor map (bulk-group completion).
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(c2), "r"(src)
+                 : "memory");
+}
+
 __device__ __forceinline__ uint64_t l2_policy_evict_last() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
@@ -339,7 +351,8 @@ __device__ __forceinline__ bool warp_wait_bar(uint32_t bar, uint32_t parity, Cta
 template <int D, int BS, bool kBf16>
 __global__ void __launch_bounds__(kPThreads, 1)
 paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
-                     const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap) {
+                     const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                     const __grid_constant__ CUtensorMap omap) {
     using Gm = PGeo<D>;
     constexpr int kTB = kKeys / BS;                  // blocks per key tile
     constexpr uint32_t kBoxBytes = BS * 128;         // one block x one 64-column chunk
@@ -671,10 +684,17 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
         tc_fence_after();
         // every lane takes part in the warp-wide TMEM loads; only rows of the chunk are stored
         const bool live = tq < rows_cta;
-        const bool nan_out = !ok || flags.bad || *reinterpret_cast<volatile int*>(&flags.abort);
+        const bool aborted = *reinterpret_cast<volatile int*>(&flags.abort) != 0;
+        const bool nan_out = !ok || flags.bad || aborted;
+        // a query tile with all TQ tokens goes through its Q tile's shared memory (free now: the
+        // last S product that read it has completed) and one TMA store per 64-column chunk, so
+        // that whole 128-byte rows reach HBM; a partial tile (or a CTA that gave up a wait, whose
+        // copies may not have landed) stores its rows directly
+        const bool staged = (t + 1) * TQ <= rows_cta && !aborted;
         uint16_t* orow = reinterpret_cast<uint16_t*>(a.out) +
                          (static_cast<size_t>(q0 + t0 + (live ? tq : 0)) * a.num_heads + kvh * G + row % G) * D +
                          half * kOCols;
+        uint8_t* srow_g = smem + Gm::kQ + t * Gm::kTile + row * 128;   // this row of the Q tile (generic)
         const float inv = 1.f / (red[my_ntk & 1][t][0][row] + red[my_ntk & 1][t][1][row]);
 #pragma unroll
         for (int c = 0; c < kOCols / 32; ++c) {
@@ -686,14 +706,22 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
                 for (int i = 0; i < 16; ++i)
                     w[i] = nan_out ? (kBf16 ? 0x7FC07FC0u : 0x7E007E00u)
                                    : pack2<kBf16>(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
-                uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+                // staged: 16-byte units of the 64-column chunk in the 128-byte swizzle the Q tile was
+                // loaded with (row = TMEM lane: token-major, head-minor); else the row in global memory
+                const int col = half * kOCols + c * 32;
+                uint8_t* sbase_c = srow_g + (col / 64) * kChunkBytes;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                for (int i = 0; i < 4; ++i) {
+                    uint4* dst = staged ? reinterpret_cast<uint4*>(sbase_c + ((((col % 64) / 8 + i) ^ (row & 7)) << 4))
+                                        : reinterpret_cast<uint4*>(orow + c * 32) + i;
+                    *dst = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                }
             }
         }
+        fence_proxy_async_smem();   // the staged rows become visible to the TMA store
         tc_fence_before();
         __syncthreads();
-        return;   // warp 1 frees TMEM after the second barrier
+        return;   // warp 1 frees TMEM after the second barrier, warp 0 stores the staged tiles
     }
     // producer and MMA warps: meet the softmax warps at both barriers
     pdl_trigger();
@@ -701,6 +729,21 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
     __syncthreads();
     __syncthreads();
     tc_fence_after();
+    if (warp == 0 && lane == 0 && !*reinterpret_cast<volatile int*>(&flags.abort)) {
+        int stores = 0;
+#pragma unroll
+        for (int t = 0; t < kTiles; ++t)
+            if ((t + 1) * TQ <= rows_cta) {
+#pragma unroll
+                for (int c = 0; c < Gm::kChunks; ++c)
+                    tma_store_3d(&omap, sQ + t * Gm::kTile + c * kChunkBytes, c * 64, kvh * G, q0 + t0 + t * TQ);
+                ++stores;
+            }
+        if (stores) {
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");   // writes done before the CTA exits
+        }
+    }
     if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
                                 : "memory");
 }
@@ -741,19 +784,20 @@ bool encode_pool_map16(CUtensorMap* map, const void* pool, int head_dim, int blo
 
 template <int D, int BS, bool kBf16>
 pkv_status launch_prefill(const PrefillArgs& a, const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm,
-                          dim3 grid, cudaStream_t st) {
+                          const CUtensorMap& om, dim3 grid, cudaStream_t st) {
     auto kern = paged_prefill_kernel<D, BS, kBf16>;
     const uint32_t smem = PGeo<D>::kSmemBytes;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return PKV_ERR_CUDA;
-    return launch_pdl(kern, grid, dim3(kPThreads), smem, st, a, qm, km, vm) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+    return launch_pdl(kern, grid, dim3(kPThreads), smem, st, a, qm, km, vm, om) == cudaSuccess ? PKV_OK
+                                                                                             : PKV_ERR_CUDA;
 }
 
 template <int D, int BS>
 pkv_status dispatch_dtype(bool bf16, const PrefillArgs& a, const CUtensorMap& qm, const CUtensorMap& km,
-                          const CUtensorMap& vm, dim3 grid, cudaStream_t st) {
-    return bf16 ? launch_prefill<D, BS, true>(a, qm, km, vm, grid, st)
-                : launch_prefill<D, BS, false>(a, qm, km, vm, grid, st);
+                          const CUtensorMap& vm, const CUtensorMap& om, dim3 grid, cudaStream_t st) {
+    return bf16 ? launch_prefill<D, BS, true>(a, qm, km, vm, om, grid, st)
+                : launch_prefill<D, BS, false>(a, qm, km, vm, om, grid, st);
 }
 
 }  // namespace
@@ -800,16 +844,18 @@ extern "C" pkv_status pkv_paged_attn_prefill(void* out, const void* q, pkv_dtype
     alignas(64) CUtensorMap qm;
     alignas(64) CUtensorMap km;
     alignas(64) CUtensorMap vm;
+    alignas(64) CUtensorMap om;   // the output has q's layout, so it is stored with q's box
     if (!encode_q_map(&qm, q, head_dim, num_heads, num_tokens, G) ||
         !encode_pool_map16(&km, k_pool, head_dim, block_size, num_kv_heads, num_blocks) ||
-        !encode_pool_map16(&vm, v_pool, head_dim, block_size, num_kv_heads, num_blocks))
+        !encode_pool_map16(&vm, v_pool, head_dim, block_size, num_kv_heads, num_blocks) ||
+        !encode_q_map(&om, out, head_dim, num_heads, num_tokens, G))
         return PKV_ERR_CUDA;
     const dim3 grid(static_cast<unsigned>(tiles), static_cast<unsigned>(num_kv_heads), static_cast<unsigned>(num_seqs));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const bool bf16 = dtype == PKV_BF16;
     if (head_dim == 128)
-        return block_size == 16 ? dispatch_dtype<128, 16>(bf16, a, qm, km, vm, grid, st)
-                                : dispatch_dtype<128, 32>(bf16, a, qm, km, vm, grid, st);
-    return block_size == 16 ? dispatch_dtype<64, 16>(bf16, a, qm, km, vm, grid, st)
-                            : dispatch_dtype<64, 32>(bf16, a, qm, km, vm, grid, st);
+        return block_size == 16 ? dispatch_dtype<128, 16>(bf16, a, qm, km, vm, om, grid, st)
+                                : dispatch_dtype<128, 32>(bf16, a, qm, km, vm, om, grid, st);
+    return block_size == 16 ? dispatch_dtype<64, 16>(bf16, a, qm, km, vm, om, grid, st)
+                            : dispatch_dtype<64, 32>(bf16, a, qm, km, vm, om, grid, st);
 }

@@ -171,3 +171,15 @@ def test_workspace_size_rules(lib):
     assert B.decode_partition_size(16, 8, 128, "e4m3", 16, 32768, 0) == 2048
     # ... shrunk when there are few work units, never below 4 blocks
     assert B.decode_partition_size(4, 8, 64, "f16", 16, 256, 0) == 64
+
+
+def test_stream_read_checks_its_buffer(lib):
+    """The read-only measurement helper refuses a misaligned buffer or size before launching."""
+    P = ctypes.c_void_p
+    f = lib.pkv_stream_read
+    f.argtypes = [P, ctypes.c_size_t, P, P]
+    assert f(P(16), 0, None, None) == 0                 # nothing to read
+    assert f(None, 64, None, None) == 1
+    assert f(P(24), 64, None, None) == 5                # buffer not 16-byte aligned
+    assert f(P(16), 40, None, None) == 5                # size not a multiple of 16
+    assert f(P(16), 64, P(18), None) == 5               # misaligned sink word
