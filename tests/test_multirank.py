@@ -78,3 +78,41 @@ def test_cpu_baseline_sample_reports_a_one_core_figure():
     n, nbytes, el, cores, (n1, b1, el1) = bench.cpu_oracle_sample(w, 0.05, one_core_s=0.05)
     assert n >= 1 and nbytes == n * wl.step_algorithmic_bytes(w) and el > 0 and cores >= 1
     assert 1 <= n1 <= w.num_seqs and b1 > 0 and el1 > 0
+
+
+def _sharded_worker(rank, world, port, q):
+    """One rank of a head-sharded decode: its share of the KV heads (identical block tables), its
+    outputs computed alone, then gathered over gloo the way the ranks' outputs would be."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from paged_kv_cache_324_b200 import workload as wl
+        from tests import harness as H
+        w = wl.make("gqa", small=True)
+        sh = wl.shard_heads(w, rank, world)
+        out = torch.from_numpy(H.oracle_step(sh)["out"])
+        parts = [torch.empty_like(out) for _ in range(world)]
+        dist.all_gather(parts, out)
+        if rank == 0:
+            q.put(torch.cat(parts, dim=1).numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_with_head_shards_reassemble_the_whole_batch():
+    """Two processes, each holding half of the KV heads: their outputs side by side equal the
+    single-process result bit for bit (the path shards with no exchange inside attention)."""
+    import numpy as np
+    from paged_kv_cache_324_b200 import workload as wl
+    from tests import harness as H
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_sharded_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = q.get(timeout=300)
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    assert np.array_equal(got, H.oracle_step(wl.make("gqa", small=True))["out"])
