@@ -690,32 +690,78 @@ def job_throughput(step_bytes_this_rank: float, ms_total_this_rank: float, steps
     return total / (ms_step * 1e-3) / 1e9, ms_step
 
 
-def time_steps(torch, ds, K: int, dist_on: bool, local_rank: int):
-    """Device time of K back-to-back steps (no events between the kernels, so they overlap their
-    launches as a serving loop's do), with the clocks sampled meanwhile: (ms in total, clocks)."""
+def capture(torch, ds, fn, K: int):
+    """One CUDA graph of K calls of fn() (the library's launches on a capturing side stream), as a
+    serving loop replays a step; the kernels keep their programmatic-dependent-launch edges."""
+    side = torch.cuda.Stream(ds.dev)
+    side.wait_stream(torch.cuda.current_stream(ds.dev))
+    saved = ds.stream
+    ds.stream = side
+    try:
+        with torch.cuda.stream(side):
+            fn()                                   # one eager call on the side stream before capture
+        torch.cuda.current_stream(ds.dev).wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            for _ in range(K):
+                fn()
+    finally:
+        ds.stream = saved
+    torch.cuda.synchronize(ds.dev)
+    return g
+
+
+def time_graph(torch, g, dist_on: bool, local_rank: int = None):
+    """Device time (ms) of one replay, CUDA events on the stream the replay is launched on, with the
+    clocks sampled meanwhile when local_rank is given: (ms, clocks or None)."""
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local_rank) as clk:
+    g.replay()                                     # warm: the graph's first launch uploads it
+    barrier_sync(torch, dist_on)
+    clk = ClockSampler(local_rank) if local_rank is not None else None
+    if clk:
+        clk.__enter__()
+    try:
         barrier_sync(torch, dist_on)
         start.record()
-        for _ in range(K):
-            ds.step()
+        g.replay()
         end.record()
         barrier_sync(torch, dist_on)
-    return start.elapsed_time(end), clk.report()
+    finally:
+        if clk:
+            clk.__exit__(None, None, None)
+    return start.elapsed_time(end), (clk.report() if clk else None)
 
 
-def time_decode_stream(torch, ds, K: int, dist_on: bool) -> float:
-    """Milliseconds per decode call over K calls back to back (events only at both ends): the
-    dominant kernel's own rate, never more than the step that contains it, since each step
-    runs the same call plus the scatter (and copies)."""
+def time_steps(torch, ds, K: int, dist_on: bool, local_rank: int):
+    """Device time of K steps replayed from one CUDA graph (no host launch cost between kernels, and
+    no events between them, so they overlap as a serving loop's do), with the clocks sampled
+    meanwhile: (ms in total, clocks)."""
+    g = capture(torch, ds, ds.step, K)
+    ms, clocks = time_graph(torch, g, dist_on, local_rank)
+    del g
+    return ms, clocks
+
+
+def time_steps_eager(torch, ds, K: int, dist_on: bool) -> float:
+    """The same K steps launched one by one from Python (ms in total, max over ranks)."""
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier_sync(torch, dist_on)
     start.record()
     for _ in range(K):
-        ds.decode_op()
+        ds.step()
     end.record()
     barrier_sync(torch, dist_on)
-    return max_over_ranks(torch, start.elapsed_time(end), dist_on) / K
+    return max_over_ranks(torch, start.elapsed_time(end), dist_on)
+
+
+def time_decode_stream(torch, ds, K: int, dist_on: bool) -> float:
+    """Milliseconds per decode call over K calls back to back, replayed from one CUDA graph (events
+    only at both ends): the dominant kernel's own rate, never more than the step that contains
+    it, since each step runs the same call plus the scatter (and copies)."""
+    g = capture(torch, ds, ds.decode_op, K)
+    ms, _ = time_graph(torch, g, dist_on)
+    del g
+    return max_over_ranks(torch, ms, dist_on) / K
 
 
 def time_each_call(torch, ds, K: int, dist_on: bool) -> dict:
@@ -782,13 +828,14 @@ def measure_decode(torch, w, dev, ps: int, prefix_aware: bool, K: int, warmup: i
         ds.step()
     barrier_sync(torch, dist_on)
     ms_total, clocks = time_steps(torch, ds, K, dist_on, local_rank)
+    eager_ms = time_steps_eager(torch, ds, K, dist_on) / K
     dec_ms = time_decode_stream(torch, ds, K, dist_on)
     kernel_ms = time_each_call(torch, ds, K, dist_on)
     assert int(ds.err.item()) == 0, "device error during the timed region"
     value, ms_step = job_throughput(step_bytes, ms_total, K, dist_on, torch)
     achieved = roof_bytes / (dec_ms * 1e-3) / 1e9
     res = {
-        "value": round(value, 2), "ms_per_step": round(ms_step, 5),
+        "value": round(value, 2), "ms_per_step": round(ms_step, 5), "eager_ms_per_step": round(eager_ms, 5),
         "sequences_per_s": round(sum_over_ranks(torch, float(w.num_seqs), dist_on) / (ms_step * 1e-3), 1),
         "decode_ms_in_stream": round(dec_ms, 5), "kernel_ms": kernel_ms,
         "roofline": {"bound": "hbm", "kernel": "paged_decode_kernel + decode_reduce_kernel",
@@ -799,7 +846,8 @@ def measure_decode(torch, w, dev, ps: int, prefix_aware: bool, K: int, warmup: i
                      "bytes_counted": "distinct KV slots attended (each once) + q + out + table entries + lengths",
                      "peak_kind": f"{peak_kind} (copy, burst)",
                      "peak_read_kind": "measured in this run (pkv_stream_read over the K and V pools)",
-                     "duration": "decode_ms_in_stream: K decode calls back to back, CUDA events at both ends"},
+                     "duration": "decode_ms_in_stream: K decode calls back to back from one CUDA graph, CUDA "
+                                 "events at both ends"},
         "clocks": clocks,
     }
     return res, ds
@@ -927,6 +975,7 @@ def run_ours(args, rank, world, local_rank):
                                  / (ms_step * 1e-3), 1),
         "pct_of_hbm_peak": round(100 * res["value"] / world / peak, 2),
         "pct_of_nominal_8tbs": round(100 * res["value"] / world / NOMINAL_HBM_GBS, 2),
+        "eager_ms_per_step": res["eager_ms_per_step"],
         "decode_ms_in_stream": res["decode_ms_in_stream"],
         "kernel_ms": res["kernel_ms"],
         "roofline": roof,
@@ -935,9 +984,11 @@ def run_ours(args, rank, world, local_rank):
                 "overlap": PIPELINE_NOTE,
                 "serial_value": round(e2e_serial_value, 2), "serial_ms_per_step": round(e2e_serial_ms, 5)},
         "gpu_launches": ds.launches_per_step() * K,
-        "timing": ("value and ms_per_step: CUDA events around K back-to-back steps; roofline: K decode calls back "
-                   "to back in the same run (decode_ms_in_stream); kernel_ms: CUDA events around each call in a "
-                   "third pass (events between kernels stop their overlap, so those add up to more than a step)"),
+        "timing": ("value and ms_per_step: CUDA events around one replay of a CUDA graph holding K steps (as a "
+                   "serving loop replays its step; eager_ms_per_step: the same K steps launched one by one from "
+                   "Python); roofline: K decode calls back to back from one graph in the same run "
+                   "(decode_ms_in_stream); kernel_ms: CUDA events around each call in a further pass (events "
+                   "between kernels stop their overlap, so those add up to more than a step)"),
         "clocks": res["clocks"],
     }
     del ds, pinned, dq

@@ -271,8 +271,11 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
     const bool prefix_pass = a.unit_seqs != nullptr;
     int rows = G, L, start = 0, tseq = z;
     bool bad_len;
-    // Every CTA passes pdl_wait() before it exits, so that a grid only completes after the
-    // kernel before it on the stream has: the merge relies on that ordering through both passes.
+    // A grid must not complete before the kernel ahead of it on the stream has (the merge, and
+    // the next call, rely on that ordering through both passes): CTAs with work pass pdl_wait(),
+    // and of the CTAs that leave early, CTA (0, 0, 0) waits too, so at least one CTA of every
+    // grid does; the others leave at once and free their slots.
+    const bool first_cta = blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0;
     if (prefix_pass) {
         // members: valid sequence ids packed first, -1 pads after them; each member's own prefix
         // length must be the unit's (seq_start holds seq_prefix_len here)
@@ -295,7 +298,7 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
                   L > a.max_prefix_len;
         if (bad_len || L == 0 || grid_timed_out(a.err)) {
             if (bad_len && part == 0 && threadIdx.x == 0) raise_error(a.err, PKV_DEVERR_CONTEXT_LEN);
-            pdl_wait();
+            if (first_cta) pdl_wait();
             return;   // the members' prefix slots keep the tail pass's marker: their merges give NaN
         }
     } else {
@@ -316,12 +319,14 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
         }
         const bool give_up = grid_timed_out(a.err);
         if (bad_len || L == 0 || give_up) {
-            pdl_wait();
             if (part == 0 && (start == 0 || bad_len)) {
+                pdl_wait();
                 if (bad_len && threadIdx.x == 0) raise_error(a.err, PKV_DEVERR_CONTEXT_LEN);
                 const float v = (bad_len || give_up) ? __int_as_float(0x7fc00000) : 0.f;
                 const size_t row0 = static_cast<size_t>(z) * H + static_cast<size_t>(kvh) * G;
                 for (int e = threadIdx.x; e < G * D; e += kThreads) store_out<kQBf16>(a.out, row0 * D + e, v);
+            } else if (first_cta) {
+                pdl_wait();
             }
             return;
         }
@@ -336,7 +341,7 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
     const int PS = a.partition_size;
     const int nparts = (L + PS - 1) / PS;
     if (part >= nparts) {
-        pdl_wait();
+        if (first_cta) pdl_wait();
         return;
     }
     const int tok_begin = part * PS;

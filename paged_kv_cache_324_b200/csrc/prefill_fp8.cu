@@ -43,13 +43,13 @@ __device__ __forceinline__ uint32_t scaled_pair(uint32_t f16x2, float s) {
     }
 }
 
-// 16 E4M3 bytes -> 16 values of the query's type, times `s` (s = 1 for K: exact).
+// 8 E4M3 bytes -> 8 values of the query's type (one 16-byte vector), times `s` (s = 1 for K: exact).
 template <bool kBf16, bool kScale>
-__device__ __forceinline__ void widen16(const uint4& x, float s, uint4& lo, uint4& hi) {
-    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-    uint32_t o[8];
+__device__ __forceinline__ uint4 widen8(const uint2& x, float s) {
+    const uint32_t w[2] = {x.x, x.y};
+    uint32_t o[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 2; ++i) {
         const uint32_t a = e4m3x2_to_f16x2(static_cast<uint16_t>(w[i] & 0xffffu));
         const uint32_t b = e4m3x2_to_f16x2(static_cast<uint16_t>(w[i] >> 16));
         if constexpr (!kScale && !kBf16) {
@@ -60,25 +60,26 @@ __device__ __forceinline__ void widen16(const uint4& x, float s, uint4& lo, uint
             o[2 * i + 1] = scaled_pair<kBf16>(b, kScale ? s : 1.f);
         }
     }
-    lo = make_uint4(o[0], o[1], o[2], o[3]);
-    hi = make_uint4(o[4], o[5], o[6], o[7]);
+    return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// Flat index over (sequence s, table slot j, 16-byte vector of the block): block s * maxb + j of
-// the workspace pools receives the widened block block_tables[s][j], for j < ceil(L_s / B).
+// Flat index over (sequence s, table slot j, 8-byte unit of the E4M3 block): block s * maxb + j
+// of the workspace pools receives the widened block block_tables[s][j], for j < ceil(L_s / B).
+// Each thread reads 8 bytes and writes the 16-byte vector they widen to, so a warp's loads and
+// stores each cover one contiguous run (256 and 512 bytes).
 template <bool kBf16>
 __global__ void __launch_bounds__(kWidenThreads)
-widen_blocks_kernel(const uint4* __restrict__ k_pool, const uint4* __restrict__ v_pool, uint4* __restrict__ wk,
+widen_blocks_kernel(const uint2* __restrict__ k_pool, const uint2* __restrict__ v_pool, uint4* __restrict__ wk,
                     uint4* __restrict__ wv, int32_t* __restrict__ wtab, const int32_t* __restrict__ tables,
-                    const int32_t* __restrict__ lens, int num_seqs, int maxb, long long vec_per_block,
+                    const int32_t* __restrict__ lens, int num_seqs, int maxb, long long units_per_block,
                     int block_size, int num_blocks, float v_scale, uint32_t* err) {
     pdl_trigger();
     pdl_wait();   // the pool may still be written by the previous kernel (the chunk's scatter)
-    const long long total = static_cast<long long>(num_seqs) * maxb * vec_per_block;
+    const long long total = static_cast<long long>(num_seqs) * maxb * units_per_block;
     for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
          i += static_cast<long long>(gridDim.x) * blockDim.x) {
-        const long long blk = i / vec_per_block;
-        const long long e = i - blk * vec_per_block;
+        const long long blk = i / units_per_block;
+        const long long e = i - blk * units_per_block;
         const int s = static_cast<int>(blk / maxb), j = static_cast<int>(blk - static_cast<long long>(s) * maxb);
         const int L = __ldg(lens + s);
         const long long cap = static_cast<long long>(maxb) * block_size;
@@ -91,14 +92,9 @@ widen_blocks_kernel(const uint4* __restrict__ k_pool, const uint4* __restrict__ 
             if (bad) raise_error(err, PKV_DEVERR_BLOCK_ID);
         }
         if (bad) continue;
-        const long long src = static_cast<long long>(pid) * vec_per_block + e;
-        uint4 lo, hi;
-        widen16<kBf16, false>(k_pool[src], 1.f, lo, hi);
-        wk[2 * i] = lo;
-        wk[2 * i + 1] = hi;
-        widen16<kBf16, true>(v_pool[src], v_scale, lo, hi);
-        wv[2 * i] = lo;
-        wv[2 * i + 1] = hi;
+        const long long src = static_cast<long long>(pid) * units_per_block + e;
+        wk[i] = widen8<kBf16, false>(k_pool[src], 1.f);
+        wv[i] = widen8<kBf16, true>(v_pool[src], v_scale);
     }
 }
 
@@ -156,17 +152,18 @@ extern "C" pkv_status pkv_paged_attn_prefill_fp8(void* out, const void* q, pkv_d
     void* wk = ws;
     void* wv = ws + pool;
     int32_t* wtab = reinterpret_cast<int32_t*>(ws + 2 * pool);
-    const long long vec_per_block = static_cast<long long>(num_kv_heads) * block_size * head_dim / 16;
-    const long long total = static_cast<long long>(blocks) * vec_per_block;
+    // 8-byte units of an E4M3 block (head_dim 64 or 128: whole units)
+    const long long units_per_block = static_cast<long long>(num_kv_heads) * block_size * head_dim / 8;
+    const long long total = static_cast<long long>(blocks) * units_per_block;
     long long grid = (total + kWidenThreads - 1) / kWidenThreads;
     const long long cap = static_cast<long long>(num_sms()) * 8;
     if (grid > cap) grid = cap;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     auto launch = [&](auto kern) {
         return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(kWidenThreads), 0, st,
-                          static_cast<const uint4*>(k_pool), static_cast<const uint4*>(v_pool),
+                          static_cast<const uint2*>(k_pool), static_cast<const uint2*>(v_pool),
                           static_cast<uint4*>(wk), static_cast<uint4*>(wv), wtab, block_tables, context_lens, num_seqs,
-                          max_blocks_per_seq, vec_per_block, block_size, num_blocks, v_scale, device_error);
+                          max_blocks_per_seq, units_per_block, block_size, num_blocks, v_scale, device_error);
     };
     const cudaError_t e = q_dtype == PKV_BF16 ? launch(widen_blocks_kernel<true>) : launch(widen_blocks_kernel<false>);
     if (e != cudaSuccess) return PKV_ERR_CUDA;
