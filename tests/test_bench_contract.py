@@ -87,3 +87,24 @@ def test_reference_arm_runs_on_rank_zero_only():
         outs.append([ln for ln in r.stdout.splitlines() if ln.strip()])
     assert len(outs[0]) == 1 and json.loads(outs[0][0])["n_gpus"] == 2
     assert outs[1] == []
+
+
+def test_config_rows_name_decode_workloads():
+    """Every workload the default run times under "configs" is a decode workload the generator knows,
+    and the shared-prefix rows are the ones with shared prompts."""
+    import bench
+    from paged_kv_cache_324_b200 import workload as wl
+    names = set(wl.NAMES) | set(wl.EXTRA_NAMES)
+    assert bench.CONFIG_ROWS
+    for name, shared in bench.CONFIG_ROWS:
+        assert name in names, name
+        if shared:
+            assert name.startswith("prefix")
+    # the large-batch rows the 75%-of-HBM target names are among them
+    assert {"gqa", "fp8", "fp8_b32"} <= {n for n, _ in bench.CONFIG_ROWS}
+
+
+def test_l2_note_names_the_regime():
+    import bench
+    assert "more than the 126 MB L2" in bench.l2_note(2 * 10 ** 9)
+    assert "fit in the 126 MB L2" in bench.l2_note(50 * 10 ** 6)
