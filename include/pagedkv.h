@@ -27,8 +27,9 @@
  * (pkv_paged_attn_decode_shared_prefix), block swapping between the device
  * pool and pinned host memory (pkv_swap_blocks), a host-side block manager
  * with copy-on-write, chunk appends, prefix caching by block content and
- * swap bookkeeping (pkv_bm_*), and a host check of copy and swap pair lists
- * (pkv_check_block_pairs).
+ * swap bookkeeping (pkv_bm_*), a host check of copy and swap pair lists
+ * (pkv_check_block_pairs), and a read-only pass over a device buffer that
+ * measurements quote decode against (pkv_stream_read).
  *
  * Conventions shared by every entry point
  *   - All pointers except scalars are DEVICE pointers, owned by the caller
