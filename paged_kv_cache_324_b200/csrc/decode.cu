@@ -8,10 +8,14 @@
 // it further by partition and merges partitions exactly with log-sum-exp.
 //
 // Design (sm_100a):
-//   * Work unit = (partition of <= partition_size tokens, KV head, sequence):
-//     one CTA.  All G query heads of the KV head ride in the same CTA, so each
-//     K/V tile crosses HBM once per group (GQA; glossary "PagedAttention",
-//     section "Related methods").
+//   * Work unit = (partition of <= partition_size tokens, KV head, sequence).
+//     All G query heads of the KV head ride in the same CTA, so each K/V tile
+//     crosses HBM once per group (GQA; glossary "PagedAttention", section
+//     "Related methods").  A CTA streams one partition, or, when the caller
+//     states partitions smaller than the automatic size, as many consecutive
+//     ones as that size holds: the ring keeps streaming across them and each
+//     still ends in its own partial, merged exactly afterwards.  CTAs are
+//     dispatched partition index last-first.
 //   * One producer warp issues TMA tile loads.  The pool is described to TMA
 //     as a 4-D tensor [head_dim, block_size, num_kv_heads, num_blocks]; the
 //     block-table indirection is simply the outermost tile coordinate.  Tiles
@@ -33,10 +37,12 @@
 //     head_dim axis of QK and of the output is permuted (the same permutation
 //     on both operands, undone on output) so that each lane's fragment comes
 //     from contiguous bytes.
-//   * The four warps' partial states are merged in shared memory; a CTA that
-//     covers its whole sequence writes the output, otherwise it writes
-//     (max, sum, normalised output) to the workspace and a second small
-//     kernel merges the partitions.
+//   * At the end of each partition the four warps' states are merged in a
+//     shared-memory buffer of their own (a named barrier among the consumer
+//     warps; the producer keeps filling the ring); a CTA that covers its whole
+//     sequence writes the output, otherwise it writes (max, sum, normalised
+//     output) to the workspace and a second small kernel merges the
+//     partitions.
 //   * Masking: slots past the context length in the last block get score
 //     -inf (by select) and their V rows are zeroed before the MMA, so
 //     arbitrary bit patterns in unused slots (NaN/Inf) cannot leak.
@@ -87,6 +93,7 @@ struct DecodeArgs {
     int slot_base;              // first partition slot of the workspace this pass writes
     int prefix_partition_size;  // tail pass and merge: partition size of the prefix pass
     int max_prefix_len;         // bound of every unit_len and seq_start (0 in the plain call)
+    int parts_per_cta;          // consecutive partitions one CTA streams (each still gets its own partial)
 };
 
 // Written by the tail pass into every prefix slot a sequence's merge will read, before the
@@ -184,8 +191,11 @@ struct Geo {
     static constexpr int kStagesRaw = kRingTarget / kStageBytes / kConsumerWarps * kConsumerWarps;
     static constexpr int kStages = kStagesRaw < 4 ? 4 : (kStagesRaw > 32 ? 32 : kStagesRaw);
     static constexpr int kRingBytes = kStages * kStageBytes;
-    static constexpr int kMergeBytes = kConsumerWarps * 16 * (D + 2) * 4;
-    static constexpr int kDataBytes = kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes;
+    static constexpr int kRowsMax = kHi ? 16 : 8;                 // query rows of the instance
+    // the consumers' partition merge has a buffer of its own: the producer keeps filling the ring
+    // with the next partition's tiles meanwhile
+    static constexpr int kMergeBytes = kConsumerWarps * kRowsMax * (D + 2) * 4;
+    static constexpr int kDataBytes = kRingBytes + kMergeBytes;
     static constexpr int kSmemBytes = 1024 /* alignment slack */ + kDataBytes + kStages * 16 + 16;
     // CTAs per SM that the register budget must allow (shared memory permitting)
     static constexpr int kSmemCtas = (227 * 1024) / (kSmemBytes + 1024);
@@ -243,6 +253,11 @@ __device__ __forceinline__ uint32_t mask_pair(uint32_t x, int t, int valid) {
     return x & (lo | hi);
 }
 
+// Named barrier of the four consumer warps (the producer warp keeps streaming meanwhile).
+__device__ __forceinline__ void consumer_barrier() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+}
+
 // ---- pass 1: one CTA per (partition, KV head, sequence) ------------------------------
 
 template <int KV, bool kQBf16, int D, int BS, bool kHi>
@@ -262,7 +277,9 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
     const uint32_t bar_empty = bar_full + NST * 8;
     volatile int* s_abort = reinterpret_cast<volatile int*>(gbase + Gm::kDataBytes + NST * 16);
 
-    const int part = blockIdx.x, kvh = blockIdx.y, z = blockIdx.z;
+    // grid (KV heads, sequences or units, partition groups): the partition index is dispatched last
+    // first, so short trailing work does not end the grid behind long CTAs
+    const int part = static_cast<int>(gridDim.z - 1 - blockIdx.z), kvh = blockIdx.x, z = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = a.num_heads / a.num_kv_heads;
     const int H = a.num_heads;
@@ -338,14 +355,17 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
         return static_cast<size_t>(__ldg(a.unit_seqs + static_cast<size_t>(z) * a.unit_width + m)) * H +
                static_cast<size_t>(kvh) * G + (r - m * G);
     };
+    // the CTA streams partitions part0 .. part0 + nlp - 1 (consecutive, one partial each)
     const int PS = a.partition_size;
     const int nparts = (L + PS - 1) / PS;
-    if (part >= nparts) {
+    const int part0 = part * a.parts_per_cta;
+    if (part0 >= nparts) {
         if (first_cta) pdl_wait();
         return;
     }
-    const int tok_begin = part * PS;
-    const int tok_end = min(L, tok_begin + PS);
+    const int nlp = min(a.parts_per_cta, nparts - part0);
+    const int tok_begin = part0 * PS;
+    const int tok_end = min(L, tok_begin + nlp * PS);
     const int nblk = (tok_end - tok_begin + BS - 1) / BS;
     const int nstage = (nblk + Gm::kBps - 1) / Gm::kBps;
     const int blk0 = (start + tok_begin) / BS;
@@ -490,7 +510,16 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
         const int v_hi = li & 1;
         const float qk = a.qk_scale_log2;
 
-        for (int js = warp; js < nstage; js += kConsumerWarps) {
+        // stages per partition (a partition is a whole number of stages when a CTA holds several)
+        const int spp = nlp > 1 ? PS / Gm::kStageTok : nstage;
+        bool dead = false;   // a wait gave up: skip the remaining stages, still meet every barrier
+        float* sm_o = reinterpret_cast<float*>(gbase + Gm::kRingBytes);      // [warps][rows][D]
+        float* sm_m = sm_o + kConsumerWarps * Gm::kRowsMax * D;              // [warps][rows]
+        float* sm_l = sm_m + kConsumerWarps * Gm::kRowsMax;                  // [warps][rows]
+        for (int lp = 0; lp < nlp; ++lp) {
+        const int s_lo = lp * spp, s_hi = min(nstage, s_lo + spp);
+        for (int js = s_lo + (warp - s_lo % kConsumerWarps + kConsumerWarps) % kConsumerWarps; js < s_hi && !dead;
+             js += kConsumerWarps) {
             const int stage = js % NST;
             const bool got = mbar_wait(bar_full + 8 * stage, (js / NST) & 1);
             if (!__all_sync(0xffffffffu, got)) {
@@ -498,6 +527,7 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
                     raise_error(a.err, PKV_DEVERR_TIMEOUT);
                     *s_abort = 1;
                 }
+                dead = true;
                 break;
             }
             const uint32_t sb = base + stage * Gm::kStageBytes;
@@ -673,62 +703,73 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
                 v += __shfl_xor_sync(0xffffffffu, v, 16);
                 l_run[nh][hc] = v;
             }
-    }
-    pdl_trigger();     // the merge kernel (or the next step) may start its prologue
-    __syncthreads();   // ring fully consumed: reuse it for the merge
-
-    float* sm_o = reinterpret_cast<float*>(gbase);                    // [warps][16 heads][D]
-    float* sm_m = sm_o + kConsumerWarps * 16 * D;                      // [warps][16]
-    float* sm_l = sm_m + kConsumerWarps * 16;                          // [warps][16]
-    if (warp < kConsumerWarps) {
-        const int r = lane >> 2, c = lane & 3;
-        float* ow = sm_o + warp * 16 * D;
+        // ---- this partition's four warp states -> its output or partial (consumer warps only) ----
+        {
+            float* ow = sm_o + warp * Gm::kRowsMax * D;
+#pragma unroll
+            for (int md = 0; md < Gm::kMtDim; ++md)
+#pragma unroll
+                for (int nh = 0; nh < NTH; ++nh) {
+                    const int h0 = nh * 8 + 2 * c;
+                    const int d0 = Gm::o_dim(md, r), d1 = Gm::o_dim(md, r + 8);
+                    ow[h0 * D + d0] = o[md][nh][0];
+                    ow[(h0 + 1) * D + d0] = o[md][nh][1];
+                    ow[h0 * D + d1] = o[md][nh][2];
+                    ow[(h0 + 1) * D + d1] = o[md][nh][3];
+                }
+            if (r == 0) {
+#pragma unroll
+                for (int nh = 0; nh < NTH; ++nh)
+#pragma unroll
+                    for (int hc = 0; hc < 2; ++hc) {
+                        sm_m[warp * Gm::kRowsMax + nh * 8 + 2 * c + hc] = m_run[nh][hc];
+                        sm_l[warp * Gm::kRowsMax + nh * 8 + 2 * c + hc] = l_run[nh][hc];
+                    }
+            }
+        }
+        consumer_barrier();
+        {
+            if (lp == nlp - 1) pdl_trigger();   // the merge kernel (or the next step) may start its prologue
+            const bool aborted = *s_abort != 0;
+            const bool single = nparts == 1 && start == 0 && !prefix_pass;   // otherwise partials for the merge
+            const float vs = a.v_scale;
+            for (int e = threadIdx.x; e < rows * D; e += kConsumerWarps * 32) {
+                const int hh = e / D, d = e - hh * D;
+                float M = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm_m[w * Gm::kRowsMax + hh]);
+                float num = 0.f, den = 0.f;
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w) {
+                    const float f = exp2f(sm_m[w * Gm::kRowsMax + hh] - M);
+                    num += f * sm_o[(w * Gm::kRowsMax + hh) * D + d];
+                    den += f * sm_l[w * Gm::kRowsMax + hh];
+                }
+                float val = num / den * vs;
+                if (aborted) val = __int_as_float(0x7fc00000);
+                if (single) {
+                    store_out<kQBf16>(a.out, row_of(hh) * D + d, val);
+                } else {
+                    const size_t slot = row_of(hh) * a.max_partitions + a.slot_base + part0 + lp;
+                    a.ws_o[slot * D + d] = val;
+                    if (d == 0) a.ws_ml[slot] = make_float2(aborted ? __int_as_float(0x7fc00000) : M, den);
+                }
+            }
+        }
+        consumer_barrier();   // the buffer is rewritten by the next partition's states
+        // fresh state for the next partition
 #pragma unroll
         for (int md = 0; md < Gm::kMtDim; ++md)
 #pragma unroll
-            for (int nh = 0; nh < NTH; ++nh) {
-                const int h0 = nh * 8 + 2 * c;
-                const int d0 = Gm::o_dim(md, r), d1 = Gm::o_dim(md, r + 8);
-                ow[h0 * D + d0] = o[md][nh][0];
-                ow[(h0 + 1) * D + d0] = o[md][nh][1];
-                ow[h0 * D + d1] = o[md][nh][2];
-                ow[(h0 + 1) * D + d1] = o[md][nh][3];
-            }
-        if (r == 0) {
+            for (int nh = 0; nh < NTH; ++nh) o[md][nh][0] = o[md][nh][1] = o[md][nh][2] = o[md][nh][3] = 0.f;
 #pragma unroll
-            for (int nh = 0; nh < NTH; ++nh)
-#pragma unroll
-                for (int hc = 0; hc < 2; ++hc) {
-                    sm_m[warp * 16 + nh * 8 + 2 * c + hc] = m_run[nh][hc];
-                    sm_l[warp * 16 + nh * 8 + 2 * c + hc] = l_run[nh][hc];
-                }
+        for (int nh = 0; nh < NTH; ++nh) {
+            m_run[nh][0] = m_run[nh][1] = -INFINITY;
+            l_run[nh][0] = l_run[nh][1] = 0.f;
         }
+        }   // partitions of the CTA
     }
-    __syncthreads();
-    const bool aborted = *s_abort != 0;
-    const bool single = nparts == 1 && start == 0 && !prefix_pass;   // otherwise partials for the merge
-    for (int e = threadIdx.x; e < rows * D; e += kThreads) {
-        const int hh = e / D, d = e - hh * D;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm_m[w * 16 + hh]);
-        float num = 0.f, den = 0.f;
-#pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) {
-            const float f = exp2f(sm_m[w * 16 + hh] - M);
-            num += f * sm_o[(w * 16 + hh) * D + d];
-            den += f * sm_l[w * 16 + hh];
-        }
-        float val = num / den * a.v_scale;
-        if (aborted) val = __int_as_float(0x7fc00000);
-        if (single) {
-            store_out<kQBf16>(a.out, row_of(hh) * D + d, val);
-        } else {
-            const size_t slot = row_of(hh) * a.max_partitions + a.slot_base + part;
-            a.ws_o[slot * D + d] = val;
-            if (d == 0) a.ws_ml[slot] = make_float2(aborted ? __int_as_float(0x7fc00000) : M, den);
-        }
-    }
+    if (warp == kConsumerWarps) pdl_trigger();   // the producer is done issuing
 }
 
 // ---- pass 2: merge partitions by log-sum-exp -------------------------------------
@@ -888,7 +929,7 @@ pkv_status launch_pass1(const DecodeArgs& a, const CUtensorMap& km, const CUtens
     auto kern = paged_decode_kernel<KV, kQBf16, D, BS, kHi>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Gm::kSmemBytes) != cudaSuccess)
         return PKV_ERR_CUDA;
-    const dim3 grid(gx, static_cast<unsigned>(a.num_kv_heads), gz);
+    const dim3 grid(static_cast<unsigned>(a.num_kv_heads), gz, gx);
     return launch_pdl(kern, grid, dim3(kThreads), Gm::kSmemBytes, st, a, km, vm) == cudaSuccess ? PKV_OK
                                                                                                 : PKV_ERR_CUDA;
 }
@@ -991,10 +1032,30 @@ DecodeArgs base_args(void* out, const void* q, const int32_t* block_tables, int 
     a.num_blocks = num_blocks;
     a.block_size = block_size;
     a.partition_size = ps;
+    a.parts_per_cta = 1;
     const float ks = kv_dtype == PKV_FP8_E4M3 ? k_scale : 1.f;
     a.qk_scale_log2 = static_cast<float>(static_cast<double>(scale) * ks * 1.4426950408889634);
     a.v_scale = kv_dtype == PKV_FP8_E4M3 ? v_scale : 1.f;
     return a;
+}
+
+// Tokens of one ring stage of the decode kernel (the Geo rule: a stage moves at least 8 KB).
+int stage_tokens(pkv_dtype kv_dtype, int head_dim, int block_size) {
+    const int tile = block_size * head_dim * (kv_dtype == PKV_FP8_E4M3 ? 1 : 2);
+    const int bps = 2 * tile >= 8192 ? 1 : 8192 / (2 * tile);
+    return bps * block_size;
+}
+
+// Partitions one CTA streams: a stated partition size smaller than the automatic choice keeps its
+// partials (one per stated partition, merged exactly), but a CTA takes as many consecutive ones as
+// the automatic size holds, so that the ring streams across them instead of starting again.
+int partitions_per_cta(int ps, int num_seqs, int num_kv_heads, int head_dim, pkv_dtype kv_dtype, int block_size,
+                       int max_context_len, int requested) {
+    if (requested <= 0) return 1;
+    const int auto_ps = pick_partition(num_seqs, num_kv_heads, head_dim, kv_dtype == PKV_FP8_E4M3 ? 1 : 2,
+                                       block_size, max_context_len, 0);
+    if (auto_ps <= ps || ps % stage_tokens(kv_dtype, head_dim, block_size) != 0) return 1;
+    return auto_ps / ps;
 }
 
 size_t partials_bytes(size_t rows, int head_dim) {
@@ -1054,6 +1115,8 @@ extern "C" pkv_status pkv_paged_attn_decode(void* out, const void* q, pkv_dtype 
                              num_heads, num_kv_heads, num_blocks, block_size, kv_dtype, k_scale, v_scale, scale, ps,
                              device_error);
     a.max_partitions = parts;
+    a.parts_per_cta = partitions_per_cta(ps, num_seqs, num_kv_heads, head_dim, kv_dtype, block_size, max_context_len,
+                                         partition_size);
     if (need) set_partials(a, workspace, static_cast<size_t>(num_seqs) * num_heads * parts, head_dim);
 
     alignas(64) CUtensorMap km;
@@ -1063,8 +1126,9 @@ extern "C" pkv_status pkv_paged_attn_decode(void* out, const void* q, pkv_dtype 
         return PKV_ERR_CUDA;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const bool hi = num_heads / num_kv_heads > 8;
+    const unsigned groups = static_cast<unsigned>((parts + a.parts_per_cta - 1) / a.parts_per_cta);
     pkv_status r = with_instance(kv_dtype, q_dtype, head_dim, block_size, hi,
-                                 Pass1{a, km, vm, static_cast<unsigned>(parts), static_cast<unsigned>(num_seqs), st});
+                                 Pass1{a, km, vm, groups, static_cast<unsigned>(num_seqs), st});
     if (r == PKV_OK && parts > 1) r = with_instance(kv_dtype, q_dtype, head_dim, block_size, hi, Merge{a, st});
     return r;
 }
