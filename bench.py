@@ -54,17 +54,17 @@ FALLBACK_HBM_GBS = 6650.0
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by workload, valid only
 # for the decode kernel source it was measured on (sha256 prefix of decode.cu).
 NCU_TRAFFIC = {
-    "opt13b": {"bytes_per_launch": 1_316_705_536, "kernel_sha": "05714f1368298826",
+    "opt13b": {"bytes_per_launch": 1_313_395_456, "kernel_sha": "980738653df370e4",
                "capture": "ncu, opt13b_compact (the same sequences, pool cut to the blocks in use)"},
-    "gqa": {"bytes_per_launch": 1_224_799_136, "kernel_sha": "05714f1368298826",
+    "gqa": {"bytes_per_launch": 1_222_007_808, "kernel_sha": "980738653df370e4",
             "capture": "ncu, gqa_compact (the same sequences, pool cut to the blocks in use)"},
-    "fp8": {"bytes_per_launch": 1_118_479_160, "kernel_sha": "05714f1368298826",
+    "fp8": {"bytes_per_launch": 1_116_351_744, "kernel_sha": "980738653df370e4",
             "capture": "ncu, fp8_compact (the same sequences, 512-token partitions)"},
 }
 
 
 # the same for the prefill kernel (sha256 prefix of prefill.cu), on the prefill workload
-PREFILL_TRAFFIC = {"bytes_per_launch": 568_925_952, "kernel_sha": "538588bfa1f1bfab",
+PREFILL_TRAFFIC = {"bytes_per_launch": 569_112_320, "kernel_sha": "341da0a10c7c8cc7",
                    "capture": "ncu, prefill workload, paged_prefill_kernel"}
 
 
