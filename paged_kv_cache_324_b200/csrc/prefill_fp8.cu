@@ -23,6 +23,7 @@ namespace pkv {
 namespace {
 
 constexpr int kWidenThreads = 256;
+constexpr int kWidenUnroll = 4;
 
 // Two E4M3 values (low byte first) -> two f16 values in one word (exact).
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t x) {
@@ -76,25 +77,45 @@ widen_blocks_kernel(const uint2* __restrict__ k_pool, const uint2* __restrict__ 
     pdl_trigger();
     pdl_wait();   // the pool may still be written by the previous kernel (the chunk's scatter)
     const long long total = static_cast<long long>(num_seqs) * maxb * units_per_block;
-    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
-         i += static_cast<long long>(gridDim.x) * blockDim.x) {
-        const long long blk = i / units_per_block;
-        const long long e = i - blk * units_per_block;
-        const int s = static_cast<int>(blk / maxb), j = static_cast<int>(blk - static_cast<long long>(s) * maxb);
-        const int L = __ldg(lens + s);
-        const long long cap = static_cast<long long>(maxb) * block_size;
-        const int nb = L <= 0 ? 0 : static_cast<int>((min(static_cast<long long>(L), cap) + block_size - 1) / block_size);
-        if (j >= nb) continue;
-        const int pid = __ldg(tables + blk);
-        const bool bad = pid < 0 || pid >= num_blocks;
-        if (e == 0) {
-            wtab[blk] = bad ? -1 : static_cast<int32_t>(blk);
-            if (bad) raise_error(err, PKV_DEVERR_BLOCK_ID);
+    const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+    const long long cap = static_cast<long long>(maxb) * block_size;
+    // kWidenUnroll units per thread and round: their table entries, then their K and V loads, are all in
+    // flight before the first conversion
+    for (long long base = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; base < total;
+         base += stride * kWidenUnroll) {
+        long long src[kWidenUnroll];
+#pragma unroll
+        for (int u = 0; u < kWidenUnroll; ++u) {
+            src[u] = -1;
+            const long long i = base + u * stride;
+            if (i >= total) continue;
+            const long long blk = i / units_per_block;
+            const long long e = i - blk * units_per_block;
+            const int s = static_cast<int>(blk / maxb), j = static_cast<int>(blk - static_cast<long long>(s) * maxb);
+            const int L = __ldg(lens + s);
+            const int nb = L <= 0 ? 0 : static_cast<int>((min(static_cast<long long>(L), cap) + block_size - 1) / block_size);
+            if (j >= nb) continue;
+            const int pid = __ldg(tables + blk);
+            const bool bad = pid < 0 || pid >= num_blocks;
+            if (e == 0) {
+                wtab[blk] = bad ? -1 : static_cast<int32_t>(blk);
+                if (bad) raise_error(err, PKV_DEVERR_BLOCK_ID);
+            }
+            if (!bad) src[u] = static_cast<long long>(pid) * units_per_block + e;
         }
-        if (bad) continue;
-        const long long src = static_cast<long long>(pid) * units_per_block + e;
-        wk[i] = widen8<kBf16, false>(k_pool[src], 1.f);
-        wv[i] = widen8<kBf16, true>(v_pool[src], v_scale);
+        uint2 kx[kWidenUnroll], vx[kWidenUnroll];
+#pragma unroll
+        for (int u = 0; u < kWidenUnroll; ++u)
+            if (src[u] >= 0) {
+                kx[u] = k_pool[src[u]];
+                vx[u] = v_pool[src[u]];
+            }
+#pragma unroll
+        for (int u = 0; u < kWidenUnroll; ++u)
+            if (src[u] >= 0) {
+                wk[base + u * stride] = widen8<kBf16, false>(kx[u], 1.f);
+                wv[base + u * stride] = widen8<kBf16, true>(vx[u], v_scale);
+            }
     }
 }
 
