@@ -7,6 +7,7 @@ import numpy as np
 import pytest
 import torch
 
+from paged_kv_cache_324_b200 import binding as B_
 from paged_kv_cache_324_b200 import workload as wl
 from tests import harness as H
 from tests.parity import attention_close
@@ -39,6 +40,25 @@ def test_partition_size_does_not_change_result(ps):
     assert g["err"] == 0
     ok, rep = attention_close(g["out"], o["out"], w.kv_dtype, w.q_dtype)
     assert ok, (ps, rep)
+
+
+@pytest.mark.parametrize("q_dtype,kv_dtype,B", [("f16", "f16", 16), ("bf16", "bf16", 32), ("f16", "e4m3", 16),
+                                                ("bf16", "e4m3", 32)])
+def test_stated_partitions_streamed_several_per_cta(q_dtype, kv_dtype, B):
+    """Enough sequences that the automatic partition (1,024 tokens of 16-bit K/V, 2,048 of E4M3)
+    holds several stated 128-token ones: CTAs stream runs of them, each run's partitions ending in
+    partials of their own, with lengths below, at and around partition and run boundaries."""
+    lens = [1, 127, 128, 129, 700, 1023, 1024, 1025, 1500, 255, 256, 2047] * 4
+    Hkv, G, D = 8, 4, 128
+    w = wl.independent_sequences(f"runs-{q_dtype}-{kv_dtype}-{B}", 300 + B, len(lens), Hkv * G, Hkv, D, B,
+                                 4096, q_dtype, kv_dtype, lens)
+    auto = B_.decode_partition_size(w.num_seqs, Hkv, D, kv_dtype, B, w.max_context_len, 0)
+    assert auto >= 8 * 128                        # a CTA takes several stated partitions
+    g = H.gpu_step(w, partition_size=128, keep_pools=False)
+    o = H.oracle_step(w)
+    assert g["err"] == 0
+    ok, rep = attention_close(g["out"], o["out"], w.kv_dtype, w.q_dtype)
+    assert ok, rep
 
 
 EDGE_LENS = [1, 15, 16, 17, 31, 32, 33, 63, 64, 65, 511, 512, 513, 1025]
