@@ -273,6 +273,10 @@ class PrefillStep:
                                   dtype=torch.uint8, device=dev)
         else:
             self.k_pool, self.v_pool = up(w.initial_pool("k")), up(w.initial_pool("v"))
+            # bf16: the workspace V is narrowed into (f16 with a power of two per sequence and KV head)
+            need = B.prefill_workspace_bytes(w.dtype, w.num_seqs, w.max_blocks, w.num_kv_heads, w.head_dim,
+                                             w.block_size)
+            self.ws = torch.empty(need, dtype=torch.uint8, device=dev) if need else None
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
         for op in w.setup:
             if op.slots.size:
@@ -302,7 +306,7 @@ class PrefillStep:
             return
         self.B.paged_attn_prefill(self.out, self.d["q"], self.k_pool, self.v_pool, self.d["tables"], self.d["lens"],
                                   self.d["qstart"], float(w.scale), max_query_len=w.max_query_len,
-                                  device_error=self.err, stream=self.stream)
+                                  workspace=self.ws, device_error=self.err, stream=self.stream)
 
     def step(self):
         self.scatter_op()
@@ -392,8 +396,10 @@ def run_prefill(args, rank, world, local_rank):
         "metric": PREFILL_METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None,
-        "dtype": (w.dtype + " operands (E4M3 cache widened to " + w.dtype + "), f32 accumulate") if kv_fp8
-        else (w.dtype + " operands, f32 accumulate"),
+        "dtype": (w.dtype + " q.K^T (E4M3 cache widened exactly: K to " + w.dtype + ", V to f16), f16 P.V, "
+                  "f32 accumulate") if kv_fp8
+        else (w.dtype + " q.K^T, f16 P.V (V narrowed to f16 per sequence and KV head), f32 accumulate"
+              if w.dtype == "bf16" else w.dtype + " operands, f32 accumulate"),
         "data": "synthetic (seeded N(0,1) q/K/V; random-byte pool content in unwritten slots)",
         "config": {"workload": w.description + (", E4M3 cache (per-tensor amax/448 scales)" if kv_fp8 else ""),
                    "name": "prefill_fp8" if kv_fp8 else w.name, "num_seqs": w.num_seqs, "num_tokens": w.num_tokens,
@@ -402,7 +408,8 @@ def run_prefill(args, rank, world, local_rank):
                    "total_context_tokens": int(w.context_lens.sum()), "flops_per_step": flops,
                    "step": ("reshape_and_cache (the chunk's K/V, quantised to E4M3) + paged_attn_prefill_fp8 "
                             "(widen_blocks_kernel, then paged_prefill_kernel)") if kv_fp8
-                   else "reshape_and_cache (the chunk's K/V) + paged_attn_prefill",
+                   else "reshape_and_cache (the chunk's K/V) + paged_attn_prefill (v_absmax_kernel, "
+                        "v_narrow_kernel, then paged_prefill_kernel)",
                    "l2": "no flush: the step reads %.0f MB of K/V and q, %.0f MB of output are written; the "
                          "kernel is bound by the tensor cores, not HBM" % (wl.prefill_bytes(w) / 1e6,
                                                                            w.num_tokens * w.num_heads * w.head_dim * 2 / 1e6),
@@ -413,7 +420,8 @@ def run_prefill(args, rank, world, local_rank):
                       "reshape_and_cache": round(sc_ms, 5)},
         "roofline": {"bound": "tensor",
                      "kernel": ("the paged_attn_prefill_fp8 call (widen_blocks_kernel + paged_prefill_kernel)"
-                                if kv_fp8 else "paged_prefill_kernel"),
+                                if kv_fp8 else "the paged_attn_prefill call (v_absmax_kernel + v_narrow_kernel + "
+                                               "paged_prefill_kernel)"),
                      "achieved": round(achieved, 2),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "frac_of_sustained": round(achieved / peak_sus, 4),
@@ -427,7 +435,7 @@ def run_prefill(args, rank, world, local_rank):
                 "overlap": PIPELINE_NOTE,
                 "serial_value": round(total_flops / (e2e_serial_ms * 1e-3) / 1e12, 2),
                 "serial_ms_per_step": round(e2e_serial_ms, 5)},
-        "gpu_launches": (3 if kv_fp8 else 2) * K,
+        "gpu_launches": (3 if kv_fp8 else 4) * K,
         "timing": ("value: CUDA events around one replay of a CUDA graph holding K steps; roofline: K prefill "
                    "calls back to back from one graph in the same run (prefill_ms_in_stream, clocks_stream); "
                    "kernel_ms: CUDA events around each call in a third pass"),

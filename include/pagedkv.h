@@ -295,18 +295,34 @@ pkv_status pkv_paged_attn_decode_static_ws(void* out, const void* q, pkv_dtype q
  *   max_query_len  an upper bound of the chunk lengths (sizes the grid)
  *   head_dim in {64, 128}; block_size in {16, 32}; G = num_heads /
  *   num_kv_heads in {1, 2, 4, 8, 16}; scale > 0.
+ *   workspace      BF16 only, optional (see below): device memory of at least
+ *                  pkv_prefill_workspace_bytes() bytes, 256-byte aligned, or
+ *                  null; ignored for F16.  Owned by the caller, unused after
+ *                  the call's kernels complete.
  * Data-dependent problems (a chunk longer than its context, a context beyond
  * the table, a bad block id) write NaN rows for the affected query tile and
  * set PKV_DEVERR_CONTEXT_LEN / PKV_DEVERR_BLOCK_ID.  Scores and the output
- * accumulate in float32; the softmax weights enter the P.V product rounded
- * to dtype (the tensor-core operand type).  No workspace.
+ * accumulate in float32.  The softmax weights P enter the P.V tensor-core
+ * product as f16 (11 significant bits).  A bf16 V cannot meet an f16 P in
+ * one product, so for BF16:
+ *   - with a workspace, two passes first narrow V to f16 in the workspace:
+ *     for each (sequence, KV head) the power of two 2^e that brings its
+ *     largest finite |v| (positions < context_len) into [2^15, 2^16), then
+ *     v * 2^-e rounded to f16 (exact down to 2^-29 of that maximum; Inf and
+ *     NaN kept), and 2^e multiplies the head's output rows;
+ *   - without one, P enters as a bf16 high part plus a bf16 low part
+ *     (P - bf16(P)) against the bf16 V: two products, slower, no memory.
+ * Returns PKV_ERR_WORKSPACE if a non-null workspace is smaller than
+ * pkv_prefill_workspace_bytes().
  */
+size_t pkv_prefill_workspace_bytes(pkv_dtype dtype, int num_seqs, int max_blocks_per_seq, int num_kv_heads,
+                                   int head_dim, int block_size);
 pkv_status pkv_paged_attn_prefill(void* out, const void* q, pkv_dtype dtype, const void* k_pool,
                                   const void* v_pool, const int32_t* block_tables, int max_blocks_per_seq,
                                   const int32_t* context_lens, const int32_t* query_start, int max_query_len,
                                   int num_seqs, int num_tokens, int num_heads, int num_kv_heads, int head_dim,
-                                  int block_size, int num_blocks, float scale, uint32_t* device_error,
-                                  void* stream);
+                                  int block_size, int num_blocks, float scale, void* workspace,
+                                  size_t workspace_bytes, uint32_t* device_error, void* stream);
 
 /*
  * Chunked prefill over an FP8_E4M3 cache (glossary, section "Related methods":
@@ -314,8 +330,9 @@ pkv_status pkv_paged_attn_prefill(void* out, const void* q, pkv_dtype dtype, con
  * k_t = e4m3(K byte) * k_scale and v_t = e4m3(V byte) * v_scale.  A gather
  * kernel widens the blocks each sequence's queries can reach into 16-bit
  * pools inside `workspace` (one row of max_blocks_per_seq blocks per
- * sequence; K exactly, V times v_scale rounded once to q_dtype), then the
- * tensor-core prefill runs on them with scale * k_scale.  Arguments as for
+ * sequence; both exactly: K to q_dtype, V to f16), then the tensor-core
+ * prefill runs on them with scale * k_scale, one f16 P.V product, and
+ * v_scale multiplying the output rows.  Arguments as for
  * pkv_paged_attn_prefill, except: q_dtype in {F16, BF16} is also the output
  * type; the pools hold E4M3 bytes; k_scale, v_scale > 0; workspace: device
  * memory of at least pkv_prefill_fp8_workspace_bytes() bytes, 256-byte

@@ -51,7 +51,9 @@ def lib() -> ctypes.CDLL:
         L.pkv_paged_attn_decode.argtypes = [P, P, I, P, P, I, F, F, P, I, P, I, I, I, I, I, I, I, F, I,
                                             P, Z, P, P]
         L.pkv_paged_attn_decode.restype = I
-        L.pkv_paged_attn_prefill.argtypes = [P, P, I, P, P, P, I, P, P, I, I, I, I, I, I, I, I, F, P, P]
+        L.pkv_prefill_workspace_bytes.argtypes = [I, I, I, I, I, I]
+        L.pkv_prefill_workspace_bytes.restype = Z
+        L.pkv_paged_attn_prefill.argtypes = [P, P, I, P, P, P, I, P, P, I, I, I, I, I, I, I, I, F, P, Z, P, P]
         L.pkv_paged_attn_prefill.restype = I
         L.pkv_prefill_fp8_workspace_bytes.argtypes = [I, I, I, I, I]
         L.pkv_prefill_fp8_workspace_bytes.restype = Z
@@ -178,15 +180,24 @@ def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_pool: torch.Tensor, 
     return out
 
 
+def prefill_workspace_bytes(dtype, num_seqs, max_blocks_per_seq, num_kv_heads, head_dim, block_size) -> int:
+    """Bytes of device workspace with which a bf16 paged_attn_prefill narrows V to f16 (0 for f16)."""
+    return lib().pkv_prefill_workspace_bytes(_kv_code(dtype), num_seqs, max_blocks_per_seq, num_kv_heads, head_dim,
+                                             block_size)
+
+
 def paged_attn_prefill(out: torch.Tensor, q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
                        block_tables: torch.Tensor, context_lens: torch.Tensor, query_start: torch.Tensor,
-                       scale: float, *, max_query_len: int, device_error: Optional[torch.Tensor] = None,
-                       stream=None) -> torch.Tensor:
+                       scale: float, *, max_query_len: int, workspace="auto",
+                       device_error: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """out[T, H, D] = chunked causal prefill of q[T, H, D] over pools [NB, Hkv, B, D].
 
     The chunks of all sequences are packed in q; query_start int32 [S + 1] gives
     their row offsets, context_lens int32 [S] count each chunk's tokens (already
-    in the pool).  q, out and the pools share one 16-bit dtype.
+    in the pool).  q, out and the pools share one 16-bit dtype.  ``workspace``
+    (bf16 only): a uint8 tensor of at least prefill_workspace_bytes, "auto" to
+    allocate one with torch, or None for the call without one (the softmax
+    weights then enter P.V as two bf16 parts instead of V being narrowed to f16).
     """
     T, H, D = q.shape
     NB, Hkv, B, D2 = k_pool.shape
@@ -201,11 +212,17 @@ def paged_attn_prefill(out: torch.Tensor, q: torch.Tensor, k_pool: torch.Tensor,
         raise TypeError("query_start must be int32")
     if query_start.numel() != S + 1:
         raise ValueError("query_start must hold num_seqs + 1 offsets")
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise ValueError('workspace must be a tensor, "auto" or None')
+        need = prefill_workspace_bytes(q.dtype, S, block_tables.shape[1], Hkv, D, B)
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device) if need else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     status = lib().pkv_paged_attn_prefill(
         _dev(out, "out"), _dev(q, "q"), _code(q), _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"),
         _dev(block_tables, "block_tables"), block_tables.shape[1], _dev(context_lens, "context_lens"),
         _dev(query_start, "query_start"), int(max_query_len), S, T, H, Hkv, D, B, NB, float(scale),
-        _err(device_error), _stream(stream))
+        _dev(workspace, "workspace"), ws_bytes, _err(device_error), _stream(stream))
     _check(status, "paged_attn_prefill")
     return out
 

@@ -33,17 +33,22 @@
 //              base 2 with a running maximum that is only moved when the new
 //              one exceeds it by more than 2^8 (the result does not depend on
 //              the reference maximum; the lag only bounds the weights), write P
-//              as packed 16-bit pairs into the upper half of the same S columns
-//              with tcgen05.st (bf16: also the residual P - bf16(P) into the
-//              lower half, so that P.V sees ~16 significant bits of every
-//              weight, as a 16-bit f16 P's 11 bits nearly do), and rescale O in
-//              TMEM when the maximum moves; finally O / l, written into the
+//              as packed f16 pairs into the upper half of the same S columns
+//              with tcgen05.st (for a bf16 V: bf16 P, and the residual
+//              P - bf16(P) into the lower half, so that P.V sees ~16
+//              significant bits of every weight), and rescale O in TMEM when
+//              the maximum moves; finally O * f / l (f: V's scale), written into the
 //              query tile's own shared memory (free by then) and sent out by
 //              warp 0 with one TMA store per 64-column chunk, so that whole
 //              128-byte rows reach HBM (a tile cut short by the chunk's end is
 //              stored row by row instead).
 // While tile A's softmax works on S_A(j+1), the tensor core computes PV_B(j)
 // and S_B(j+1), and the other way round.
+//
+// A bf16 cache's V is normally narrowed to f16 before this kernel runs (two small passes below,
+// each (sequence, KV head) scaled by its own power of two), so that P enters P.V as one f16
+// operand with 11 significant bits: that keeps the weights' rounding inside the attention
+// tolerance with one product per key tile instead of the two the bf16 split needs.
 //
 // Keys beyond the last one any row of the CTA needs are never loaded; their V
 // rows are zeroed in shared memory (their weights are exactly 0, but 0 times
@@ -94,16 +99,20 @@ struct PGeo {
 
 struct PrefillArgs {
     void* out;
-    const int32_t* block_tables;
+    const int32_t* block_tables;   // K blocks
+    const int32_t* v_tables;       // V blocks (the same table, or a workspace pool's own)
     const int32_t* context_lens;
     const int32_t* query_start;
+    const float* v_mult;           // per (sequence, KV head) factor of the output, or null
     uint32_t* err;
     int max_blocks_per_seq;
     int num_tokens;
     int num_heads;
-    int num_blocks;
-    int group;            // G = num_heads / num_kv_heads
-    float scale_log2;     // scale * log2(e)
+    int num_blocks;                // of the K pool
+    int v_num_blocks;              // of the V pool
+    int group;                     // G = num_heads / num_kv_heads
+    float scale_log2;              // scale * log2(e)
+    float v_mult_all;              // factor of every output row (an E4M3 cache's V scale, else 1)
 };
 
 // ---- tcgen05 / TMEM primitives (inline PTX) ---------------------------------------
@@ -323,6 +332,7 @@ struct CtaFlags {
     int abort;
     int bad;
     uint32_t tmem_base;
+    float vmul;           // the factor of this CTA's output rows (V's scale)
 };
 
 // Bounded wait that also stops when another role of the CTA already gave up.
@@ -348,12 +358,17 @@ __device__ __forceinline__ bool warp_wait_bar(uint32_t bar, uint32_t parity, Cta
     return __all_sync(0xffffffffu, ok);
 }
 
-template <int D, int BS, bool kBf16>
+// kBf16: q, K and the output are bf16 (else f16).  kSplitP (bf16 only): V is bf16 too and the
+// weights enter P.V as a high and a low bf16 part; otherwise V is f16 (an f16 cache, or V narrowed
+// or widened to f16 with its scale applied to the output) and P is one f16 operand.
+template <int D, int BS, bool kBf16, bool kSplitP>
 __global__ void __launch_bounds__(kPThreads, 1)
 paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
                      const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                      const __grid_constant__ CUtensorMap omap) {
     using Gm = PGeo<D>;
+    static_assert(kBf16 || !kSplitP, "the two-part weights are for bf16 V");
+    constexpr bool kPvBf16 = kSplitP;                // the type of P and V in O += P V
     constexpr int kTB = kKeys / BS;                  // blocks per key tile
     constexpr uint32_t kBoxBytes = BS * 128;         // one block x one 64-column chunk
     extern __shared__ uint8_t smem_raw[];
@@ -434,6 +449,7 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
         mbar_init(drain, 1);
         flags.abort = 0;
         flags.bad = 0;
+        flags.vmul = a.v_mult_all * (a.v_mult ? __ldg(a.v_mult + static_cast<size_t>(s) * gridDim.y + kvh) : 1.f);
         mbar_fence_init();
     }
     if (warp == 1) {
@@ -466,7 +482,8 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
         }
         const CUtensorMap* map = is_k ? &kmap : &vmap;
         const uint32_t ring = is_k ? sK : sV;
-        const int32_t* trow = a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq;
+        const int32_t* trow = (is_k ? a.block_tables : a.v_tables) + static_cast<size_t>(s) * a.max_blocks_per_seq;
+        const int nblocks = is_k ? a.num_blocks : a.v_num_blocks;
         int issued = 0;                                   // tiles whose copies were issued
         // table entries are read one tile ahead so that their latency hides behind the copies
         int pid_next = (lane < kTB && lane < nblk) ? __ldg(trow + lane) : -1;
@@ -475,9 +492,9 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
             const int nb = (j + 1) * kTB + lane;
             pid_next = (j + 1 < ntk && lane < kTB && nb < nblk) ? __ldg(trow + nb) : -1;
             const bool want = lane < kTB && j * kTB + lane < nblk;
-            const bool bad = want && (pid < 0 || pid >= a.num_blocks);
+            const bool bad = want && (pid < 0 || pid >= nblocks);
             const unsigned ok_mask = __ballot_sync(0xffffffffu, want && !bad);
-            if (is_k && __any_sync(0xffffffffu, bad) && lane == 0) {
+            if (__any_sync(0xffffffffu, bad) && lane == 0) {
                 raise_error(a.err, PKV_DEVERR_BLOCK_ID);
                 flags.bad = 1;
             }
@@ -508,7 +525,7 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
         // ---------------- MMA issuer (one thread) ----------------
         if (lane == 0) {
             constexpr uint32_t idesc_s = mma_idesc(kBf16, false, kRows, kKeys);
-            constexpr uint32_t idesc_o = mma_idesc(kBf16, true, kRows, D);
+            constexpr uint32_t idesc_o = mma_idesc(kPvBf16, true, kRows, D);
             int k_waited = -1;                            // the last key tile whose arrival was awaited
             auto issue_s = [&](int t, int j) -> bool {    // S_t(j) = Q_t K_j^T into S_t
                 const int ks = j % kKStages;
@@ -535,7 +552,7 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
                     const uint64_t vdesc = smem_desc(sV + vs * Gm::kTile + kk * 16 * 128, kChunkBytes, 1024);
                     mma_f16_ts(tmem + kTmemO + t * 128, tmem + kTmemS + t * kKeys + kTmemP + kk * 8, vdesc, idesc_o,
                                j > 0 || kk > 0);
-                    if constexpr (kBf16)   // the weights' bf16 residual against the same V rows
+                    if constexpr (kSplitP)   // the weights' bf16 residual against the same V rows
                         mma_f16_ts(tmem + kTmemO + t * 128, tmem + kTmemS + t * kKeys + kTmemPlo + kk * 8, vdesc,
                                    idesc_o, true);
                 }
@@ -633,8 +650,8 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
                     const float2 e = fma2(make_float2(x[8 * h + c], x[8 * h + c + 1]), sc2, nm2);
                     const float2 p = make_float2(ex2(e.x), ex2(e.y));
                     sp[(c >> 1) & 1] = add2(sp[(c >> 1) & 1], p);
-                    pk[c / 2] = pack2<kBf16>(p.x, p.y);
-                    if constexpr (kBf16) {
+                    pk[c / 2] = pack2<kPvBf16>(p.x, p.y);
+                    if constexpr (kSplitP) {
                         // p - bf16(p) is exact in fp32; widening bf16 is a 16-bit shift
                         const float2 r = sub2(p, make_float2(__uint_as_float(pk[c / 2] << 16),
                                                              __uint_as_float(pk[c / 2] & 0xffff0000u)));
@@ -642,7 +659,7 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
                     }
                 }
                 tmem_st4(tS + kTmemP + half * 32 + h * 4, pk);
-                if constexpr (kBf16) tmem_st4(tS + kTmemPlo + half * 32 + h * 4, pl);
+                if constexpr (kSplitP) tmem_st4(tS + kTmemPlo + half * 32 + h * 4, pl);
             }
             const float2 s01 = add2(sp[0], sp[1]);
             l = l * alpha + (s01.x + s01.y);
@@ -677,7 +694,8 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
         if (ok && my_ntk > 0) ok = warp_wait_bar(o_done(t), 0, &flags, a.err);
         pdl_trigger();
         // partial row sums: the parity buffer the last exchange did not use is free by now
-        red[my_ntk & 1][t][half][row] = l;
+        // the output factor (V's scale) divides the row sum, so that 1 / sum brings it in
+        red[my_ntk & 1][t][half][row] = l / flags.vmul;
         // the output is written after the CTA-wide barrier below, which also publishes flags.bad
         tc_fence_before();
         __syncthreads();
@@ -782,10 +800,10 @@ bool encode_pool_map16(CUtensorMap* map, const void* pool, int head_dim, int blo
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int BS, bool kBf16>
+template <int D, int BS, bool kBf16, bool kSplitP>
 pkv_status launch_prefill(const PrefillArgs& a, const CUtensorMap& qm, const CUtensorMap& km, const CUtensorMap& vm,
                           const CUtensorMap& om, dim3 grid, cudaStream_t st) {
-    auto kern = paged_prefill_kernel<D, BS, kBf16>;
+    auto kern = paged_prefill_kernel<D, BS, kBf16, kSplitP>;
     const uint32_t smem = PGeo<D>::kSmemBytes;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return PKV_ERR_CUDA;
@@ -794,68 +812,344 @@ pkv_status launch_prefill(const PrefillArgs& a, const CUtensorMap& qm, const CUt
 }
 
 template <int D, int BS>
-pkv_status dispatch_dtype(bool bf16, const PrefillArgs& a, const CUtensorMap& qm, const CUtensorMap& km,
-                          const CUtensorMap& vm, const CUtensorMap& om, dim3 grid, cudaStream_t st) {
-    return bf16 ? launch_prefill<D, BS, true>(a, qm, km, vm, om, grid, st)
-                : launch_prefill<D, BS, false>(a, qm, km, vm, om, grid, st);
+pkv_status dispatch_mode(bool bf16, bool v_f16, const PrefillArgs& a, const CUtensorMap& qm, const CUtensorMap& km,
+                         const CUtensorMap& vm, const CUtensorMap& om, dim3 grid, cudaStream_t st) {
+    if (!bf16) return launch_prefill<D, BS, false, false>(a, qm, km, vm, om, grid, st);
+    return v_f16 ? launch_prefill<D, BS, true, false>(a, qm, km, vm, om, grid, st)
+                 : launch_prefill<D, BS, true, true>(a, qm, km, vm, om, grid, st);
+}
+
+// ---- narrowing a bf16 V to f16 (the workspace path of pkv_paged_attn_prefill) -------------
+
+constexpr int kNarrowThreads = 256;
+constexpr int kNarrowChunk = 16;       // table slots per CTA of the two passes
+constexpr int kNarrowUnroll = 4;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct NarrowLayout {                  // the workspace of the bf16 path, in this order
+    size_t pool, table, mult, parts, total;
+    int chunks;
+};
+
+NarrowLayout narrow_layout(int num_seqs, int maxb, int num_kv_heads, int head_dim, int block_size) {
+    NarrowLayout l{};
+    const size_t blocks = static_cast<size_t>(num_seqs) * maxb;
+    const size_t sh = static_cast<size_t>(num_seqs) * num_kv_heads;
+    l.chunks = (maxb + kNarrowChunk - 1) / kNarrowChunk;
+    l.pool = align256(blocks * num_kv_heads * block_size * head_dim * 2);
+    l.table = align256(blocks * sizeof(int32_t));
+    l.mult = align256(sh * sizeof(float));
+    l.parts = align256(sh * l.chunks * sizeof(uint32_t));
+    l.total = l.pool + l.table + l.mult + l.parts;
+    return l;
+}
+
+// The largest finite magnitude among 8 bf16 values (as the bits of |v|; bf16 magnitudes order as
+// integers), those at key positions >= limit excluded.
+__device__ __forceinline__ uint32_t absmax8(const uint4& x, bool valid) {
+    if (!valid) return 0;
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    uint32_t m = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t lo = w[i] & 0x7fffu, hi = (w[i] >> 16) & 0x7fffu;
+        m = max(m, lo < 0x7f80u ? lo : 0u);   // exponent all ones: Inf or NaN, not scaled for
+        m = max(m, hi < 0x7f80u ? hi : 0u);
+    }
+    return m;
+}
+
+// Pass 1: for each (sequence s, KV head h, chunk of kNarrowChunk table slots) the largest finite
+// |v| of the V rows at positions < L_s, into parts[(s, h)][chunk].
+template <int BS, int D>
+__global__ void __launch_bounds__(kNarrowThreads)
+v_absmax_kernel(const uint4* __restrict__ v_pool, const int32_t* __restrict__ tables,
+                const int32_t* __restrict__ lens, uint32_t* __restrict__ parts, int maxb, int num_kv_heads,
+                int num_blocks) {
+    constexpr int kRun = BS * D / 8;                 // 16-byte units of one block and head
+    pdl_trigger();
+    pdl_wait();                                      // the pool may still be written by the previous kernel
+    const int chunk = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
+    const int L = __ldg(lens + s);
+    const long long cap = static_cast<long long>(maxb) * BS;
+    const int nb = L <= 0 ? 0 : static_cast<int>((min(static_cast<long long>(L), cap) + BS - 1) / BS);
+    const int j0 = chunk * kNarrowChunk, j1 = min(nb, j0 + kNarrowChunk);
+    uint32_t m = 0;
+    for (int u0 = threadIdx.x; u0 < (j1 - j0) * kRun; u0 += kNarrowThreads * kNarrowUnroll) {
+        uint4 x[kNarrowUnroll];
+        bool valid[kNarrowUnroll];
+#pragma unroll
+        for (int k = 0; k < kNarrowUnroll; ++k) {
+            const int u = u0 + k * kNarrowThreads;
+            const int j = j0 + u / kRun, e = u % kRun;
+            valid[k] = false;
+            if (u < (j1 - j0) * kRun) {
+                const int pid = __ldg(tables + static_cast<size_t>(s) * maxb + j);
+                valid[k] = pid >= 0 && pid < num_blocks && j * BS + e / (D / 8) < L;
+                if (valid[k])
+                    x[k] = __ldg(v_pool + ((static_cast<size_t>(pid) * num_kv_heads + h) * kRun + e));
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < kNarrowUnroll; ++k) m = max(m, absmax8(x[k], valid[k]));
+    }
+    m = __reduce_max_sync(0xffffffffu, m);
+    __shared__ uint32_t wm[kNarrowThreads / 32];
+    if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < kNarrowThreads / 32; ++w) m = max(m, wm[w]);
+        parts[(static_cast<size_t>(s) * num_kv_heads + h) * gridDim.x + chunk] = m;
+    }
+}
+
+// The power of two e with which v * 2^-e fits f16: the largest finite |v| (bf16 bits) lands in
+// [2^15, 2^16), so no value overflows and every value down to 2^-29 of the largest stays a normal
+// f16 (exact: bf16 carries 8 significant bits, f16 11).  Clamped so that 2^e and 2^-e are normal
+// floats; 0 for a head without finite values.
+__device__ __forceinline__ int narrow_exponent(uint32_t maxbits) {
+    if (maxbits == 0) return 0;
+    const int eb = static_cast<int>(maxbits >> 7);   // biased bf16 exponent, 0 for subnormals
+    const int e = (eb == 0 ? -126 : eb - 127) - 15;
+    return min(max(e, -96), 112);
+}
+
+// Pass 2: the same slots; V rows at positions < L_s become f16(v * 2^-e) in the workspace pool
+// (block s * maxb + j), later rows zeros; the workspace table and the output factor 2^e are
+// written alongside.  A bad block id leaves a -1 in the workspace table, which the prefill kernel
+// reports; raised here too.
+template <int BS, int D>
+__global__ void __launch_bounds__(kNarrowThreads)
+v_narrow_kernel(const uint4* __restrict__ v_pool, const int32_t* __restrict__ tables,
+                const int32_t* __restrict__ lens, const uint32_t* __restrict__ parts, uint4* __restrict__ wv,
+                int32_t* __restrict__ wtab, float* __restrict__ mult, int maxb, int num_kv_heads, int num_blocks,
+                uint32_t* err) {
+    constexpr int kRun = BS * D / 8;
+    pdl_trigger();
+    pdl_wait();                                      // every partial maximum is written
+    const int chunk = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
+    const size_t sh = static_cast<size_t>(s) * num_kv_heads + h;
+    __shared__ float down;
+    if (threadIdx.x < 32) {
+        uint32_t m = 0;
+        for (int c = threadIdx.x; c < static_cast<int>(gridDim.x); c += 32) m = max(m, __ldg(parts + sh * gridDim.x + c));
+        m = __reduce_max_sync(0xffffffffu, m);
+        if (threadIdx.x == 0) {
+            const int e = narrow_exponent(m);
+            down = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);    // 2^-e
+            if (chunk == 0) mult[sh] = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);   // 2^e
+        }
+    }
+    __syncthreads();
+    const float f = down;
+    const int L = __ldg(lens + s);
+    const long long cap = static_cast<long long>(maxb) * BS;
+    const int nb = L <= 0 ? 0 : static_cast<int>((min(static_cast<long long>(L), cap) + BS - 1) / BS);
+    const int j0 = chunk * kNarrowChunk, j1 = min(maxb, j0 + kNarrowChunk);
+    if (h == 0)
+        for (int j = j0 + static_cast<int>(threadIdx.x); j < j1; j += kNarrowThreads) {
+            const int pid = j < nb ? __ldg(tables + static_cast<size_t>(s) * maxb + j) : -1;
+            const bool bad = j < nb && (pid < 0 || pid >= num_blocks);
+            if (bad) raise_error(err, PKV_DEVERR_BLOCK_ID);
+            wtab[static_cast<size_t>(s) * maxb + j] = (j < nb && !bad) ? static_cast<int32_t>(s * maxb + j) : -1;
+        }
+    const int jn = min(nb, j1);
+    for (int u0 = threadIdx.x; u0 < (jn - j0) * kRun; u0 += kNarrowThreads * kNarrowUnroll) {
+        uint4 x[kNarrowUnroll];
+        int dst[kNarrowUnroll];                      // -1: nothing to write; else the unit's slot j (and e)
+        bool live[kNarrowUnroll];
+#pragma unroll
+        for (int k = 0; k < kNarrowUnroll; ++k) {
+            const int u = u0 + k * kNarrowThreads;
+            dst[k] = -1;
+            live[k] = false;
+            if (u < (jn - j0) * kRun) {
+                const int j = j0 + u / kRun, e = u % kRun;
+                const int pid = __ldg(tables + static_cast<size_t>(s) * maxb + j);
+                if (pid >= 0 && pid < num_blocks) {
+                    dst[k] = u;
+                    live[k] = j * BS + e / (D / 8) < L;
+                    if (live[k]) x[k] = __ldg(v_pool + ((static_cast<size_t>(pid) * num_kv_heads + h) * kRun + e));
+                }
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < kNarrowUnroll; ++k) {
+            if (dst[k] < 0) continue;
+            const int j = j0 + dst[k] / kRun, e = dst[k] % kRun;
+            uint4 o = make_uint4(0u, 0u, 0u, 0u);
+            if (live[k]) {
+                const uint32_t w[4] = {x[k].x, x[k].y, x[k].z, x[k].w};
+                uint32_t r[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const __half2 v = __floats2half2_rn(__uint_as_float(w[i] << 16) * f,
+                                                        __uint_as_float(w[i] & 0xffff0000u) * f);
+                    r[i] = *reinterpret_cast<const uint32_t*>(&v);
+                }
+                o = make_uint4(r[0], r[1], r[2], r[3]);
+            }
+            wv[((static_cast<size_t>(s) * maxb + j) * num_kv_heads + h) * kRun + e] = o;
+        }
+    }
+}
+
+template <int BS, int D>
+pkv_status launch_narrow(const void* v_pool, const int32_t* tables, const int32_t* lens, uint8_t* ws,
+                         const NarrowLayout& l, int num_seqs, int maxb, int num_kv_heads, int num_blocks,
+                         uint32_t* err, cudaStream_t st) {
+    const dim3 grid(static_cast<unsigned>(l.chunks), static_cast<unsigned>(num_kv_heads),
+                    static_cast<unsigned>(num_seqs));
+    uint4* wv = reinterpret_cast<uint4*>(ws);
+    int32_t* wtab = reinterpret_cast<int32_t*>(ws + l.pool);
+    float* mult = reinterpret_cast<float*>(ws + l.pool + l.table);
+    uint32_t* parts = reinterpret_cast<uint32_t*>(ws + l.pool + l.table + l.mult);
+    if (launch_pdl(v_absmax_kernel<BS, D>, grid, dim3(kNarrowThreads), 0, st, static_cast<const uint4*>(v_pool),
+                   tables, lens, parts, maxb, num_kv_heads, num_blocks) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    return launch_pdl(v_narrow_kernel<BS, D>, grid, dim3(kNarrowThreads), 0, st, static_cast<const uint4*>(v_pool),
+                      tables, lens, static_cast<const uint32_t*>(parts), wv, wtab, mult, maxb, num_kv_heads,
+                      num_blocks, err) == cudaSuccess
+               ? PKV_OK
+               : PKV_ERR_CUDA;
 }
 
 }  // namespace
+
+pkv_status prefill_check(const PrefillLaunch& p, bool dtype_supported) {
+    if (p.num_seqs < 0 || p.num_tokens < 0 || p.max_query_len < 0 || p.num_heads <= 0 || p.num_kv_heads <= 0 ||
+        p.num_blocks <= 0 || p.max_blocks_per_seq <= 0 || !(p.scale > 0.f) || !std::isfinite(p.scale))
+        return PKV_ERR_INVALID_ARG;
+    if (p.num_heads % p.num_kv_heads != 0) return PKV_ERR_INVALID_ARG;
+    if (!dtype_supported) return PKV_ERR_UNSUPPORTED;
+    const int G = p.num_heads / p.num_kv_heads;
+    if ((p.head_dim != 64 && p.head_dim != 128) || (p.block_size != 16 && p.block_size != 32) ||
+        (G != 1 && G != 2 && G != 4 && G != 8 && G != 16))
+        return PKV_ERR_UNSUPPORTED;
+    if (p.num_seqs == 0 || p.num_tokens == 0 || p.max_query_len == 0) return PKV_OK;
+    if (!p.out || !p.q || !p.k_pool || !p.v_pool || !p.k_tables || !p.context_lens || !p.query_start)
+        return PKV_ERR_INVALID_ARG;
+    if (!aligned16(p.out) || !aligned16(p.q) || !aligned16(p.k_pool) || !aligned16(p.v_pool) ||
+        (reinterpret_cast<uintptr_t>(p.k_tables) & 3) || (reinterpret_cast<uintptr_t>(p.context_lens) & 3) ||
+        (reinterpret_cast<uintptr_t>(p.query_start) & 3) || (reinterpret_cast<uintptr_t>(p.err) & 3))
+        return PKV_ERR_ALIGNMENT;
+    const long long tiles = (static_cast<long long>(p.max_query_len) * G + kTiles * kRows - 1) / (kTiles * kRows);
+    if (p.num_seqs > 65535 || p.num_kv_heads > 65535 || tiles > 0x7fffffffLL ||
+        static_cast<long long>(p.num_seqs) * p.max_blocks_per_seq > 0x7fffffffLL)
+        return PKV_ERR_INVALID_ARG;
+    return PKV_OK;
+}
+
+pkv_status prefill_launch(const PrefillLaunch& p) {
+    const int G = p.num_heads / p.num_kv_heads;
+    const long long tiles = (static_cast<long long>(p.max_query_len) * G + kTiles * kRows - 1) / (kTiles * kRows);
+    PrefillArgs a{};
+    a.out = p.out;
+    a.block_tables = p.k_tables;
+    a.v_tables = p.v_tables ? p.v_tables : p.k_tables;
+    a.context_lens = p.context_lens;
+    a.query_start = p.query_start;
+    a.v_mult = p.v_mult;
+    a.err = p.err;
+    a.max_blocks_per_seq = p.max_blocks_per_seq;
+    a.num_tokens = p.num_tokens;
+    a.num_heads = p.num_heads;
+    a.num_blocks = p.num_blocks;
+    a.v_num_blocks = p.v_tables ? p.v_num_blocks : p.num_blocks;
+    a.group = G;
+    a.scale_log2 = p.scale * 1.4426950408889634f;
+    a.v_mult_all = p.v_mult_all;
+
+    alignas(64) CUtensorMap qm;
+    alignas(64) CUtensorMap km;
+    alignas(64) CUtensorMap vm;
+    alignas(64) CUtensorMap om;   // the output has q's layout, so it is stored with q's box
+    if (!encode_q_map(&qm, p.q, p.head_dim, p.num_heads, p.num_tokens, G) ||
+        !encode_pool_map16(&km, p.k_pool, p.head_dim, p.block_size, p.num_kv_heads, p.num_blocks) ||
+        !encode_pool_map16(&vm, p.v_pool, p.head_dim, p.block_size, p.num_kv_heads, a.v_num_blocks) ||
+        !encode_q_map(&om, p.out, p.head_dim, p.num_heads, p.num_tokens, G))
+        return PKV_ERR_CUDA;
+    const dim3 grid(static_cast<unsigned>(tiles), static_cast<unsigned>(p.num_kv_heads),
+                    static_cast<unsigned>(p.num_seqs));
+    cudaStream_t st = p.stream;
+    if (p.head_dim == 128)
+        return p.block_size == 16 ? dispatch_mode<128, 16>(p.bf16, p.v_f16, a, qm, km, vm, om, grid, st)
+                                  : dispatch_mode<128, 32>(p.bf16, p.v_f16, a, qm, km, vm, om, grid, st);
+    return p.block_size == 16 ? dispatch_mode<64, 16>(p.bf16, p.v_f16, a, qm, km, vm, om, grid, st)
+                              : dispatch_mode<64, 32>(p.bf16, p.v_f16, a, qm, km, vm, om, grid, st);
+}
+
 }  // namespace pkv
+
+extern "C" size_t pkv_prefill_workspace_bytes(pkv_dtype dtype, int num_seqs, int max_blocks_per_seq,
+                                              int num_kv_heads, int head_dim, int block_size) {
+    if (dtype != PKV_BF16 || num_seqs <= 0 || max_blocks_per_seq <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        block_size <= 0)
+        return 0;
+    return pkv::narrow_layout(num_seqs, max_blocks_per_seq, num_kv_heads, head_dim, block_size).total;
+}
 
 extern "C" pkv_status pkv_paged_attn_prefill(void* out, const void* q, pkv_dtype dtype, const void* k_pool,
                                              const void* v_pool, const int32_t* block_tables, int max_blocks_per_seq,
                                              const int32_t* context_lens, const int32_t* query_start,
                                              int max_query_len, int num_seqs, int num_tokens, int num_heads,
                                              int num_kv_heads, int head_dim, int block_size, int num_blocks,
-                                             float scale, uint32_t* device_error, void* stream) {
+                                             float scale, void* workspace, size_t workspace_bytes,
+                                             uint32_t* device_error, void* stream) {
     using namespace pkv;
-    if (num_seqs < 0 || num_tokens < 0 || max_query_len < 0 || num_heads <= 0 || num_kv_heads <= 0 ||
-        num_blocks <= 0 || max_blocks_per_seq <= 0 || !(scale > 0.f) || !std::isfinite(scale))
-        return PKV_ERR_INVALID_ARG;
-    if (num_heads % num_kv_heads != 0) return PKV_ERR_INVALID_ARG;
-    if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
-    const int G = num_heads / num_kv_heads;
-    if ((head_dim != 64 && head_dim != 128) || (block_size != 16 && block_size != 32) ||
-        (G != 1 && G != 2 && G != 4 && G != 8 && G != 16))
-        return PKV_ERR_UNSUPPORTED;
-    if (num_seqs == 0 || num_tokens == 0 || max_query_len == 0) return PKV_OK;
-    if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens || !query_start) return PKV_ERR_INVALID_ARG;
-    if (!aligned16(out) || !aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) ||
-        (reinterpret_cast<uintptr_t>(block_tables) & 3) || (reinterpret_cast<uintptr_t>(context_lens) & 3) ||
-        (reinterpret_cast<uintptr_t>(query_start) & 3) || (reinterpret_cast<uintptr_t>(device_error) & 3))
-        return PKV_ERR_ALIGNMENT;
-    const long long tiles = (static_cast<long long>(max_query_len) * G + kTiles * kRows - 1) / (kTiles * kRows);
-    if (num_seqs > 65535 || num_kv_heads > 65535 || tiles > 0x7fffffffLL) return PKV_ERR_INVALID_ARG;
-
-    PrefillArgs a{};
-    a.out = out;
-    a.block_tables = block_tables;
-    a.context_lens = context_lens;
-    a.query_start = query_start;
-    a.err = device_error;
-    a.max_blocks_per_seq = max_blocks_per_seq;
-    a.num_tokens = num_tokens;
-    a.num_heads = num_heads;
-    a.num_blocks = num_blocks;
-    a.group = G;
-    a.scale_log2 = scale * 1.4426950408889634f;
-
-    alignas(64) CUtensorMap qm;
-    alignas(64) CUtensorMap km;
-    alignas(64) CUtensorMap vm;
-    alignas(64) CUtensorMap om;   // the output has q's layout, so it is stored with q's box
-    if (!encode_q_map(&qm, q, head_dim, num_heads, num_tokens, G) ||
-        !encode_pool_map16(&km, k_pool, head_dim, block_size, num_kv_heads, num_blocks) ||
-        !encode_pool_map16(&vm, v_pool, head_dim, block_size, num_kv_heads, num_blocks) ||
-        !encode_q_map(&om, out, head_dim, num_heads, num_tokens, G))
-        return PKV_ERR_CUDA;
-    const dim3 grid(static_cast<unsigned>(tiles), static_cast<unsigned>(num_kv_heads), static_cast<unsigned>(num_seqs));
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const bool bf16 = dtype == PKV_BF16;
-    if (head_dim == 128)
-        return block_size == 16 ? dispatch_dtype<128, 16>(bf16, a, qm, km, vm, om, grid, st)
-                                : dispatch_dtype<128, 32>(bf16, a, qm, km, vm, om, grid, st);
-    return block_size == 16 ? dispatch_dtype<64, 16>(bf16, a, qm, km, vm, om, grid, st)
-                            : dispatch_dtype<64, 32>(bf16, a, qm, km, vm, om, grid, st);
+    PrefillLaunch p{};
+    p.out = out;
+    p.q = q;
+    p.bf16 = dtype == PKV_BF16;
+    p.k_pool = k_pool;
+    p.v_pool = v_pool;
+    p.k_tables = block_tables;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.context_lens = context_lens;
+    p.query_start = query_start;
+    p.max_query_len = max_query_len;
+    p.num_seqs = num_seqs;
+    p.num_tokens = num_tokens;
+    p.num_heads = num_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.head_dim = head_dim;
+    p.block_size = block_size;
+    p.num_blocks = num_blocks;
+    p.scale = scale;
+    p.v_mult_all = 1.f;
+    p.err = device_error;
+    p.stream = static_cast<cudaStream_t>(stream);
+    p.v_f16 = !p.bf16;
+    const pkv_status chk = prefill_check(p, dtype == PKV_F16 || dtype == PKV_BF16);
+    if (chk != PKV_OK || num_seqs == 0 || num_tokens == 0 || max_query_len == 0) return chk;
+    if (p.bf16 && workspace) {
+        // V narrowed to f16 with a power-of-two scale per (sequence, KV head): one f16 P.V product
+        const NarrowLayout l = narrow_layout(num_seqs, max_blocks_per_seq, num_kv_heads, head_dim, block_size);
+        if (workspace_bytes < l.total) return PKV_ERR_WORKSPACE;
+        if (reinterpret_cast<uintptr_t>(workspace) & 255) return PKV_ERR_ALIGNMENT;
+        uint8_t* ws = static_cast<uint8_t*>(workspace);
+        pkv_status st;
+        if (head_dim == 128)
+            st = block_size == 16 ? launch_narrow<16, 128>(v_pool, block_tables, context_lens, ws, l, num_seqs,
+                                                           max_blocks_per_seq, num_kv_heads, num_blocks,
+                                                           device_error, p.stream)
+                                  : launch_narrow<32, 128>(v_pool, block_tables, context_lens, ws, l, num_seqs,
+                                                           max_blocks_per_seq, num_kv_heads, num_blocks,
+                                                           device_error, p.stream);
+        else
+            st = block_size == 16 ? launch_narrow<16, 64>(v_pool, block_tables, context_lens, ws, l, num_seqs,
+                                                          max_blocks_per_seq, num_kv_heads, num_blocks, device_error,
+                                                          p.stream)
+                                  : launch_narrow<32, 64>(v_pool, block_tables, context_lens, ws, l, num_seqs,
+                                                          max_blocks_per_seq, num_kv_heads, num_blocks, device_error,
+                                                          p.stream);
+        if (st != PKV_OK) return st;
+        p.v_pool = ws;
+        p.v_tables = reinterpret_cast<const int32_t*>(ws + l.pool);
+        p.v_num_blocks = num_seqs * max_blocks_per_seq;
+        p.v_mult = reinterpret_cast<const float*>(ws + l.pool + l.table);
+        p.v_f16 = true;
+    }
+    return prefill_launch(p);
 }

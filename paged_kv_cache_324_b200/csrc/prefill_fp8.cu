@@ -3,12 +3,13 @@
 //
 // Prefill is bound by the tensor cores, not by the cache bytes (each K/V tile is used by
 // 2 x 128 query rows), so the FP8 case reuses the 16-bit tensor-core kernel: a gather kernel
-// first widens the blocks each sequence's queries can reach into a 16-bit workspace pool laid
-// out one row of max_blocks_per_seq blocks per sequence, with a block table of its own.  E4M3
-// values are exactly representable in f16 and bf16, so K is widened exactly and its scale is
-// folded into the softmax scale; V is multiplied by its scale and rounded once to the query's
-// type.  A block id outside the pool becomes an out-of-range entry of the workspace table, which
-// the prefill kernel reports (PKV_DEVERR_BLOCK_ID) with NaN rows, as for a 16-bit cache.
+// first widens the blocks each sequence's queries can reach into 16-bit workspace pools laid
+// out one row of max_blocks_per_seq blocks per sequence, with a block table of their own.  E4M3
+// values are exactly representable in f16 and bf16, so both are widened exactly: K to the
+// query's type, its scale folded into the softmax scale; V to f16, its scale applied to the
+// output rows, so that P.V is one f16 product for either query type.  A block id outside the
+// pool becomes an out-of-range entry of the workspace table, which the prefill kernel reports
+// (PKV_DEVERR_BLOCK_ID) with NaN rows, as for a 16-bit cache.
 
 #include <cmath>
 #include <cstdint>
@@ -32,40 +33,31 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t x) {
     return h;
 }
 
-template <bool kBf16>
-__device__ __forceinline__ uint32_t scaled_pair(uint32_t f16x2, float s) {
+// Two f16 values -> the same two values as bf16 (exact for widened E4M3: 4 significant bits).
+__device__ __forceinline__ uint32_t f16x2_to_bf16x2(uint32_t f16x2) {
     const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&f16x2));
-    if constexpr (kBf16) {
-        const __nv_bfloat162 b = __floats2bfloat162_rn(f.x * s, f.y * s);
-        return *reinterpret_cast<const uint32_t*>(&b);
-    } else {
-        const __half2 h = __floats2half2_rn(f.x * s, f.y * s);
-        return *reinterpret_cast<const uint32_t*>(&h);
-    }
+    const __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);
+    return *reinterpret_cast<const uint32_t*>(&b);
 }
 
-// 8 E4M3 bytes -> 8 values of the query's type (one 16-byte vector), times `s` (s = 1 for K: exact).
-template <bool kBf16, bool kScale>
-__device__ __forceinline__ uint4 widen8(const uint2& x, float s) {
+// 8 E4M3 bytes -> 8 f16 (or bf16) values, one 16-byte vector (exact).
+template <bool kBf16>
+__device__ __forceinline__ uint4 widen8(const uint2& x) {
     const uint32_t w[2] = {x.x, x.y};
     uint32_t o[4];
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
         const uint32_t a = e4m3x2_to_f16x2(static_cast<uint16_t>(w[i] & 0xffffu));
         const uint32_t b = e4m3x2_to_f16x2(static_cast<uint16_t>(w[i] >> 16));
-        if constexpr (!kScale && !kBf16) {
-            o[2 * i] = a;
-            o[2 * i + 1] = b;
-        } else {
-            o[2 * i] = scaled_pair<kBf16>(a, kScale ? s : 1.f);
-            o[2 * i + 1] = scaled_pair<kBf16>(b, kScale ? s : 1.f);
-        }
+        o[2 * i] = kBf16 ? f16x2_to_bf16x2(a) : a;
+        o[2 * i + 1] = kBf16 ? f16x2_to_bf16x2(b) : b;
     }
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 // Flat index over (sequence s, table slot j, 8-byte unit of the E4M3 block): block s * maxb + j
-// of the workspace pools receives the widened block block_tables[s][j], for j < ceil(L_s / B).
+// of the workspace pools receives the widened block block_tables[s][j], for j < ceil(L_s / B):
+// K in the query's type (kBf16), V in f16.
 // Each thread reads 8 bytes and writes the 16-byte vector they widen to, so a warp's loads and
 // stores each cover one contiguous run (256 and 512 bytes).
 template <bool kBf16>
@@ -73,7 +65,7 @@ __global__ void __launch_bounds__(kWidenThreads)
 widen_blocks_kernel(const uint2* __restrict__ k_pool, const uint2* __restrict__ v_pool, uint4* __restrict__ wk,
                     uint4* __restrict__ wv, int32_t* __restrict__ wtab, const int32_t* __restrict__ tables,
                     const int32_t* __restrict__ lens, int num_seqs, int maxb, long long units_per_block,
-                    int block_size, int num_blocks, float v_scale, uint32_t* err) {
+                    int block_size, int num_blocks, uint32_t* err) {
     pdl_trigger();
     pdl_wait();   // the pool may still be written by the previous kernel (the chunk's scatter)
     const long long total = static_cast<long long>(num_seqs) * maxb * units_per_block;
@@ -113,8 +105,8 @@ widen_blocks_kernel(const uint2* __restrict__ k_pool, const uint2* __restrict__ 
 #pragma unroll
         for (int u = 0; u < kWidenUnroll; ++u)
             if (src[u] >= 0) {
-                wk[base + u * stride] = widen8<kBf16, false>(kx[u], 1.f);
-                wv[base + u * stride] = widen8<kBf16, true>(vx[u], v_scale);
+                wk[base + u * stride] = widen8<kBf16>(kx[u]);
+                wv[base + u * stride] = widen8<false>(vx[u]);
             }
     }
 }
@@ -141,27 +133,35 @@ extern "C" pkv_status pkv_paged_attn_prefill_fp8(void* out, const void* q, pkv_d
                                                  float scale, void* workspace, size_t workspace_bytes,
                                                  uint32_t* device_error, void* stream) {
     using namespace pkv;
-    // the same checks as pkv_paged_attn_prefill, before anything is launched
-    if (num_seqs < 0 || num_tokens < 0 || max_query_len < 0 || num_heads <= 0 || num_kv_heads <= 0 ||
-        num_blocks <= 0 || max_blocks_per_seq <= 0 || !(scale > 0.f) || !std::isfinite(scale) ||
-        !(k_scale > 0.f) || !std::isfinite(k_scale) || !(v_scale > 0.f) || !std::isfinite(v_scale))
+    PrefillLaunch p{};
+    p.out = out;
+    p.q = q;
+    p.bf16 = q_dtype == PKV_BF16;
+    p.v_f16 = true;
+    p.k_pool = k_pool;
+    p.v_pool = v_pool;
+    p.k_tables = block_tables;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.context_lens = context_lens;
+    p.query_start = query_start;
+    p.max_query_len = max_query_len;
+    p.num_seqs = num_seqs;
+    p.num_tokens = num_tokens;
+    p.num_heads = num_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.head_dim = head_dim;
+    p.block_size = block_size;
+    p.num_blocks = num_blocks;
+    p.scale = scale * k_scale;   // K is widened exactly; its scale joins the softmax scale
+    p.v_mult_all = v_scale;      // V too; its scale multiplies the output rows
+    p.err = device_error;
+    p.stream = static_cast<cudaStream_t>(stream);
+    // the checks of pkv_paged_attn_prefill, the scales first, before anything is launched
+    if (!(scale > 0.f) || !std::isfinite(scale) || !(k_scale > 0.f) || !std::isfinite(k_scale) ||
+        !(v_scale > 0.f) || !std::isfinite(v_scale) || !(p.scale > 0.f) || !std::isfinite(p.scale))
         return PKV_ERR_INVALID_ARG;
-    if (num_heads % num_kv_heads != 0) return PKV_ERR_INVALID_ARG;
-    if (q_dtype != PKV_F16 && q_dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
-    const int G = num_heads / num_kv_heads;
-    if ((head_dim != 64 && head_dim != 128) || (block_size != 16 && block_size != 32) ||
-        (G != 1 && G != 2 && G != 4 && G != 8 && G != 16))
-        return PKV_ERR_UNSUPPORTED;
-    const float folded = scale * k_scale;
-    if (!(folded > 0.f) || !std::isfinite(folded)) return PKV_ERR_INVALID_ARG;
-    if (num_seqs == 0 || num_tokens == 0 || max_query_len == 0) return PKV_OK;
-    if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens || !query_start) return PKV_ERR_INVALID_ARG;
-    if (!aligned16(out) || !aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) ||
-        (reinterpret_cast<uintptr_t>(block_tables) & 3) || (reinterpret_cast<uintptr_t>(context_lens) & 3) ||
-        (reinterpret_cast<uintptr_t>(query_start) & 3) || (reinterpret_cast<uintptr_t>(device_error) & 3))
-        return PKV_ERR_ALIGNMENT;
-    if (num_seqs > 65535 || static_cast<long long>(num_seqs) * max_blocks_per_seq > 0x7fffffffLL)
-        return PKV_ERR_INVALID_ARG;
+    const pkv_status chk = prefill_check(p, q_dtype == PKV_F16 || q_dtype == PKV_BF16);
+    if (chk != PKV_OK || num_seqs == 0 || num_tokens == 0 || max_query_len == 0) return chk;
     const size_t need = pkv_prefill_fp8_workspace_bytes(num_seqs, max_blocks_per_seq, num_kv_heads, head_dim,
                                                         block_size);
     if (!workspace || workspace_bytes < need) return PKV_ERR_WORKSPACE;
@@ -184,11 +184,13 @@ extern "C" pkv_status pkv_paged_attn_prefill_fp8(void* out, const void* q, pkv_d
         return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(kWidenThreads), 0, st,
                           static_cast<const uint2*>(k_pool), static_cast<const uint2*>(v_pool),
                           static_cast<uint4*>(wk), static_cast<uint4*>(wv), wtab, block_tables, context_lens, num_seqs,
-                          max_blocks_per_seq, units_per_block, block_size, num_blocks, v_scale, device_error);
+                          max_blocks_per_seq, units_per_block, block_size, num_blocks, device_error);
     };
-    const cudaError_t e = q_dtype == PKV_BF16 ? launch(widen_blocks_kernel<true>) : launch(widen_blocks_kernel<false>);
+    const cudaError_t e = p.bf16 ? launch(widen_blocks_kernel<true>) : launch(widen_blocks_kernel<false>);
     if (e != cudaSuccess) return PKV_ERR_CUDA;
-    return pkv_paged_attn_prefill(out, q, q_dtype, wk, wv, wtab, max_blocks_per_seq, context_lens, query_start,
-                                  max_query_len, num_seqs, num_tokens, num_heads, num_kv_heads, head_dim, block_size,
-                                  static_cast<int>(blocks), folded, device_error, stream);
+    p.k_pool = wk;
+    p.v_pool = wv;
+    p.k_tables = wtab;
+    p.num_blocks = static_cast<int>(blocks);
+    return prefill_launch(p);
 }

@@ -92,9 +92,11 @@ def oracle_step(w: wl.DecodeWorkload, block_tables=None, context_lens=None):
     return {"out": out, "k_pool": kp, "v_pool": vp}
 
 
-def gpu_prefill(w, dev="cuda:0", block_tables=None, context_lens=None, query_start=None, q_bits=None):
+def gpu_prefill(w, dev="cuda:0", block_tables=None, context_lens=None, query_start=None, q_bits=None,
+                workspace="auto"):
     """Build the cache (setup scatter), scatter the chunk's K/V, run the prefill; returns
-    (out tensor, device error word, k pool, v pool)."""
+    (out tensor, device error word, k pool, v pool).  workspace: "auto" (bf16: V narrowed to f16
+    in a workspace) or None (bf16: the two-part weights, no workspace)."""
     from paged_kv_cache_324_b200 import binding as B
     dev = torch.device(dev)
     kp = to_dev_bits(w.initial_pool("k"), w.dtype, dev)
@@ -112,7 +114,7 @@ def gpu_prefill(w, dev="cuda:0", block_tables=None, context_lens=None, query_sta
     B.paged_attn_prefill(out, q, kp, vp, torch.from_numpy(np.ascontiguousarray(bt)).to(dev),
                          torch.from_numpy(np.ascontiguousarray(cl)).to(dev),
                          torch.from_numpy(np.ascontiguousarray(qs)).to(dev), float(w.scale),
-                         max_query_len=w.max_query_len, device_error=err)
+                         max_query_len=w.max_query_len, workspace=workspace, device_error=err)
     torch.cuda.synchronize()
     return out, int(err.item()), kp, vp
 

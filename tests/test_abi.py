@@ -7,6 +7,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "pagedkv.h")
@@ -121,9 +122,13 @@ def _prefill(lib, **over):
     P = ctypes.c_void_p
     args = dict(out=P(16), q=P(16), dtype=1, k_pool=P(16), v_pool=P(16), block_tables=P(16), max_blocks=4,
                 context_lens=P(16), query_start=P(16), max_q=64, S=2, T=100, H=8, Hkv=2, D=128, B=16, NB=10,
-                scale=0.1, err=None, stream=None)
+                scale=0.1, ws=None, ws_bytes=0, err=None, stream=None)
     args.update(over)
-    return lib.pkv_paged_attn_prefill(*args.values())
+    f = lib.pkv_paged_attn_prefill
+    P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    f.argtypes = [P, P, I, P, P, P, I, P, P, I, I, I, I, I, I, I, I, F, P, Z, P, P]
+    f.restype = I
+    return f(*args.values())
 
 
 @pytest.mark.parametrize("over,status", [
@@ -133,6 +138,8 @@ def _prefill(lib, **over):
     (dict(q=None), 1), (dict(query_start=None), 1), (dict(out=ctypes.c_void_p(24)), 5),
     (dict(query_start=ctypes.c_void_p(18)), 5),
     (dict(T=0), 0), (dict(S=0), 0), (dict(max_q=0), 0),
+    # bf16 with a workspace: too small, or not 256-byte aligned (the workspace path's own checks)
+    (dict(ws=ctypes.c_void_p(256), ws_bytes=1024), 3), (dict(ws=ctypes.c_void_p(272), ws_bytes=1 << 20), 5),
 ])
 def test_prefill_rejects_bad_arguments(lib, over, status):
     """Host-side checks of pkv_paged_attn_prefill (group size 3 and 32, FP8, odd sizes, a
@@ -171,6 +178,21 @@ def test_workspace_size_rules(lib):
     assert B.decode_partition_size(16, 8, 128, "e4m3", 16, 32768, 0) == 2048
     # ... shrunk when there are few work units, never below 4 blocks
     assert B.decode_partition_size(4, 8, 64, "f16", 16, 256, 0) == 64
+
+
+def test_prefill_workspace_size(lib):
+    """The bf16 prefill's narrowing workspace: the f16 V pool (num_seqs x max_blocks_per_seq blocks),
+    its table, one factor per (sequence, KV head) and one partial maximum per (sequence, KV head,
+    16 table slots), each part rounded up to 256 bytes; none for f16 or E4M3."""
+    from paged_kv_cache_324_b200 import binding as B
+    assert B.prefill_workspace_bytes("f16", 2, 4, 2, 128, 16) == 0
+    assert B.prefill_workspace_bytes("e4m3", 2, 4, 2, 128, 16) == 0
+    assert B.prefill_workspace_bytes("bf16", 2, 4, 2, 128, 16) == 8 * 2 * 16 * 128 * 2 + 3 * 256
+    S, maxb, Hkv, D, Bs = 16, 320, 8, 128, 16
+    pool = S * maxb * Hkv * Bs * D * 2
+    parts = -(-(S * Hkv * 20 * 4) // 256) * 256
+    assert B.prefill_workspace_bytes(torch.bfloat16, S, maxb, Hkv, D, Bs) == pool + S * maxb * 4 + 512 + parts
+    assert B.prefill_workspace_bytes("bf16", 0, 4, 2, 128, 16) == 0
 
 
 def test_stream_read_checks_its_buffer(lib):

@@ -95,9 +95,13 @@ def test_prefill_writes_nothing_outside_its_buffers(fp8):
         guards.append((ws, "workspace"))
         B.paged_attn_prefill_fp8(out.t, q, kp.t, vp.t, tables, lens, qs, float(w.scale), ks, vs,
                                  max_query_len=w.max_query_len, workspace=ws.t, device_error=err.t)
-    else:
+    else:   # bf16: V is narrowed to f16 in the workspace first
+        need = B.prefill_workspace_bytes(w.dtype, w.num_seqs, w.max_blocks, w.num_kv_heads, w.head_dim, w.block_size)
+        assert need > 0
+        ws = H.Guarded((need,), torch.uint8, dev)
+        guards.append((ws, "workspace"))
         B.paged_attn_prefill(out.t, q, kp.t, vp.t, tables, lens, qs, float(w.scale), max_query_len=w.max_query_len,
-                             device_error=err.t)
+                             workspace=ws.t, device_error=err.t)
     torch.cuda.synchronize()
     assert int(err.t.item()) == 0
     for g, what in guards:

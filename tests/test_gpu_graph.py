@@ -96,11 +96,13 @@ def test_prefill_graph_replays_with_new_inputs():
     qs = torch.from_numpy(w.query_start).to(dev)
     out = torch.empty_like(q)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws = torch.empty(B.prefill_workspace_bytes("bf16", w.num_seqs, w.max_blocks, Hkv, D, w.block_size),
+                     dtype=torch.uint8, device=dev)
 
     def step():
         B.reshape_and_cache(kn, vn, kp, vp, slots, device_error=err)
         B.paged_attn_prefill(out, q, kp, vp, tables, lens, qs, float(w.scale), max_query_len=w.max_query_len,
-                             device_error=err)
+                             workspace=ws, device_error=err)
 
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())

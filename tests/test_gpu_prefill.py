@@ -54,15 +54,55 @@ def make_case(name):
     return wl.chunked_prefill(name, 100 + len(name), Hq, Hkv, D, Bs, NB, dt, prior, chunks)
 
 
+@pytest.mark.parametrize("ws", ["auto", None], ids=["workspace", "no_workspace"])
 @pytest.mark.parametrize("name", list(CASES))
-def test_prefill_matches_oracle(name):
+def test_prefill_matches_oracle(name, ws):
+    """bf16 runs both ways: V narrowed to f16 in a workspace, and the two-part weights without one."""
     w = make_case(name)
-    out, err, _, _ = H.gpu_prefill(w)
+    if ws is None and w.dtype != "bf16":
+        pytest.skip("f16 takes no workspace")
+    out, err, _, _ = H.gpu_prefill(w, workspace=ws)
     assert err == 0
     kp, vp = H.oracle_prefill_pools(w)
     ref = oracle_out(w, kp, vp)
     ok, rep = prefill_close(H.out_f64(out), ref, w.dtype)
     assert ok, (name, rep)
+
+
+def scaled_v(w, factor):
+    """The workload with every scattered V row of KV head h multiplied by factor[h] (bf16 bits)."""
+    import dataclasses
+
+    def scale(op):
+        v = H.out_f64(H.to_dev_bits(op.v, w.dtype, "cpu")) * np.asarray(factor, np.float64)[None, :, None]
+        bits = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        return dataclasses.replace(op, v=bits.reshape(op.v.shape))
+
+    return dataclasses.replace(w, setup=[scale(op) for op in w.setup], step_scatter=scale(w.step_scatter))
+
+
+@pytest.mark.parametrize("ws", ["auto", None], ids=["workspace", "no_workspace"])
+def test_bf16_v_far_outside_the_f16_range(ws):
+    """KV heads whose V values lie far above the f16 range (x 3e5 and x 2^60) or far below it
+    (x 1e-6 and x 2^-100): narrowing scales each (sequence, KV head) by its own power of two, so
+    every head keeps the accuracy of a unit-scale one.  Checked per head against the oracle,
+    relative to the head's largest |v| (the 2e-3 bound of a unit-scale V)."""
+    factors = [3e5, 1e-6, 2.0 ** 60, 2.0 ** -100, 1.0, 7.0, 0.01, 1.0]
+    w = scaled_v(wl.chunked_prefill("vrange", 12, 16, 8, 128, 16, 256, "bf16", [300, 40, 0], [200, 150, 90]),
+                 factors)
+    out, err, _, _ = H.gpu_prefill(w, workspace=ws)
+    assert err == 0
+    o = H.out_f64(out)
+    assert np.isfinite(o).all()
+    kp, vp = H.oracle_prefill_pools(w)
+    ref = oracle_out(w, kp, vp)
+    G = w.num_heads // w.num_kv_heads
+    ops = [op for op in list(w.setup) + [w.step_scatter] if op.slots.size]
+    vmax = [max(np.abs(H.out_f64(H.to_dev_bits(op.v, "bf16", "cpu"))[:, h]).max() for op in ops)
+            for h in range(w.num_kv_heads)]
+    for h in range(w.num_kv_heads):
+        d = np.abs(o[:, h * G:(h + 1) * G] - ref[:, h * G:(h + 1) * G]).max()
+        assert d <= 4e-3 * vmax[h], (h, factors[h], d, vmax[h])
 
 
 def test_wide_logits_move_the_running_maximum():
