@@ -63,14 +63,21 @@ NCU_TRAFFIC = {
 }
 
 
-# the same for the prefill kernel (sha256 prefix of prefill.cu), on the prefill workload
-PREFILL_TRAFFIC = {"bytes_per_launch": 569_112_320, "kernel_sha": "341da0a10c7c8cc7",
-                   "capture": "ncu, prefill workload, paged_prefill_kernel"}
+# the same for the prefill calls (every kernel of one call, summed), keyed on the sha256 prefix of
+# prefill.cu followed by prefill_fp8.cu, on the prefill workload
+PREFILL_TRAFFIC = {
+    "prefill": {"bytes_per_launch": 823_535_104, "kernel_sha": "e7cc85da49e0ea19",
+                "capture": "ncu, prefill workload: v_absmax_kernel + v_narrow_kernel + paged_prefill_kernel"},
+    "prefill_fp8": {"bytes_per_launch": 819_885_824, "kernel_sha": "e7cc85da49e0ea19",
+                    "capture": "ncu, prefill workload over an E4M3 cache: widen_blocks_kernel + paged_prefill_kernel"},
+}
 
 
 def prefill_source_sha() -> str:
-    p = os.path.join(ROOT, "paged_kv_cache_324_b200", "csrc", "prefill.cu")
-    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+    h = hashlib.sha256()
+    for f in ("prefill.cu", "prefill_fp8.cu"):
+        h.update(open(os.path.join(ROOT, "paged_kv_cache_324_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
 
 
 def decode_source_sha() -> str:
@@ -425,8 +432,8 @@ def run_prefill(args, rank, world, local_rank):
                      "achieved": round(achieved, 2),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "frac_of_sustained": round(achieved / peak_sus, 4),
-                     "traffic": (PREFILL_TRAFFIC["bytes_per_launch"]
-                                 if PREFILL_TRAFFIC["kernel_sha"] == prefill_source_sha() and not kv_fp8 else None),
+                     "traffic": (PREFILL_TRAFFIC[args.config]["bytes_per_launch"]
+                                 if PREFILL_TRAFFIC[args.config]["kernel_sha"] == prefill_source_sha() else None),
                      "flops_per_launch": flops,
                      "flops_counted": "4 * head_dim * num_heads * causal (query, key) pairs",
                      "peak_kind": f"{kind} (cuBLAS bf16, burst; sustained {peak_sus})"},

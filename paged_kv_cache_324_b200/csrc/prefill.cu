@@ -823,7 +823,24 @@ pkv_status dispatch_mode(bool bf16, bool v_f16, const PrefillArgs& a, const CUte
 
 constexpr int kNarrowThreads = 256;
 constexpr int kNarrowChunk = 16;       // table slots per CTA of the two passes
-constexpr int kNarrowUnroll = 4;
+
+constexpr int kNarrowUnroll = 8;       // 16-byte loads each thread has in flight
+
+// The chunk's block ids (slots j0 .. j0 + kNarrowChunk - 1) into shared memory, -1 for slots past
+// the sequence's last reachable block (jn) and for ids outside the pool (reported when `err`).
+__device__ __forceinline__ void load_chunk_ids(int* pids, const int32_t* __restrict__ trow, int j0, int jn,
+                                               int num_blocks, uint32_t* err) {
+    if (threadIdx.x < kNarrowChunk) {
+        const int j = j0 + static_cast<int>(threadIdx.x);
+        int pid = j < jn ? __ldg(trow + j) : -1;
+        if (j < jn && (pid < 0 || pid >= num_blocks)) {
+            if (err) raise_error(err, PKV_DEVERR_BLOCK_ID);
+            pid = -1;
+        }
+        pids[threadIdx.x] = pid;
+    }
+    __syncthreads();
+}
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -875,6 +892,8 @@ v_absmax_kernel(const uint4* __restrict__ v_pool, const int32_t* __restrict__ ta
     const long long cap = static_cast<long long>(maxb) * BS;
     const int nb = L <= 0 ? 0 : static_cast<int>((min(static_cast<long long>(L), cap) + BS - 1) / BS);
     const int j0 = chunk * kNarrowChunk, j1 = min(nb, j0 + kNarrowChunk);
+    __shared__ int pids[kNarrowChunk];
+    load_chunk_ids(pids, tables + static_cast<size_t>(s) * maxb, j0, j1, num_blocks, nullptr);
     uint32_t m = 0;
     for (int u0 = threadIdx.x; u0 < (j1 - j0) * kRun; u0 += kNarrowThreads * kNarrowUnroll) {
         uint4 x[kNarrowUnroll];
@@ -882,11 +901,11 @@ v_absmax_kernel(const uint4* __restrict__ v_pool, const int32_t* __restrict__ ta
 #pragma unroll
         for (int k = 0; k < kNarrowUnroll; ++k) {
             const int u = u0 + k * kNarrowThreads;
-            const int j = j0 + u / kRun, e = u % kRun;
+            const int jj = u / kRun, e = u % kRun;
             valid[k] = false;
             if (u < (j1 - j0) * kRun) {
-                const int pid = __ldg(tables + static_cast<size_t>(s) * maxb + j);
-                valid[k] = pid >= 0 && pid < num_blocks && j * BS + e / (D / 8) < L;
+                const int pid = pids[jj];
+                valid[k] = pid >= 0 && (j0 + jj) * BS + e / (D / 8) < L;
                 if (valid[k])
                     x[k] = __ldg(v_pool + ((static_cast<size_t>(pid) * num_kv_heads + h) * kRun + e));
             }
@@ -947,17 +966,15 @@ v_narrow_kernel(const uint4* __restrict__ v_pool, const int32_t* __restrict__ ta
     const long long cap = static_cast<long long>(maxb) * BS;
     const int nb = L <= 0 ? 0 : static_cast<int>((min(static_cast<long long>(L), cap) + BS - 1) / BS);
     const int j0 = chunk * kNarrowChunk, j1 = min(maxb, j0 + kNarrowChunk);
-    if (h == 0)
-        for (int j = j0 + static_cast<int>(threadIdx.x); j < j1; j += kNarrowThreads) {
-            const int pid = j < nb ? __ldg(tables + static_cast<size_t>(s) * maxb + j) : -1;
-            const bool bad = j < nb && (pid < 0 || pid >= num_blocks);
-            if (bad) raise_error(err, PKV_DEVERR_BLOCK_ID);
-            wtab[static_cast<size_t>(s) * maxb + j] = (j < nb && !bad) ? static_cast<int32_t>(s * maxb + j) : -1;
-        }
     const int jn = min(nb, j1);
+    __shared__ int pids[kNarrowChunk];
+    load_chunk_ids(pids, tables + static_cast<size_t>(s) * maxb, j0, jn, num_blocks, h == 0 ? err : nullptr);
+    if (h == 0 && static_cast<int>(threadIdx.x) < j1 - j0)
+        wtab[static_cast<size_t>(s) * maxb + j0 + threadIdx.x] =
+            pids[threadIdx.x] >= 0 ? static_cast<int32_t>(s * maxb + j0 + threadIdx.x) : -1;
     for (int u0 = threadIdx.x; u0 < (jn - j0) * kRun; u0 += kNarrowThreads * kNarrowUnroll) {
         uint4 x[kNarrowUnroll];
-        int dst[kNarrowUnroll];                      // -1: nothing to write; else the unit's slot j (and e)
+        int dst[kNarrowUnroll];                      // -1: nothing to write; else the unit's index in the chunk
         bool live[kNarrowUnroll];
 #pragma unroll
         for (int k = 0; k < kNarrowUnroll; ++k) {
@@ -965,11 +982,11 @@ v_narrow_kernel(const uint4* __restrict__ v_pool, const int32_t* __restrict__ ta
             dst[k] = -1;
             live[k] = false;
             if (u < (jn - j0) * kRun) {
-                const int j = j0 + u / kRun, e = u % kRun;
-                const int pid = __ldg(tables + static_cast<size_t>(s) * maxb + j);
-                if (pid >= 0 && pid < num_blocks) {
+                const int jj = u / kRun, e = u % kRun;
+                const int pid = pids[jj];
+                if (pid >= 0) {
                     dst[k] = u;
-                    live[k] = j * BS + e / (D / 8) < L;
+                    live[k] = (j0 + jj) * BS + e / (D / 8) < L;
                     if (live[k]) x[k] = __ldg(v_pool + ((static_cast<size_t>(pid) * num_kv_heads + h) * kRun + e));
                 }
             }
