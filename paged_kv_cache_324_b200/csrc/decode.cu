@@ -61,6 +61,13 @@
 namespace pkv {
 namespace {
 
+// 2^x on the exponential unit (PTX ex2.approx.ftz: results below 2^-126 flush to zero)
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Occupancy plan: the kernel streams HBM through TMA, so what keeps the memory
 // system busy is the number of consumer warps ready to drain the ring.  With
 // query groups of up to 8 heads a CTA fits in 96 registers per thread and a
@@ -592,14 +599,14 @@ paged_decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap
                     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
                     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
                     const float mnew = fmaxf(m_run[nh][hc], mx);
-                    alpha[nh][hc] = exp2f(m_run[nh][hc] - mnew);
+                    alpha[nh][hc] = ex2(m_run[nh][hc] - mnew);
                     rescale |= alpha[nh][hc] != 1.f;
                     m_run[nh][hc] = mnew;
                     float sum = 0.f;
 #pragma unroll
                     for (int mt = 0; mt < Gm::kMtTok; ++mt) {
-                        sc[mt][nh][hc] = exp2f(sc[mt][nh][hc] - mnew);
-                        sc[mt][nh][hc + 2] = exp2f(sc[mt][nh][hc + 2] - mnew);
+                        sc[mt][nh][hc] = ex2(sc[mt][nh][hc] - mnew);
+                        sc[mt][nh][hc + 2] = ex2(sc[mt][nh][hc + 2] - mnew);
                         sum += sc[mt][nh][hc] + sc[mt][nh][hc + 2];
                     }
                     l_run[nh][hc] = l_run[nh][hc] * alpha[nh][hc] + sum;
