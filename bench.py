@@ -54,11 +54,11 @@ FALLBACK_HBM_GBS = 6650.0
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by workload, valid only
 # for the decode kernel source it was measured on (sha256 prefix of decode.cu).
 NCU_TRAFFIC = {
-    "opt13b": {"bytes_per_launch": 1_313_395_456, "kernel_sha": "980738653df370e4",
+    "opt13b": {"bytes_per_launch": 1_313_689_344, "kernel_sha": "1e2ef54f9309f55c",
                "capture": "ncu, opt13b_compact (the same sequences, pool cut to the blocks in use)"},
-    "gqa": {"bytes_per_launch": 1_222_007_808, "kernel_sha": "980738653df370e4",
+    "gqa": {"bytes_per_launch": 1_222_165_760, "kernel_sha": "1e2ef54f9309f55c",
             "capture": "ncu, gqa_compact (the same sequences, pool cut to the blocks in use)"},
-    "fp8": {"bytes_per_launch": 1_116_351_744, "kernel_sha": "980738653df370e4",
+    "fp8": {"bytes_per_launch": 1_116_366_848, "kernel_sha": "1e2ef54f9309f55c",
             "capture": "ncu, fp8_compact (the same sequences, 512-token partitions)"},
 }
 
