@@ -449,8 +449,17 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
         mbar_init(drain, 1);
         flags.abort = 0;
         flags.bad = 0;
-        flags.vmul = a.v_mult_all * (a.v_mult ? __ldg(a.v_mult + static_cast<size_t>(s) * gridDim.y + kvh) : 1.f);
         mbar_fence_init();
+        // both Q tiles are requested at once, so that their load overlaps the TMEM allocation and
+        // the CTA-wide barrier below
+        tma_prefetch_desc(&qmap);
+        mbar_arrive_expect_tx(bar_q, kTiles * Gm::kTile);
+#pragma unroll
+        for (int t = 0; t < kTiles; ++t)
+#pragma unroll
+            for (int c = 0; c < Gm::kChunks; ++c)
+                tma_load_3d(sQ + t * Gm::kTile + c * kChunkBytes, &qmap, bar_q, c * 64, kvh * G, q0 + t0 + t * TQ);
+        flags.vmul = a.v_mult_all * (a.v_mult ? __ldg(a.v_mult + static_cast<size_t>(s) * gridDim.y + kvh) : 1.f);
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -470,15 +479,8 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
         const int nst = is_k ? kKStages : kVStages;
         const uint64_t pol = l2_policy_evict_last();      // K/V tiles are read again by the other query tiles
         if (is_k && lane == 0) {
-            tma_prefetch_desc(&qmap);
             tma_prefetch_desc(&kmap);
             tma_prefetch_desc(&vmap);
-            mbar_arrive_expect_tx(bar_q, kTiles * Gm::kTile);
-#pragma unroll
-            for (int t = 0; t < kTiles; ++t)
-#pragma unroll
-                for (int c = 0; c < Gm::kChunks; ++c)
-                    tma_load_3d(sQ + t * Gm::kTile + c * kChunkBytes, &qmap, bar_q, c * 64, kvh * G, q0 + t0 + t * TQ);
         }
         const CUtensorMap* map = is_k ? &kmap : &vmap;
         const uint32_t ring = is_k ? sK : sV;
@@ -759,7 +761,9 @@ paged_prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qm
             }
         if (stores) {
             asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-            asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");   // writes done before the CTA exits
+            // the shared memory must stay until the copies have read it; their writes to global memory
+            // complete with the grid
+            asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
         }
     }
     if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
