@@ -312,8 +312,10 @@ pkv_status pkv_paged_attn_decode_static_ws(void* out, const void* q, pkv_dtype q
  *     NaN kept), and 2^e multiplies the head's output rows;
  *   - without one, P enters as a bf16 high part plus a bf16 low part
  *     (P - bf16(P)) against the bf16 V: two products, slower, no memory.
- * Returns PKV_ERR_WORKSPACE if a non-null workspace is smaller than
- * pkv_prefill_workspace_bytes().
+ * For BF16, returns PKV_ERR_WORKSPACE if a non-null workspace is smaller
+ * than pkv_prefill_workspace_bytes() and PKV_ERR_ALIGNMENT if it is not
+ * 256-byte aligned, launching nothing.  pkv_prefill_workspace_bytes() is 0
+ * for F16 (and any dtype but BF16) and for non-positive sizes.
  */
 size_t pkv_prefill_workspace_bytes(pkv_dtype dtype, int num_seqs, int max_blocks_per_seq, int num_kv_heads,
                                    int head_dim, int block_size);
