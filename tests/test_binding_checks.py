@@ -63,6 +63,26 @@ def test_prefill_rejects_short_tables_and_bad_offsets():
                                  qs, 0.1, 1.0, 1.0, max_query_len=5)
 
 
+def test_prefill_workspace_choice():
+    """workspace is a tensor, "auto" (a bf16 call gets one of prefill_workspace_bytes) or None (the
+    two-part weights); anything else is refused before a pointer is taken."""
+    T = 10
+    q = torch.zeros((T, H, D), dtype=torch.bfloat16)
+    pool = torch.zeros((NB, Hkv, Bs, D), dtype=torch.bfloat16)
+    lens = torch.tensor([5, 5], dtype=torch.int32)
+    qs = torch.tensor([0, 5, 10], dtype=torch.int32)
+    tables = torch.zeros((2, 2), dtype=torch.int32)
+    with pytest.raises(ValueError, match="workspace must be"):
+        B.paged_attn_prefill(torch.empty_like(q), q, pool, pool, tables, lens, qs, 0.1, max_query_len=5,
+                             workspace="none")
+    for ws in ("auto", None):   # well-formed: passes the checks, then needs GPU tensors
+        with pytest.raises(ValueError, match="CUDA tensor"):
+            B.paged_attn_prefill(torch.empty_like(q), q, pool, pool, tables, lens, qs, 0.1, max_query_len=5,
+                                 workspace=ws)
+    assert B.prefill_workspace_bytes(torch.bfloat16, 2, 2, Hkv, D, Bs) > 0
+    assert B.prefill_workspace_bytes(torch.float16, 2, 2, Hkv, D, Bs) == 0
+
+
 def test_shared_prefix_rejects_inconsistent_arguments():
     out, q, kp, vp, tables, lens, scale = decode_args()
     i32 = torch.zeros(S, dtype=torch.int32)
