@@ -133,6 +133,25 @@ def test_bad_block_id_gives_nan_rows_and_flag():
     assert ok, rep
 
 
+@pytest.mark.parametrize("ws", ["auto", None], ids=["workspace", "no_workspace"])
+def test_bf16_bad_block_id_gives_nan_rows_and_flag(ws):
+    """A bad id in a bf16 call: with a workspace the narrowing passes skip that block and leave -1
+    in the workspace table (NaN rows for the tiles that need it, PKV_DEVERR_BLOCK_ID), without one
+    the prefill kernel finds it; the other sequence is unaffected either way."""
+    w = wl.chunked_prefill("badbf", 18, 8, 2, 128, 16, 128, "bf16", [40, 100], [30, 60])
+    tab = w.block_tables.copy()
+    tab[1, 3] = -7                               # a block sequence 1 needs
+    out, err, _, _ = H.gpu_prefill(w, block_tables=tab, workspace=ws)
+    assert err & 0x1
+    o = H.out_f64(out)
+    r0, r1 = int(w.query_start[1]), int(w.query_start[2])
+    assert np.isnan(o[r0:r1]).any()
+    kp, vp = H.oracle_prefill_pools(w)
+    ref = oracle_out(w, kp, vp)
+    ok, rep = prefill_close(o[:r0], ref[:r0], "bf16")
+    assert ok, rep
+
+
 def test_chunk_longer_than_context_is_flagged():
     w = wl.chunked_prefill("ctx", 9, 4, 4, 128, 16, 64, "bf16", [20, 5], [10, 12])
     lens = w.context_lens.copy()
