@@ -66,9 +66,9 @@ NCU_TRAFFIC = {
 # the same for the prefill calls (every kernel of one call, summed), keyed on the sha256 prefix of
 # prefill.cu followed by prefill_fp8.cu, on the prefill workload
 PREFILL_TRAFFIC = {
-    "prefill": {"bytes_per_launch": 823_833_856, "kernel_sha": "3adbb7f1d82660ad",
+    "prefill": {"bytes_per_launch": 823_833_856, "kernel_sha": "bcbb51e41e176572",
                 "capture": "ncu, prefill workload: v_absmax_kernel + v_narrow_kernel + paged_prefill_kernel"},
-    "prefill_fp8": {"bytes_per_launch": 820_305_408, "kernel_sha": "3adbb7f1d82660ad",
+    "prefill_fp8": {"bytes_per_launch": 820_305_408, "kernel_sha": "bcbb51e41e176572",
                     "capture": "ncu, prefill workload over an E4M3 cache: widen_blocks_kernel + paged_prefill_kernel"},
 }
 

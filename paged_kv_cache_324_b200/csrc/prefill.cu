@@ -827,7 +827,6 @@ pkv_status dispatch_mode(bool bf16, bool v_f16, const PrefillArgs& a, const CUte
 
 constexpr int kNarrowThreads = 256;
 constexpr int kNarrowChunk = 16;       // table slots per CTA of the two passes
-
 constexpr int kNarrowUnroll = 8;       // 16-byte loads each thread has in flight
 
 // The chunk's block ids (slots j0 .. j0 + kNarrowChunk - 1) into shared memory, -1 for slots past
@@ -867,7 +866,8 @@ NarrowLayout narrow_layout(int num_seqs, int maxb, int num_kv_heads, int head_di
 }
 
 // The largest finite magnitude among 8 bf16 values (as the bits of |v|; bf16 magnitudes order as
-// integers), those at key positions >= limit excluded.
+// integers); 0 for a unit that does not count (its key position is past the context, or its block
+// id is bad).
 __device__ __forceinline__ uint32_t absmax8(const uint4& x, bool valid) {
     if (!valid) return 0;
     const uint32_t w[4] = {x.x, x.y, x.z, x.w};
